@@ -1,0 +1,185 @@
+"""Block manager of the paged KV cache, restated in plain Python (oracle side).
+
+What the pages fix:
+  * The cache is a pool of equal fixed-size blocks, each holding the keys and
+    values of 16 tokens, allocated once up front ("PagedAttention: The vLLM
+    Paper", "The Core Idea" figure and "Implementation Essentials").
+  * Each sequence has a block table mapping its logical blocks to physical
+    ones; blocks are taken on demand as tokens arrive and only the last block
+    of a sequence can be partly filled ("PagedAttention and Continuous
+    Batching", "Pages, from operating systems"; "PagedAttention: The vLLM
+    Paper", "The design yields three immediate wins", item 1).
+  * Blocks are reference counted so sequences can share them; a shared block
+    is copied only when one sequence has to write into it, as with fork and
+    copy-on-write in an operating system ("Pages, from operating systems";
+    "The OS paging analogy" table; "Implementation Essentials").
+  * Finished sequences return their blocks to the pool for any request to use
+    ("The Core Idea" figure caption).
+
+Readings where the pages are silent (the CUDA-side library follows the same
+rules so that tables can be compared bit for bit):
+  * The free list is a stack. ``initial_free_order[0]`` is handed out first;
+    freed blocks go on top and are reused first.
+  * ``free_seq`` releases a sequence's blocks from its last logical block to
+    its first.
+  * Copy-on-write happens when an append writes into a partly filled last
+    block whose refcount is above one: the appending sequence gets a fresh
+    block, a ``(old, new)`` copy pair is emitted and the old block's count
+    drops by one. A sequence whose last block has refcount one writes in place.
+  * Every call is all-or-nothing: when the pool cannot cover it, nothing changes.
+  * Block tables are padded with -1.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# Status codes shared in meaning with the C interface.
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_NO_FREE_BLOCKS = 2
+ERR_UNKNOWN_SEQ = 3
+ERR_SEQ_EXISTS = 6
+
+
+class BlockManagerError(Exception):
+    def __init__(self, code: int, msg: str):
+        super().__init__(msg)
+        self.code = code
+
+
+def _ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+class BlockManager:
+    def __init__(self, num_blocks: int, block_size: int, initial_free_order=None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise BlockManagerError(ERR_INVALID_ARG, "num_blocks and block_size must be positive")
+        if initial_free_order is None:
+            order = list(range(num_blocks))
+        else:
+            order = [int(b) for b in initial_free_order]
+            if sorted(order) != list(range(num_blocks)):
+                raise BlockManagerError(ERR_INVALID_ARG,
+                                        "initial_free_order must be a permutation of the pool")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        # Top of the stack is the end of the list, so order[0] is popped first.
+        self._free = list(reversed(order))
+        self._ref = [0] * num_blocks
+        self._tables: dict[int, list[int]] = {}
+        self._lens: dict[int, int] = {}
+
+    # -- queries ---------------------------------------------------------
+    def num_free(self) -> int:
+        return len(self._free)
+
+    def refcount(self, block: int) -> int:
+        if not 0 <= block < self.num_blocks:
+            raise BlockManagerError(ERR_INVALID_ARG, "block id out of range")
+        return self._ref[block]
+
+    def seq_len(self, seq_id: int) -> int:
+        self._need(seq_id)
+        return self._lens[seq_id]
+
+    def table(self, seq_id: int) -> list[int]:
+        self._need(seq_id)
+        return list(self._tables[seq_id])
+
+    def seq_ids(self):
+        return list(self._tables)
+
+    def free_list(self) -> list[int]:
+        """Free blocks in the order they would be handed out."""
+        return list(reversed(self._free))
+
+    # -- helpers ---------------------------------------------------------
+    def _need(self, seq_id):
+        if seq_id not in self._tables:
+            raise BlockManagerError(ERR_UNKNOWN_SEQ, f"unknown sequence {seq_id}")
+
+    def _slot(self, table, pos):
+        return table[pos // self.block_size] * self.block_size + pos % self.block_size
+
+    # -- mutations -------------------------------------------------------
+    def add_seq(self, seq_id: int, num_tokens: int) -> list[int]:
+        """Register a sequence holding ``num_tokens`` tokens; return their slots."""
+        if num_tokens < 0:
+            raise BlockManagerError(ERR_INVALID_ARG, "num_tokens must be >= 0")
+        if seq_id in self._tables:
+            raise BlockManagerError(ERR_SEQ_EXISTS, f"sequence {seq_id} exists")
+        need = _ceil_div(num_tokens, self.block_size)
+        if need > len(self._free):
+            raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
+        table = []
+        for _ in range(need):
+            b = self._free.pop()
+            self._ref[b] = 1
+            table.append(b)
+        self._tables[seq_id] = table
+        self._lens[seq_id] = num_tokens
+        return [self._slot(table, p) for p in range(num_tokens)]
+
+    def fork(self, parent: int, child: int) -> None:
+        """Child starts as a copy of the parent's table; every block is shared."""
+        self._need(parent)
+        if child in self._tables:
+            raise BlockManagerError(ERR_SEQ_EXISTS, f"sequence {child} exists")
+        table = list(self._tables[parent])
+        for b in table:
+            self._ref[b] += 1
+        self._tables[child] = table
+        self._lens[child] = self._lens[parent]
+
+    def append_slots(self, seq_id: int, n: int):
+        """Append ``n`` tokens; return ``(slots, cow_pairs)``."""
+        self._need(seq_id)
+        if n < 0:
+            raise BlockManagerError(ERR_INVALID_ARG, "n must be >= 0")
+        table = self._tables[seq_id]
+        length = self._lens[seq_id]
+        bs = self.block_size
+        new_blocks = _ceil_div(length + n, bs) - len(table)
+        cow = n > 0 and length % bs != 0 and self._ref[table[-1]] > 1
+        if new_blocks + int(cow) > len(self._free):
+            raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
+        pairs = []
+        if cow:
+            old = table[-1]
+            new = self._free.pop()
+            self._ref[old] -= 1
+            self._ref[new] = 1
+            table[-1] = new
+            pairs.append((old, new))
+        slots = []
+        for p in range(length, length + n):
+            if p % bs == 0:
+                b = self._free.pop()
+                self._ref[b] = 1
+                table.append(b)
+            slots.append(self._slot(table, p))
+        self._lens[seq_id] = length + n
+        return slots, pairs
+
+    def free_seq(self, seq_id: int) -> None:
+        self._need(seq_id)
+        for b in reversed(self._tables[seq_id]):
+            self._ref[b] -= 1
+            if self._ref[b] == 0:
+                self._free.append(b)
+        del self._tables[seq_id]
+        del self._lens[seq_id]
+
+    def block_tables(self, seq_ids, max_blocks: int) -> np.ndarray:
+        """Tables of ``seq_ids`` as int32 ``[n, max_blocks]``, padded with -1."""
+        seq_ids = list(seq_ids)
+        out = np.full((len(seq_ids), max_blocks), -1, dtype=np.int32)
+        for i, s in enumerate(seq_ids):
+            self._need(s)
+            t = self._tables[s]
+            if len(t) > max_blocks:
+                raise BlockManagerError(ERR_INVALID_ARG, "table longer than max_blocks")
+            out[i, :len(t)] = t
+        return out
