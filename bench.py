@@ -1,0 +1,474 @@
+"""Benchmark of the paged-decode step on B200.
+
+One step = the whole decode-step path of one attention layer for a batch:
+copy-on-write block copies (when the workload has any), writing each new
+token's K/V into its slot, and paged decode attention with the split-KV merge.
+The default workload is the 7B-like MHA batch (64 sequences, 32 heads,
+head_dim 128, fp16, contexts U[128, 2048], 16384-block pool, one new token
+per sequence).
+
+Metric: KV-read GB/s (algorithmic bytes of the step / device time of the
+step; % of measured HBM peak alongside) and decode tokens/s.
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events
+on the launching stream, with an L2 flush (a 256 MiB write, more than the
+126 MB L2) between steps outside the events; a barrier + synchronize on both
+sides of the timed region; max over ranks. The decode kernel alone is timed
+the same way for the roofline. ``e2e`` repeats the step through the same
+C interface fed from pinned host buffers: every step copies its inputs
+host -> device and its output device -> host inside the timed region.
+
+Multi-GPU (torchrun, one process per GPU): the decode step has no exchange
+between GPUs, so each rank runs an independent replica with its own pool and
+its own seeded batch (weak scaling); timing is the max over ranks.
+
+``--impl reference`` times the CPU oracle (float64 NumPy) on a bounded sample
+of the same workload on the host cores; only rank 0 does work.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode tokens/s"
+UNIT = "GB/s"
+DEFAULT_WORKLOAD = "mha_7b_fp16"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------
+# byte accounting
+# --------------------------------------------------------------------------
+
+def decode_bytes(wl) -> int:
+    """Algorithmic bytes of one paged-decode call: each token's K and V once per KV
+    head, q read and out written once, the used block-table entries and the
+    context lengths."""
+    ctx = wl.context_lens.astype(np.int64)
+    e = wl.elem_bytes
+    kv = int(ctx.sum()) * wl.num_kv_heads * wl.head_dim * e * 2
+    qo = 2 * wl.num_seqs * wl.num_q_heads * wl.head_dim * e
+    tables = 4 * int(((ctx + wl.block_size - 1) // wl.block_size).sum())
+    return kv + qo + tables + 4 * wl.num_seqs
+
+
+def unique_decode_bytes(wl, runner) -> int:
+    """For workloads whose sequences share blocks: K/V bytes of distinct physical
+    blocks read (whole used blocks), plus q/out/tables as above."""
+    used = set()
+    ctx = wl.context_lens.astype(np.int64)
+    for s in range(wl.num_seqs):
+        n = int((ctx[s] + wl.block_size - 1) // wl.block_size)
+        used.update(runner.block_tables_host[s, :n].tolist())
+    e = wl.elem_bytes
+    kv = len(used) * wl.block_size * wl.num_kv_heads * wl.head_dim * e * 2
+    return kv + decode_bytes(wl) - int(ctx.sum()) * wl.num_kv_heads * wl.head_dim * e * 2
+
+
+def step_bytes(wl, runner) -> int:
+    """Algorithmic bytes of one step: decode + new-token writes + block copies."""
+    row = wl.num_kv_heads * wl.head_dim * wl.elem_bytes
+    t = len(runner.step_slots_host)
+    writes = t * (2 * row * 2 + 8)           # read key+value rows, write them, read slot
+    blk = wl.block_size * row
+    copies = len(runner.cow_pairs) * 2 * blk * 2   # K and V blocks, read + write
+    return decode_bytes(wl) + writes + copies
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", "-i", str(self.gpu),
+               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                bits = int(parts[3], 16) if parts[3].startswith("0x") else int(parts[3])
+            except ValueError:
+                continue
+            for b, name in _REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# helpers
+# --------------------------------------------------------------------------
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def _traffic_for(kernel_src: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+        with open(kernel_src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except (OSError, ValueError, AttributeError):
+        return None
+    if not rec or rec.get("source_sha") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def _rank_info():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def _max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_workload(name: str, rank: int):
+    """The named workload; rank r > 0 gets an independent batch (seed shifted)."""
+    import workloads
+    from workloads import configs
+    if rank == 0:
+        return workloads.workload(name)
+    base = workloads.workload(name)
+    fn = configs.WORKLOADS[name]
+    return fn(seed=base.seed + 7919 * rank)
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and --impl reference)
+# --------------------------------------------------------------------------
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()
+             if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(wl, budget_s: float = 15.0, max_seq: int | None = None):
+    """Times the oracle's paged decode on the first sequences of the workload.
+
+    Grows the sample one sequence at a time until ``budget_s`` of oracle time is
+    used (or the batch is exhausted). Returns (GB/s, tokens/s, description)."""
+    from oracle.attention import paged_decode
+    import time as _t
+    total_t, total_b, total_seq, total_tok = 0.0, 0, 0, 0
+    limit = wl.num_seqs if max_seq is None else min(max_seq, wl.num_seqs)
+    first = 0
+    chunk = 1
+    while first < limit and (total_seq == 0 or total_t < budget_s):
+        n = min(chunk, limit - first)
+        sub, st = oracle_sample_setup_range(wl, first, n)
+        t0 = _t.perf_counter()
+        paged_decode(st.q, st.k_cache, st.v_cache, st.block_tables, sub.context_lens, sub.scale,
+                     sub.dtype, sub.block_size)
+        total_t += _t.perf_counter() - t0
+        total_b += decode_bytes(sub)
+        total_seq += n
+        total_tok += int(sub.context_lens.sum())
+        first += n
+        chunk = min(8, chunk * 2)
+    desc = (f"oracle paged_decode (fp64 NumPy) on {total_seq} of {wl.num_seqs} sequences "
+            f"({total_tok} context tokens, all {wl.num_q_heads} query heads), "
+            f"{total_t:.1f} s of oracle time")
+    return total_b / total_t / 1e9, total_seq / total_t, desc, total_t
+
+
+def oracle_sample_setup_range(wl, first: int, n: int):
+    from oracle import step as OS
+    from workloads.configs import DecodeWorkload
+    ctx = wl.context_lens[first:first + n]
+    nb = int(sum(-(-int(c) // wl.block_size) for c in ctx)) + 1
+    sub = DecodeWorkload(f"{wl.name}[{first}:{first + n}]", wl.seed + first, n, wl.num_q_heads,
+                         wl.num_kv_heads, wl.head_dim, wl.dtype, ctx, nb,
+                         np.random.default_rng([wl.seed, 5, first]).permutation(nb))
+    return sub, OS.decode_step(sub, compute_out=False)
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = _rank_info()
+    if rank != 0:
+        return 0
+    import workloads
+    wl = workloads.workload(args.workload)
+    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    # calibrate the sample size per step on one sequence
+    _, _, _, t1 = time_oracle(wl, budget_s=0.0, max_seq=1)
+    nseq = int(max(1, min(wl.num_seqs, per_step_budget / max(t1, 1e-3))))
+    from oracle.attention import paged_decode
+    sub, st = oracle_sample_setup_range(wl, 0, nseq)
+
+    def one():
+        paged_decode(st.q, st.k_cache, st.v_cache, st.block_tables, sub.context_lens, sub.scale,
+                     sub.dtype, sub.block_size)
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    bytes_per = decode_bytes(sub)
+    value = bytes_per * args.steps / el / 1e9
+    desc = (f"oracle paged_decode (fp64 NumPy) per step on {nseq} of {wl.num_seqs} sequences "
+            f"({int(sub.context_lens.sum())} context tokens, all {wl.num_q_heads} query heads)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, **{k: v for k, v in wl.describe().items()
+                                           if k != "workload"}},
+        "decode_tokens_per_s": round(nseq * args.steps / el, 3),
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": _oracle_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = _rank_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+
+    from paged_kv_cache_352_b200 import build as pabuild
+    pabuild.build()
+    from paged_kv_cache_352_b200.runner import DecodeRunner, HostStep
+
+    wl = rank_workload(args.workload, rank)
+    r = DecodeRunner(wl, device=device,
+                     partition_tokens=args.partition_tokens if args.partition_tokens >= 0 else None)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(3, args.warmup)):
+        r.step()
+    torch.cuda.synchronize(device)
+    if r.error_bits():
+        raise RuntimeError(f"device error bits {r.error_bits()} during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    gpu_index = device.index if device.index is not None else 0
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if visible:
+        try:
+            gpu_index = int(visible.split(",")[gpu_index])
+        except (ValueError, IndexError):
+            pass
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_index) as clocks:
+        time.sleep(0.3)
+        for k in range(K):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            r.copy_blocks()
+            r.reshape_and_cache()
+            ev[k][1].record(stream)
+            r.decode()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize(device)
+    _barrier(world)
+    t_step = np.array([ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]) / 1e3
+    t_dec = np.array([ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]) / 1e3
+    step_s = _max_over_ranks(float(t_step.mean()), world, device)
+    dec_s = _max_over_ranks(float(t_dec.mean()), world, device)
+    if r.error_bits():
+        raise RuntimeError(f"device error bits {r.error_bits()} during timing")
+
+    # e2e: the same step fed from pinned host buffers, result read back
+    hs = HostStep(r)
+    for _ in range(3):
+        hs()
+    torch.cuda.synchronize(device)
+    E = max(5, K // 2)
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(E)]
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    for k in range(E):
+        flush.fill_(k & 0xFF)
+        ee[k][0].record(stream)
+        hs()
+        ee[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    _barrier(world)
+    e2e_s = _max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ee]) / 1e3), world,
+                            device)
+
+    sb = step_bytes(wl, r)
+    db = decode_bytes(wl)
+    peak, peak_kind = _peaks()
+    value = world * sb / step_s / 1e9
+    achieved = db / dec_s / 1e9
+    traffic = _traffic_for(os.path.join(ROOT, "paged_kv_cache_352_b200", "csrc",
+                                        "paged_decode.cu"), wl.name)
+    csum = clocks.summary()
+    launches_per_step = r.launches_per_step()
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": round(step_s * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, **{k: v for k, v in wl.describe().items()
+                                           if k != "workload"},
+                   "partition_tokens": r.partition_tokens or 512,
+                   "l2": "flushed between steps (256 MiB write), outside the timed events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
+        "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
+        "decode_tokens_per_s": round(world * wl.num_seqs / step_s, 1),
+        "decode_only_tokens_per_s": round(world * wl.num_seqs / dec_s, 1),
+        "bytes_per_step": sb,
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": db,
+                     "launch_ms": round(dec_s * 1e3, 4), "peak_kind": peak_kind},
+        "e2e": {"value": round(world * sb / e2e_s / 1e9, 2), "unit": UNIT,
+                "h2d_bytes_per_step": hs.h2d_bytes, "d2h_bytes_per_step": hs.d2h_bytes,
+                "ms_per_step": round(e2e_s * 1e3, 4)},
+        "gpu_launches": K * launches_per_step,
+        "clocks": csum,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, tps, desc, _ = time_oracle(wl, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": _oracle_threads(),
+                                "kind": "oracle", "sample": desc,
+                                "decode_tokens_per_s": round(tps, 3)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--partition-tokens", type=int, default=-1,
+                    help="split-KV partition size (default: the workload's / library default)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle time for the cpu_baseline sample")
+    args = ap.parse_args(argv)
+    if args.steps < 1 or args.warmup < 0:
+        ap.error("--steps >= 1 and --warmup >= 0")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,227 @@
+/*
+ * pa.h — C interface of libpa, a paged KV cache and paged-decode attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (PagedAttention) keeps every sequence's attention keys and values
+ * in fixed-size blocks of 16 tokens taken on demand from a pool allocated once
+ * up front; a per-sequence block table maps logical blocks to physical ones, and
+ * attention reads the cache through that table. Blocks can be shared between
+ * sequences and are copied only when one of them writes (copy-on-write).
+ * Sources: "PagedAttention and Continuous Batching" (roadtointelligence.com),
+ * section "Pages, from operating systems"; "PagedAttention: The vLLM Paper"
+ * (ai.zenoagi.com), sections "The Core Idea", "The OS paging analogy" and
+ * "Implementation Essentials"; "vLLM: PagedAttention and continuous batching"
+ * (llmstudy.shddai.net), direct answer. The pages define no programming
+ * interface; the calls below are this library's.
+ *
+ * Conventions for every call
+ *   - Return value: a pa_status (0 = PA_OK). On failure, pa_last_error() holds a
+ *     message for the calling thread until its next libpa call.
+ *   - Device calls (pa_reshape_and_cache, pa_copy_blocks, pa_paged_decode) take
+ *     device pointers owned by the caller, enqueue kernels on the caller's CUDA
+ *     stream (`stream` is a cudaStream_t; NULL = legacy default stream), never
+ *     synchronise, never allocate device memory, and return after the launch.
+ *     Scalar arguments are checked on the host before anything is launched; a
+ *     failed check launches nothing. Data-dependent faults (a slot or block id
+ *     outside the pool, a context longer than the table) are never trapped on the
+ *     device: the offending access is skipped and a bit is OR-ed into *dev_error
+ *     when dev_error is non-NULL (a device int the caller zeroes and reads back).
+ *   - Supported shapes: block_size 16, head_dim 64 or 128, num_q_heads a
+ *     multiple of num_kv_heads with a ratio of 1, 2, 4 or 8, fp16 or bf16 storage.
+ *     Other shapes return PA_ERR_UNSUPPORTED.
+ *   - Cache layout: two arrays, k_cache and v_cache, each
+ *     [num_blocks][num_kv_heads][block_size][head_dim] row-major in the storage
+ *     type; slot s is offset s % block_size of block s / block_size. Base
+ *     pointers must be 16-byte aligned.
+ *   - Host block-manager calls (pa_bm_*) are all-or-nothing: on failure the
+ *     manager's state is unchanged. A manager is not thread-safe.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,    /* bad pointer, size or value */
+  PA_ERR_NO_FREE_BLOCKS = 2, /* the pool cannot cover the request */
+  PA_ERR_UNKNOWN_SEQ = 3,    /* sequence id not registered */
+  PA_ERR_CUDA = 4,           /* a CUDA runtime call failed */
+  PA_ERR_UNSUPPORTED = 5,    /* shape or type outside the supported set */
+  PA_ERR_SEQ_EXISTS = 6      /* sequence id already registered */
+} pa_status;
+
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits OR-ed into *dev_error by device calls. */
+#define PA_DEVERR_SLOT_RANGE 1    /* slot >= num_blocks * block_size: token not written */
+#define PA_DEVERR_BLOCK_RANGE 2   /* block-table entry outside [0, num_blocks): block skipped */
+#define PA_DEVERR_CONTEXT_RANGE 4 /* context_lens[s] < 0, > max_blocks_per_seq*block_size,
+                                     or > max_context_len: sequence skipped (zero output) */
+#define PA_DEVERR_WAIT_TIMEOUT 8  /* a bounded on-chip wait gave up: output invalid */
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Library interface version (major * 100 + minor). */
+int pa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * pa_reshape_and_cache — store new tokens' keys and values in their slots.
+ *
+ * Every generated token's K/V is cached so decode need not recompute it
+ * ("PagedAttention: The vLLM Paper", "Background and Motivation"), and blocks
+ * are filled as tokens arrive ("PagedAttention and Continuous Batching",
+ * "Pages, from operating systems"). For each token t with slot_mapping[t] >= 0:
+ *   k_cache[slot / bs][h][slot % bs][:] = key[t][h][:]   for every KV head h,
+ * and likewise for value / v_cache. slot_mapping[t] < 0 skips token t.
+ *
+ *   key, value        device, [num_tokens][num_kv_heads][head_dim] with a token
+ *                     stride of key_token_stride / value_token_stride elements
+ *                     (>= num_kv_heads*head_dim, a multiple of 8); 16-byte aligned
+ *   k_cache, v_cache  device, cache layout above; written in place
+ *   slot_mapping      device, int64 [num_tokens]
+ *   dev_error         device int or NULL (PA_DEVERR_SLOT_RANGE)
+ * Slots must be distinct among the tokens of one call (which write wins is
+ * otherwise unspecified). num_tokens == 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_stride,
+                         int64_t value_token_stride, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, int dtype,
+                         int* dev_error, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_copy_blocks — the copy half of copy-on-write.
+ *
+ * A block shared by several sequences is copied only when one of them must
+ * modify it ("PagedAttention and Continuous Batching", "Pages, from operating
+ * systems"; "PagedAttention: The vLLM Paper", "The OS paging analogy", page
+ * sharing). For each pair i: block pairs[2i+1] of k_cache and of v_cache
+ * becomes a copy of block pairs[2i] (all KV heads, all 16 slots).
+ *
+ *   pairs   HOST array, int64 [num_pairs][2] = (src, dst); read before return.
+ *           Every id in [0, num_blocks); dst ids distinct; no dst equal to any
+ *           src of the same call (so the copies are independent). Violations
+ *           return PA_ERR_INVALID_ARG and launch nothing.
+ * The pairs travel in the kernel's parameter block: no device buffer is needed.
+ * num_pairs == 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                   void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_paged_decode — decode-step attention through the block tables.
+ *
+ * Attention follows the block-table mapping, reading the cache where it lies
+ * ("vLLM: PagedAttention and continuous batching", direct answer; "PagedAttention:
+ * The vLLM Paper", "The Core Idea", the note under the block-table figure). For
+ * sequence s and query head h, with G = num_q_heads / num_kv_heads and
+ * g = h / G:
+ *   K_s[t] = k_cache[block_tables[s][t / bs]][g][t % bs][:]   t < context_lens[s]
+ *   out[s][h] = softmax(scale * K_s q[s][h]) V_s
+ * computed in fp32 (online softmax) and rounded to the storage type (nearest
+ * even). A zero-length context gives a zero row. Long contexts are cut into
+ * partitions of `partition_tokens` tokens processed in parallel and merged by
+ * log-sum-exp rescaling inside the same kernel launch (split-KV).
+ *
+ *   out                device, [num_seqs][num_q_heads][head_dim], storage type
+ *   q                  device, [num_seqs][num_q_heads][head_dim], storage type
+ *   k_cache, v_cache   device, cache layout above (read only)
+ *   block_tables       device, int32 [num_seqs][max_blocks_per_seq], padded with -1
+ *   context_lens       device, int32 [num_seqs], tokens per sequence including the
+ *                      token written this step
+ *   max_context_len    host-known upper bound of context_lens (sizes the grid
+ *                      without a device read); longer sequences are flagged
+ *   scale              softmax scale, usually 1/sqrt(head_dim)
+ *   partition_tokens   0 = library default (512); else a multiple of block_size
+ *   workspace          device scratch of pa_paged_decode_workspace_size() bytes,
+ *                      ZERO-FILLED before its first use; every completed call
+ *                      leaves it zero-filled again, so it can be reused without
+ *                      clearing. Calls that run concurrently need separate
+ *                      workspaces. May be NULL when the size is 0. After a call
+ *                      that reported PA_DEVERR_WAIT_TIMEOUT, zero it again.
+ *   dev_error          device int or NULL
+ * Reduction order depends only on logical token positions, so results are
+ * bit-identical whatever the physical placement of blocks and whether blocks
+ * are shared or duplicated.
+ * ------------------------------------------------------------------------- */
+int pa_paged_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int max_context_len, int block_size,
+                                   int partition_tokens, size_t* bytes);
+
+int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* context_lens, int num_seqs, int max_context_len,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, float scale, int partition_tokens, void* workspace,
+                    size_t workspace_bytes, int* dev_error, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Host block manager.
+ *
+ * "A pre-allocated memory pool, block allocation/reclamation, and refcounts
+ * enabling cross-sequence sharing" ("PagedAttention: The vLLM Paper",
+ * "Implementation Essentials"); blocks are taken on demand and only the last
+ * block of a sequence may be partly filled ("The design yields three immediate
+ * wins", item 1); parallel samples share the prompt's blocks (item 3 and
+ * "Implementation Essentials", prefix sharing).
+ *
+ * Rules the pages leave open, fixed here:
+ *   - The free list is a stack: initial_free_order[0] is handed out first;
+ *     released blocks go on top. NULL initial_free_order = 0, 1, 2, ...
+ *   - pa_bm_free_seq releases a sequence's blocks from its last logical block
+ *     to its first; a block returns to the free list when its refcount hits 0.
+ *   - pa_bm_append_slots: when the first appended token falls in a partly
+ *     filled last block whose refcount is > 1, the sequence gets a fresh block,
+ *     (old, new) is written to cow_pairs_out and old's refcount drops by one.
+ *     The caller must run pa_copy_blocks on those pairs before writing the
+ *     appended tokens. At most one pair per call.
+ * Slots are block * block_size + offset (the slot_mapping of
+ * pa_reshape_and_cache). Sequence ids are arbitrary int64 values.
+ * ------------------------------------------------------------------------- */
+typedef struct pa_bm pa_bm;
+
+int pa_bm_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                 pa_bm** out);
+void pa_bm_destroy(pa_bm* bm);
+
+/* Register seq_id holding num_tokens tokens; their slots go to slots_out[num_tokens]
+ * (may be NULL when num_tokens == 0). */
+int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens, int64_t* slots_out);
+
+/* child shares every block of parent (refcounts + 1). */
+int pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child);
+
+/* Append n tokens to seq_id: slots_out[n]; cow_pairs_out[2] receives at most one
+ * (src, dst) pair and *n_cow its count (0 or 1). */
+int pa_bm_append_slots(pa_bm* bm, int64_t seq_id, int n, int64_t* slots_out,
+                       int64_t* cow_pairs_out, int* n_cow);
+
+int pa_bm_free_seq(pa_bm* bm, int64_t seq_id);
+
+/* Tables of seq_ids[0..n) into out[n][max_blocks], padded with -1;
+ * PA_ERR_INVALID_ARG if a table is longer than max_blocks. */
+int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* out,
+                       int max_blocks);
+
+/* Queries. pa_bm_refcount and pa_bm_seq_len return -1 for an unknown block or
+ * sequence (and set pa_last_error). */
+int pa_bm_num_free(const pa_bm* bm);
+int pa_bm_refcount(const pa_bm* bm, int32_t block);
+int pa_bm_seq_len(const pa_bm* bm, int64_t seq_id);
+int pa_bm_num_seqs(const pa_bm* bm);
+/* Free blocks in hand-out order into out[capacity]; returns the count written or -1. */
+int pa_bm_free_list(const pa_bm* bm, int32_t* out, int capacity);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,26 @@
+"""Paged KV cache and paged-decode attention for NVIDIA B200 (sm_100a).
+
+The C library ``libpa.so`` (kernels + host block manager, interface in
+``include/pa.h``) does the work; this package is its ctypes binding
+(``_lib``), a build script (``build``) and a runner that drives one decode
+step of a workload through the library (``runner``).
+"""
+
+from ._lib import (  # noqa: F401
+    BLOCK_SIZE,
+    BlockManager,
+    PAError,
+    PA_BF16,
+    PA_DEVERR_BLOCK_RANGE,
+    PA_DEVERR_CONTEXT_RANGE,
+    PA_DEVERR_SLOT_RANGE,
+    PA_DEVERR_WAIT_TIMEOUT,
+    PA_F16,
+    decode_workspace,
+    last_error,
+    lib,
+    pa_copy_blocks,
+    pa_paged_decode,
+    pa_paged_decode_workspace_size,
+    pa_reshape_and_cache,
+)

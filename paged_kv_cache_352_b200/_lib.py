@@ -1,0 +1,318 @@
+"""ctypes binding to libpa.so: the C interface's calls under the same names.
+
+Only argument marshalling happens here: tensors become device pointers, the
+current PyTorch CUDA stream becomes the launch stream, and non-zero statuses
+become ``PAError``. Every step of the decode path runs in libpa's kernels.
+The library must be built (``python -m paged_kv_cache_352_b200.build``); there
+is no fallback when it is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpa.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_NO_FREE_BLOCKS = 2
+PA_ERR_UNKNOWN_SEQ = 3
+PA_ERR_CUDA = 4
+PA_ERR_UNSUPPORTED = 5
+PA_ERR_SEQ_EXISTS = 6
+
+PA_F16 = 0
+PA_BF16 = 1
+
+PA_DEVERR_SLOT_RANGE = 1
+PA_DEVERR_BLOCK_RANGE = 2
+PA_DEVERR_CONTEXT_RANGE = 4
+PA_DEVERR_WAIT_TIMEOUT = 8
+
+BLOCK_SIZE = 16
+
+
+class PAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libpa status {code}: {msg}")
+        self.code = code
+
+
+_c_int = ctypes.c_int
+_c_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+_SIGS = {
+    "pa_last_error": (ctypes.c_char_p, []),
+    "pa_version": (_c_int, []),
+    "pa_reshape_and_cache": (_c_int, [_vp, _vp, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int,
+                                      _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
+    "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _vp]),
+    "pa_paged_decode_workspace_size": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                                _c_int, ctypes.POINTER(ctypes.c_size_t)]),
+    "pa_paged_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_int, ctypes.c_float, _c_int, _vp,
+                                 ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_bm_create": (_c_int, [_c_int, _c_int, _vp, ctypes.POINTER(_vp)]),
+    "pa_bm_destroy": (None, [_vp]),
+    "pa_bm_add_seq": (_c_int, [_vp, _c_i64, _c_int, _vp]),
+    "pa_bm_fork": (_c_int, [_vp, _c_i64, _c_i64]),
+    "pa_bm_append_slots": (_c_int, [_vp, _c_i64, _c_int, _vp, _vp, ctypes.POINTER(_c_int)]),
+    "pa_bm_free_seq": (_c_int, [_vp, _c_i64]),
+    "pa_bm_block_tables": (_c_int, [_vp, _vp, _c_int, _vp, _c_int]),
+    "pa_bm_num_free": (_c_int, [_vp]),
+    "pa_bm_refcount": (_c_int, [_vp, ctypes.c_int32]),
+    "pa_bm_seq_len": (_c_int, [_vp, _c_i64]),
+    "pa_bm_num_seqs": (_c_int, [_vp]),
+    "pa_bm_free_list": (_c_int, [_vp, _vp, _c_int]),
+}
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libpa (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m paged_kv_cache_352_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = h
+    return _LIB
+
+
+def last_error() -> str:
+    return lib().pa_last_error().decode()
+
+
+def _check(status: int):
+    if status != PA_OK:
+        raise PAError(status, last_error())
+
+
+# --------------------------------------------------------------------------
+# tensor marshalling
+# --------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise PAError(PA_ERR_UNSUPPORTED, f"storage type {t.dtype}: expected float16 or bfloat16")
+
+
+def _dev_ptr(t, name, dtype=None, contiguous=True):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise PAError(PA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise PAError(PA_ERR_INVALID_ARG, f"{name} must be {dtype}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise PAError(PA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _cache_dims(k_cache, v_cache):
+    if k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype or k_cache.dim() != 4:
+        raise PAError(PA_ERR_INVALID_ARG,
+                      "k_cache and v_cache must both be [num_blocks, num_kv_heads, block_size, "
+                      "head_dim] with one dtype")
+    nb, hkv, bs, d = k_cache.shape
+    return nb, hkv, bs, d
+
+
+# --------------------------------------------------------------------------
+# device calls
+# --------------------------------------------------------------------------
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, dev_error=None, stream=None):
+    """Store ``key``/``value`` ``[T, num_kv_heads, head_dim]`` at ``slot_mapping`` (int64 [T])."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    T = key.shape[0]
+    if key.shape[1:] != (hkv, d) or value.shape[1:] != (hkv, d) or value.shape[0] != T:
+        raise PAError(PA_ERR_INVALID_ARG, "key/value must be [T, num_kv_heads, head_dim]")
+    if key.stride(2) != 1 or key.stride(1) != d or value.stride(2) != 1 or value.stride(1) != d:
+        raise PAError(PA_ERR_INVALID_ARG, "key/value rows must be dense per token")
+    if slot_mapping.shape != (T,):
+        raise PAError(PA_ERR_INVALID_ARG, "slot_mapping must be [T]")
+    _check(lib().pa_reshape_and_cache(
+        _dev_ptr(key, "key", k_cache.dtype, contiguous=False),
+        _dev_ptr(value, "value", k_cache.dtype, contiguous=False),
+        key.stride(0), value.stride(0),
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, hkv, d, bs, nb,
+        dtype_code(k_cache), _dev_ptr(dev_error, "dev_error", torch.int32), _stream(stream)))
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
+    """Copy blocks ``pairs[i, 0] -> pairs[i, 1]`` (host int64 array ``[n, 2]``)."""
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    p = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    _check(lib().pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+                                p.ctypes.data if len(p) else None, len(p), hkv, d, bs, nb,
+                                dtype_code(k_cache), _stream(stream)))
+
+
+def pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                   max_context_len, block_size=BLOCK_SIZE, partition_tokens=0):
+    out = ctypes.c_size_t(0)
+    _check(lib().pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                max_context_len, block_size, partition_tokens,
+                                                ctypes.byref(out)))
+    return out.value
+
+
+def decode_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                     partition_tokens=0, device=None):
+    """A zero-filled workspace tensor of the size pa_paged_decode needs (None if 0)."""
+    torch = _torch()
+    n = pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                       max_context_len, BLOCK_SIZE, partition_tokens)
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                    scale, partition_tokens=0, workspace=None, dev_error=None, stream=None):
+    """Decode attention through block tables; writes ``out`` ``[B, Hq, d]``.
+
+    ``workspace`` must be a zero-filled uint8 CUDA tensor of at least
+    ``pa_paged_decode_workspace_size(...)`` bytes when that size is non-zero.
+    """
+    torch = _torch()
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    B, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or out.dtype != k_cache.dtype or q.dtype != k_cache.dtype:
+        raise PAError(PA_ERR_INVALID_ARG, "q/out must be [B, num_q_heads, head_dim] in the "
+                                          "cache's dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
+    ws_bytes = 0
+    if workspace is not None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().pa_paged_decode(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32), B,
+        int(max_context_len), hq, hkv, d, bs, nb, float(scale), int(partition_tokens),
+        _dev_ptr(workspace, "workspace"), ws_bytes,
+        _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
+
+
+# --------------------------------------------------------------------------
+# host block manager
+# --------------------------------------------------------------------------
+
+def _i64p(a):
+    return a.ctypes.data if a is not None and a.size else None
+
+
+class BlockManager:
+    """Owner of one ``pa_bm`` handle (the pa_bm_* calls as methods)."""
+
+    def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE, initial_free_order=None):
+        self._lib = lib()
+        order = None
+        if initial_free_order is not None:
+            order = np.ascontiguousarray(np.asarray(initial_free_order, dtype=np.int32))
+            if order.shape != (num_blocks,):
+                raise PAError(PA_ERR_INVALID_ARG, "initial_free_order must have num_blocks ids")
+        h = ctypes.c_void_p()
+        _check(self._lib.pa_bm_create(num_blocks, block_size,
+                                      order.ctypes.data if order is not None else None,
+                                      ctypes.byref(h)))
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id: int, num_tokens: int) -> np.ndarray:
+        slots = np.empty(max(num_tokens, 0), np.int64)
+        _check(self._lib.pa_bm_add_seq(self._h, seq_id, num_tokens, _i64p(slots)))
+        return slots
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(self._lib.pa_bm_fork(self._h, parent, child))
+
+    def append_slots(self, seq_id: int, n: int):
+        slots = np.empty(max(n, 0), np.int64)
+        pairs = np.empty(2, np.int64)
+        ncow = ctypes.c_int(0)
+        _check(self._lib.pa_bm_append_slots(self._h, seq_id, n, _i64p(slots), pairs.ctypes.data,
+                                            ctypes.byref(ncow)))
+        return slots, pairs[:2 * ncow.value].reshape(-1, 2).copy()
+
+    def free_seq(self, seq_id: int) -> None:
+        _check(self._lib.pa_bm_free_seq(self._h, seq_id))
+
+    def block_tables(self, seq_ids, max_blocks: int) -> np.ndarray:
+        ids = np.ascontiguousarray(np.asarray(list(seq_ids), dtype=np.int64))
+        out = np.empty((len(ids), max_blocks), np.int32)
+        _check(self._lib.pa_bm_block_tables(self._h, _i64p(ids), len(ids),
+                                            out.ctypes.data if out.size else None, max_blocks))
+        return out
+
+    def num_free(self) -> int:
+        return self._lib.pa_bm_num_free(self._h)
+
+    def refcount(self, block: int) -> int:
+        r = self._lib.pa_bm_refcount(self._h, block)
+        if r < 0:
+            raise PAError(PA_ERR_INVALID_ARG, last_error())
+        return r
+
+    def seq_len(self, seq_id: int) -> int:
+        r = self._lib.pa_bm_seq_len(self._h, seq_id)
+        if r < 0:
+            raise PAError(PA_ERR_UNKNOWN_SEQ, last_error())
+        return r
+
+    def num_seqs(self) -> int:
+        return self._lib.pa_bm_num_seqs(self._h)
+
+    def free_list(self) -> list:
+        out = np.empty(self.num_blocks, np.int32)
+        n = self._lib.pa_bm_free_list(self._h, out.ctypes.data, self.num_blocks)
+        return out[:n].tolist()
+
+    def table(self, seq_id: int) -> list:
+        n = -(-self.seq_len(seq_id) // self.block_size)
+        return self.block_tables([seq_id], max(n, 1))[0, :n].tolist()

@@ -1,0 +1,222 @@
+// Host block manager of the paged KV cache.
+//
+// A pool of equal blocks allocated once; per-sequence block tables mapping
+// logical to physical blocks; blocks taken on demand as tokens arrive; refcounts
+// so forked sequences share blocks, with a copy only when a sharer writes
+// ("PagedAttention: The vLLM Paper", "Implementation Essentials" and "The OS
+// paging analogy"; "PagedAttention and Continuous Batching", "Pages, from
+// operating systems").
+//
+// Every mutating call first works out how many free blocks it needs and fails
+// before touching any state when the pool cannot cover it.
+#include <stdint.h>
+
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pa_internal.h"
+
+struct pa_bm {
+  struct Seq {
+    std::vector<int32_t> table;
+    int64_t len = 0;
+  };
+  int num_blocks = 0;
+  int block_size = 0;
+  std::vector<int32_t> free_stack;  // back() is handed out next
+  std::vector<int32_t> ref;
+  std::unordered_map<int64_t, Seq> seqs;
+
+  int32_t pop() {
+    const int32_t b = free_stack.back();
+    free_stack.pop_back();
+    ref[b] = 1;
+    return b;
+  }
+  int64_t slot(const Seq& s, int64_t pos) const {
+    return (int64_t)s.table[pos / block_size] * block_size + pos % block_size;
+  }
+};
+
+using pa::fail;
+
+namespace {
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+extern "C" {
+
+int pa_bm_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                 pa_bm** out) {
+  pa::clear_error();
+  if (!out) return fail(PA_ERR_INVALID_ARG, "out must not be NULL");
+  *out = nullptr;
+  if (num_blocks <= 0 || block_size <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_blocks and block_size must be positive");
+  pa_bm* bm = new (std::nothrow) pa_bm;
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "out of host memory");
+  bm->num_blocks = num_blocks;
+  bm->block_size = block_size;
+  bm->ref.assign(num_blocks, 0);
+  bm->free_stack.resize(num_blocks);
+  if (initial_free_order) {
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+      const int32_t b = initial_free_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete bm;
+        return fail(PA_ERR_INVALID_ARG, "initial_free_order is not a permutation of the pool");
+      }
+      seen[b] = 1;
+      bm->free_stack[num_blocks - 1 - i] = b;
+    }
+  } else {
+    for (int i = 0; i < num_blocks; ++i) bm->free_stack[num_blocks - 1 - i] = i;
+  }
+  *out = bm;
+  return PA_OK;
+}
+
+void pa_bm_destroy(pa_bm* bm) { delete bm; }
+
+int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens, int64_t* slots_out) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0");
+  if (num_tokens > 0 && !slots_out) return fail(PA_ERR_INVALID_ARG, "slots_out is NULL");
+  if (bm->seqs.count(seq_id))
+    return fail(PA_ERR_SEQ_EXISTS, "sequence %lld exists", (long long)seq_id);
+  const int64_t need = ceil_div(num_tokens, bm->block_size);
+  if (need > (int64_t)bm->free_stack.size())
+    return fail(PA_ERR_NO_FREE_BLOCKS, "need %lld blocks, %zu free", (long long)need,
+                bm->free_stack.size());
+  pa_bm::Seq s;
+  s.table.reserve(need);
+  for (int64_t i = 0; i < need; ++i) s.table.push_back(bm->pop());
+  s.len = num_tokens;
+  for (int64_t p = 0; p < num_tokens; ++p) slots_out[p] = bm->slot(s, p);
+  bm->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+int pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  auto it = bm->seqs.find(parent);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)parent);
+  if (bm->seqs.count(child))
+    return fail(PA_ERR_SEQ_EXISTS, "sequence %lld exists", (long long)child);
+  pa_bm::Seq s = it->second;
+  for (int32_t b : s.table) ++bm->ref[b];
+  bm->seqs.emplace(child, std::move(s));
+  return PA_OK;
+}
+
+int pa_bm_append_slots(pa_bm* bm, int64_t seq_id, int n, int64_t* slots_out,
+                       int64_t* cow_pairs_out, int* n_cow) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  if (n < 0) return fail(PA_ERR_INVALID_ARG, "n must be >= 0");
+  if ((n > 0 && !slots_out) || !cow_pairs_out || !n_cow)
+    return fail(PA_ERR_INVALID_ARG, "null output pointer");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+  pa_bm::Seq& s = it->second;
+  const int bs = bm->block_size;
+  const int64_t new_blocks = ceil_div(s.len + n, bs) - (int64_t)s.table.size();
+  const bool cow = n > 0 && s.len % bs != 0 && bm->ref[s.table.back()] > 1;
+  if (new_blocks + (cow ? 1 : 0) > (int64_t)bm->free_stack.size())
+    return fail(PA_ERR_NO_FREE_BLOCKS, "need %lld blocks, %zu free",
+                (long long)(new_blocks + (cow ? 1 : 0)), bm->free_stack.size());
+  *n_cow = 0;
+  if (cow) {
+    const int32_t old = s.table.back();
+    const int32_t fresh = bm->pop();
+    --bm->ref[old];
+    s.table.back() = fresh;
+    cow_pairs_out[0] = old;
+    cow_pairs_out[1] = fresh;
+    *n_cow = 1;
+  }
+  for (int64_t p = s.len; p < s.len + n; ++p) {
+    if (p % bs == 0) s.table.push_back(bm->pop());
+    slots_out[p - s.len] = bm->slot(s, p);
+  }
+  s.len += n;
+  return PA_OK;
+}
+
+int pa_bm_free_seq(pa_bm* bm, int64_t seq_id) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+  const std::vector<int32_t>& t = it->second.table;
+  for (auto b = t.rbegin(); b != t.rend(); ++b)
+    if (--bm->ref[*b] == 0) bm->free_stack.push_back(*b);
+  bm->seqs.erase(it);
+  return PA_OK;
+}
+
+int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* out,
+                       int max_blocks) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  if (n < 0 || max_blocks < 0) return fail(PA_ERR_INVALID_ARG, "negative size");
+  if (n == 0) return PA_OK;
+  if (!seq_ids || !out) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  for (int i = 0; i < n; ++i) {  // validate everything before writing anything
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end())
+      return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_ids[i]);
+    if ((int64_t)it->second.table.size() > max_blocks)
+      return fail(PA_ERR_INVALID_ARG, "sequence %lld holds %zu blocks > max_blocks %d",
+                  (long long)seq_ids[i], it->second.table.size(), max_blocks);
+  }
+  for (int i = 0; i < n; ++i) {
+    const std::vector<int32_t>& t = bm->seqs.find(seq_ids[i])->second.table;
+    int32_t* row = out + (size_t)i * max_blocks;
+    size_t k = 0;
+    for (; k < t.size(); ++k) row[k] = t[k];
+    for (; k < (size_t)max_blocks; ++k) row[k] = -1;
+  }
+  return PA_OK;
+}
+
+int pa_bm_num_free(const pa_bm* bm) { return bm ? (int)bm->free_stack.size() : -1; }
+
+int pa_bm_refcount(const pa_bm* bm, int32_t block) {
+  if (!bm || block < 0 || block >= bm->num_blocks) {
+    fail(PA_ERR_INVALID_ARG, "block id out of range");
+    return -1;
+  }
+  return bm->ref[block];
+}
+
+int pa_bm_seq_len(const pa_bm* bm, int64_t seq_id) {
+  if (!bm) return -1;
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) {
+    fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+    return -1;
+  }
+  return (int)it->second.len;
+}
+
+int pa_bm_num_seqs(const pa_bm* bm) { return bm ? (int)bm->seqs.size() : -1; }
+
+int pa_bm_free_list(const pa_bm* bm, int32_t* out, int capacity) {
+  if (!bm || (!out && capacity > 0) || capacity < 0) return -1;
+  const int n = (int)bm->free_stack.size();
+  const int m = n < capacity ? n : capacity;
+  for (int i = 0; i < m; ++i) out[i] = bm->free_stack[n - 1 - i];
+  return m;
+}
+
+}  // extern "C"

@@ -1,0 +1,247 @@
+// C interface of libpa: argument checks on the host, then kernel launches on the
+// caller's stream. Nothing here synchronises or allocates device memory.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <string>
+#include <unordered_set>
+#include <vector>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+static thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cache_shape(int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype) {
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "dtype %d: expected PA_F16 or PA_BF16", dtype);
+  if (block_size != kBlockSize)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d: only %d is supported", block_size,
+                kBlockSize);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", head_dim);
+  if (num_kv_heads <= 0) return fail(PA_ERR_INVALID_ARG, "num_kv_heads must be positive");
+  if (num_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "num_blocks must be positive");
+  return PA_OK;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return PA_OK;
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                  int max_context_len, int partition_tokens, DecodeLayout* lay) {
+  if (partition_tokens == 0) partition_tokens = kDefaultPartitionTokens;
+  if (partition_tokens < 0 || partition_tokens % kBlockSize != 0)
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens %d: must be 0 or a positive multiple of %d",
+                partition_tokens, kBlockSize);
+  if (max_context_len < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len must be >= 0");
+  const int group = num_q_heads / num_kv_heads;
+  const int part_blocks = partition_tokens / kBlockSize;
+  const int max_blocks = (max_context_len + kBlockSize - 1) / kBlockSize;
+  int max_parts = (max_blocks + part_blocks - 1) / part_blocks;
+  if (max_parts < 1) max_parts = 1;
+  if (max_parts > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "%d partitions per sequence exceed the grid limit", max_parts);
+  lay->part_blocks = part_blocks;
+  lay->max_parts = max_parts;
+  if (max_parts == 1) {
+    lay->count_off = lay->ml_off = lay->acc_off = lay->bytes = 0;
+    return PA_OK;
+  }
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t units = (size_t)num_seqs * num_kv_heads;
+  lay->count_off = 0;
+  lay->ml_off = up(units * sizeof(int));
+  lay->acc_off = up(lay->ml_off + units * max_parts * group * 2 * sizeof(float));
+  lay->bytes = up(lay->acc_off + units * max_parts * group * head_dim * sizeof(float));
+  return PA_OK;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_last_error(void) { return g_last_error.c_str(); }
+
+int pa_version(void) { return 100; }
+
+int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_stride,
+                         int64_t value_token_stride, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, int dtype,
+                         int* dev_error, void* stream) {
+  clear_error();
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0");
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  const int64_t row = (int64_t)num_kv_heads * head_dim;
+  if (key_token_stride < row || value_token_stride < row || key_token_stride % 8 ||
+      value_token_stride % 8)
+    return fail(PA_ERR_INVALID_ARG,
+                "token strides (%lld, %lld) must be >= num_kv_heads*head_dim (%lld) and a "
+                "multiple of 8",
+                (long long)key_token_stride, (long long)value_token_stride, (long long)row);
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "key, value and cache pointers must be 16-byte aligned");
+  return cuda_status(launch_reshape_and_cache(key, value, key_token_stride, value_token_stride,
+                                              k_cache, v_cache, slot_mapping, num_tokens,
+                                              num_kv_heads, head_dim, num_blocks, dev_error,
+                                              static_cast<cudaStream_t>(stream)),
+                     "reshape_and_cache launch");
+}
+
+int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                   void* stream) {
+  clear_error();
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
+  if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs must be >= 0");
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !pairs) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "cache pointers must be 16-byte aligned");
+  std::unordered_set<int64_t> dsts, srcs;
+  dsts.reserve(num_pairs * 2);
+  srcs.reserve(num_pairs * 2);
+  for (int i = 0; i < num_pairs; ++i) {
+    const int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks)
+      return fail(PA_ERR_INVALID_ARG, "pair %d (%lld -> %lld) outside the pool of %d blocks", i,
+                  (long long)s, (long long)d, num_blocks);
+    if (!dsts.insert(d).second)
+      return fail(PA_ERR_INVALID_ARG, "destination block %lld appears twice", (long long)d);
+    srcs.insert(s);
+  }
+  for (int64_t d : dsts)
+    if (srcs.count(d))
+      return fail(PA_ERR_INVALID_ARG, "block %lld is both a source and a destination",
+                  (long long)d);
+  const int64_t block_bytes = (int64_t)num_kv_heads * kBlockSize * head_dim * 2;
+  for (int first = 0; first < num_pairs; first += kMaxCopyPairsPerLaunch) {
+    const int n = std::min(kMaxCopyPairsPerLaunch, num_pairs - first);
+    CopyPairs cp;
+    for (int i = 0; i < n; ++i) {
+      cp.src[i] = (int32_t)pairs[2 * (first + i)];
+      cp.dst[i] = (int32_t)pairs[2 * (first + i) + 1];
+    }
+    if (int st = cuda_status(launch_copy_blocks(k_cache, v_cache, cp, n, block_bytes,
+                                                static_cast<cudaStream_t>(stream)),
+                             "copy_blocks launch"))
+      return st;
+  }
+  return PA_OK;
+}
+
+int pa_paged_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int max_context_len, int block_size, int partition_tokens,
+                                   size_t* bytes) {
+  clear_error();
+  if (!bytes) return fail(PA_ERR_INVALID_ARG, "bytes must not be NULL");
+  if (block_size != kBlockSize)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d: only %d is supported", block_size,
+                kBlockSize);
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "bad sequence or head counts");
+  DecodeLayout lay;
+  if (int st = decode_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                             partition_tokens, &lay))
+    return st;
+  *bytes = lay.bytes;
+  return PA_OK;
+}
+
+int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* context_lens, int num_seqs, int max_context_len,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, float scale, int partition_tokens, void* workspace,
+                    size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
+  clear_error();
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "num_seqs must be >= 0");
+  if (num_seqs > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "num_seqs %d exceeds 65535 per call", num_seqs);
+  if (num_q_heads <= 0 || num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads %d must be a positive multiple of num_kv_heads %d",
+                num_q_heads, num_kv_heads);
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return fail(PA_ERR_UNSUPPORTED, "query heads per KV head = %d: supported 1, 2, 4, 8", group);
+  if (num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "too many KV heads");
+  if (max_blocks_per_seq <= 0) return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq must be > 0");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "out, q and cache pointers must be 16-byte aligned");
+  DecodeLayout lay;
+  if (int st = decode_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                             partition_tokens, &lay))
+    return st;
+  if (lay.bytes > 0) {
+    if (!workspace || workspace_bytes < lay.bytes)
+      return fail(PA_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", lay.bytes,
+                  workspace ? workspace_bytes : (size_t)0);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  a.ws_count = lay.bytes ? reinterpret_cast<int*>(ws + lay.count_off) : nullptr;
+  a.ws_ml = lay.bytes ? reinterpret_cast<float*>(ws + lay.ml_off) : nullptr;
+  a.ws_acc = lay.bytes ? reinterpret_cast<float*>(ws + lay.acc_off) : nullptr;
+  a.dev_error = dev_error;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.max_context_len = max_context_len;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.part_blocks = lay.part_blocks;
+  a.max_parts = lay.max_parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e =
+      launch_paged_decode(a, head_dim, group, dtype, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidConfiguration)
+    return fail(PA_ERR_UNSUPPORTED,
+                "%d partitions per sequence need more shared memory than the kernel allows; "
+                "use a larger partition_tokens",
+                lay.max_parts);
+  return cuda_status(e, "paged_decode launch");
+}
+
+}  // extern "C"

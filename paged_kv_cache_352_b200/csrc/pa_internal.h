@@ -1,0 +1,70 @@
+// Internal declarations shared by libpa's translation units (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+constexpr int kBlockSize = 16;                 // tokens per cache block
+constexpr int kDefaultPartitionTokens = 512;   // split-KV partition when the caller passes 0
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // bounded on-chip waits: 1 s
+constexpr int kMaxCopyPairsPerLaunch = 1024;   // pairs carried in one kernel parameter block
+
+// Records a message for pa_last_error() and returns `code`.
+int fail(int code, const char* fmt, ...);
+void clear_error();
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* ws_ml;      // [B][Hkv][max_parts][G][2]  (m, l) per partition
+  float* ws_acc;     // [B][Hkv][max_parts][G][D]  unnormalised partition outputs
+  int* ws_count;     // [B][Hkv]  partitions finished (returned to 0 by the merging CTA)
+  int* dev_error;
+  int max_blocks_per_seq;
+  int max_context_len;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int num_blocks;
+  int part_blocks;   // blocks per split-KV partition
+  int max_parts;     // partitions per sequence the grid covers
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+struct DecodeLayout {
+  int part_blocks;
+  int max_parts;
+  size_t count_off, ml_off, acc_off, bytes;
+};
+
+// Workspace layout for a decode call (bytes == 0 when no sequence can split).
+int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                  int max_context_len, int partition_tokens, DecodeLayout* lay);
+
+cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
+                                cudaStream_t stream);
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, int64_t key_stride,
+                                     int64_t value_stride, void* k_cache, void* v_cache,
+                                     const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int num_blocks,
+                                     int* dev_error, cudaStream_t stream);
+
+struct CopyPairs {
+  int32_t src[kMaxCopyPairsPerLaunch];
+  int32_t dst[kMaxCopyPairsPerLaunch];
+};
+
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const CopyPairs& pairs, int n,
+                               int64_t block_bytes, cudaStream_t stream);
+
+}  // namespace pa

@@ -1,0 +1,216 @@
+"""Drives decode steps of a workload through libpa (block manager + kernels).
+
+The order of a step is the method's: the block manager hands out the new
+tokens' slots (and copy-on-write pairs), shared blocks are copied, the new
+tokens' keys and values are written into their slots, and decode attention
+reads the cache through the block tables ("PagedAttention and Continuous
+Batching", "Pages, from operating systems"; "PagedAttention: The vLLM Paper",
+"Implementation Essentials").
+
+Two kinds of workloads are supported, matching ``workloads.configs``:
+  * independent sequences: sequence s holds ctx_s - 1 earlier tokens (written
+    with pa_reshape_and_cache once, at set-up); each step writes token ctx_s - 1
+    and decodes over ctx_s tokens;
+  * prompts forked into samples: each prompt is written once and forked; the
+    step applies the samples' copy-on-write pairs, writes their own tokens and
+    decodes every sample. With ``duplicate=True`` every sample instead gets a
+    private copy of the prompt (same logical sequences, no sharing).
+
+The pool is allocated once, at set-up, with PyTorch; steps allocate nothing.
+Re-running a step rewrites the same slots with the same values, so steps can be
+repeated for timing.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from workloads import gen
+
+from . import _lib as L
+
+_TORCH_DTYPE = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def _to_dev(bits: np.ndarray, dtype: str, device) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits)).view(_TORCH_DTYPE[dtype])
+    return t.to(device, non_blocking=False)
+
+
+class DecodeRunner:
+    def __init__(self, wl, device="cuda", partition_tokens=None, duplicate=False):
+        self.wl = wl
+        self.duplicate = duplicate
+        self.device = torch.device(device)
+        self.dtype = _TORCH_DTYPE[wl.dtype]
+        self.partition_tokens = wl.partition_tokens if partition_tokens is None else partition_tokens
+        shape = (wl.num_blocks, wl.num_kv_heads, wl.block_size, wl.head_dim)
+        self.k_cache = torch.zeros(shape, dtype=self.dtype, device=self.device)
+        self.v_cache = torch.zeros(shape, dtype=self.dtype, device=self.device)
+        self.bm = L.BlockManager(wl.num_blocks, wl.block_size, wl.free_order)
+        self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.prefill_slots = []
+        if wl.kind == "shared_prefix":
+            self._setup_shared()
+        else:
+            self._setup_decode()
+        self.max_blocks = wl.max_blocks_per_seq
+        self.block_tables_host = self.bm.block_tables(range(wl.num_seqs), self.max_blocks)
+        self.block_tables = torch.from_numpy(self.block_tables_host).to(self.device)
+        self.context_lens_host = wl.context_lens.astype(np.int32)
+        self.context_lens = torch.from_numpy(self.context_lens_host).to(self.device)
+        self.q_host = gen.query_bits(wl.seed, wl.num_seqs, wl.num_q_heads, wl.head_dim, wl.dtype)
+        self.q = _to_dev(self.q_host, wl.dtype, self.device)
+        self.out = torch.empty_like(self.q)
+        self.workspace = L.decode_workspace(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                            wl.head_dim, wl.max_context_len,
+                                            self.partition_tokens, self.device)
+        torch.cuda.synchronize(self.device)
+
+    # -- set-up -----------------------------------------------------------------
+    def _write(self, k_bits, v_bits, slots):
+        if len(slots) == 0:
+            return
+        k = _to_dev(k_bits, self.wl.dtype, self.device)
+        v = _to_dev(v_bits, self.wl.dtype, self.device)
+        s = torch.from_numpy(np.asarray(slots, np.int64)).to(self.device)
+        L.pa_reshape_and_cache(k, v, self.k_cache, self.v_cache, s, self.dev_error)
+
+    def _setup_decode(self):
+        wl = self.wl
+        ctx = wl.context_lens.astype(np.int64)
+        step_k, step_v = [], []
+        chunk = 16
+        for first in range(0, wl.num_seqs, chunk):
+            seqs = list(range(first, min(wl.num_seqs, first + chunk)))
+            kvs = gen.many_seq_kv_bits(wl.seed, seqs, ctx[seqs], wl.num_kv_heads, wl.head_dim,
+                                       wl.dtype)
+            for s, (kb, vb) in zip(seqs, kvs):
+                n = int(ctx[s]) - 1
+                slots = self.bm.add_seq(s, n)
+                self._write(kb[:n], vb[:n], slots)
+                self.prefill_slots.append(slots)
+                step_k.append(kb[n])
+                step_v.append(vb[n])
+        slots = []
+        for s in range(wl.num_seqs):
+            sl, pairs = self.bm.append_slots(s, 1)
+            assert len(pairs) == 0
+            slots.append(sl)
+        self.step_slots_host = np.concatenate(slots).astype(np.int64)
+        self.cow_pairs = np.zeros((0, 2), np.int64)
+        self.step_k_host = np.stack(step_k)
+        self.step_v_host = np.stack(step_v)
+        self._finish_step_inputs()
+
+    def _setup_shared(self):
+        wl = self.wl
+        S, P, Lp = wl.samples, wl.num_prompts, wl.prompt_len
+        prompts = gen.many_seq_kv_bits(wl.seed, range(P), [Lp] * P, wl.num_kv_heads, wl.head_dim,
+                                       wl.dtype)
+        for p in range(P):
+            owners = [p * S + i for i in range(S)] if self.duplicate else [p * S]
+            for seq in owners:
+                slots = self.bm.add_seq(seq, Lp)
+                self._write(prompts[p][0], prompts[p][1], slots)
+                self.prefill_slots.append(slots)
+            if not self.duplicate:
+                for i in range(1, S):
+                    self.bm.fork(p * S, p * S + i)
+        slots, pairs, ks, vs = [], [], [], []
+        for seq in range(P * S):
+            n = int(wl.own_lens[seq])
+            if n == 0:
+                continue
+            sl, cow = self.bm.append_slots(seq, n)
+            k, v = gen.own_token_kv_bits(wl.seed, seq, n, wl.num_kv_heads, wl.head_dim, wl.dtype)
+            slots.append(sl)
+            pairs.append(cow)
+            ks.append(k)
+            vs.append(v)
+        self.step_slots_host = np.concatenate(slots).astype(np.int64) if slots else \
+            np.zeros(0, np.int64)
+        self.cow_pairs = np.concatenate(pairs).astype(np.int64).reshape(-1, 2) if pairs else \
+            np.zeros((0, 2), np.int64)
+        shp = (0, wl.num_kv_heads, wl.head_dim)
+        self.step_k_host = np.concatenate(ks) if ks else np.zeros(shp, np.uint16)
+        self.step_v_host = np.concatenate(vs) if vs else np.zeros(shp, np.uint16)
+        self._finish_step_inputs()
+
+    def _finish_step_inputs(self):
+        self.step_k = _to_dev(self.step_k_host, self.wl.dtype, self.device)
+        self.step_v = _to_dev(self.step_v_host, self.wl.dtype, self.device)
+        self.step_slots = torch.from_numpy(self.step_slots_host).to(self.device)
+
+    # -- the step ---------------------------------------------------------------
+    def copy_blocks(self):
+        if len(self.cow_pairs):
+            L.pa_copy_blocks(self.k_cache, self.v_cache, self.cow_pairs)
+
+    def reshape_and_cache(self):
+        if len(self.step_slots_host):
+            L.pa_reshape_and_cache(self.step_k, self.step_v, self.k_cache, self.v_cache,
+                                   self.step_slots, self.dev_error)
+
+    def decode(self, out=None, partition_tokens=None):
+        out = self.out if out is None else out
+        pt = self.partition_tokens if partition_tokens is None else partition_tokens
+        ws = self.workspace
+        if pt != self.partition_tokens:
+            ws = L.decode_workspace(self.wl.num_seqs, self.wl.num_q_heads, self.wl.num_kv_heads,
+                                    self.wl.head_dim, self.wl.max_context_len, pt, self.device)
+        L.pa_paged_decode(out, self.q, self.k_cache, self.v_cache, self.block_tables,
+                          self.context_lens, self.wl.max_context_len, self.wl.scale, pt, ws,
+                          self.dev_error)
+        return out
+
+    def step(self):
+        """One decode step: copy-on-write copies, cache writes, decode attention."""
+        self.copy_blocks()
+        self.reshape_and_cache()
+        return self.decode()
+
+    def launches_per_step(self) -> int:
+        return int(len(self.cow_pairs) > 0) * -(-len(self.cow_pairs) // 1024) + \
+            int(len(self.step_slots_host) > 0) + 1
+
+    def error_bits(self) -> int:
+        return int(self.dev_error.item())
+
+
+class HostStep:
+    """One step fed from pinned host buffers and read back to the host.
+
+    Every call copies the step's inputs (queries, new keys/values, slot
+    mapping, block tables, context lengths) host -> device, runs the step's
+    kernels, and copies the attention output device -> host, all on the
+    current stream.
+    """
+
+    def __init__(self, runner: DecodeRunner):
+        r = self.r = runner
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+        self.h_q = pin(r.q_host).view(r.dtype)
+        self.h_k = pin(r.step_k_host).view(r.dtype)
+        self.h_v = pin(r.step_v_host).view(r.dtype)
+        self.h_slots = pin(r.step_slots_host)
+        self.h_tables = pin(r.block_tables_host)
+        self.h_ctx = pin(r.context_lens_host)
+        self.h_out = torch.empty(r.out.shape, dtype=r.dtype).pin_memory()
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in
+                             (self.h_q, self.h_k, self.h_v, self.h_slots, self.h_tables,
+                              self.h_ctx))
+        self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
+
+    def __call__(self):
+        r = self.r
+        r.q.copy_(self.h_q, non_blocking=True)
+        r.step_k.copy_(self.h_k, non_blocking=True)
+        r.step_v.copy_(self.h_v, non_blocking=True)
+        r.step_slots.copy_(self.h_slots, non_blocking=True)
+        r.block_tables.copy_(self.h_tables, non_blocking=True)
+        r.context_lens.copy_(self.h_ctx, non_blocking=True)
+        r.step()
+        self.h_out.copy_(r.out, non_blocking=True)
+        return self.h_out
