@@ -101,59 +101,93 @@ _REASONS = {
 
 
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+    """SM clock and clock-event reasons sampled every 2 ms through NVML (read-only)
+    while a region runs; falls back to ``nvidia-smi -lms 100`` without NVML."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.stop = threading.Event()
         self.thread = None
+        self.proc = None
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def _poll(self, h):
+        import pynvml
+        while not self.stop.is_set():
+            try:
+                mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(mhz), int(bits)))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __enter__(self):
-        cmd = ["nvidia-smi", "-i", str(self.gpu),
-               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-               "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            import pynvml
+            h = self._nvml_handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._poll, args=(h,), daemon=True)
+            self.thread.start()
+        except Exception:
+            self._start_smi()
+        return self
+
+    def _start_smi(self):
+        cmd = ["nvidia-smi", "-i", str(self.dev.index or 0),
+               "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "100"]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
-        return self
 
-    def _read(self):
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.split(",")]
+            try:
+                self.max_mhz = float(parts[1])
+                bits = int(parts[2], 16) if parts[2].startswith("0x") else int(parts[2])
+                self.samples.append((float(parts[0]), bits))
+            except (ValueError, IndexError):
+                continue
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self.thread is not None:
-                self.thread.join(timeout=2)
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 4:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-                bits = int(parts[3], 16) if parts[3].startswith("0x") else int(parts[3])
-            except ValueError:
-                continue
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        sm = [m for m, _ in self.samples]
+        reasons = set()
+        for _, bits in self.samples:
             for b, name in _REASONS.items():
                 if bits & b and name != "gpu_idle":
                     reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
@@ -210,15 +244,21 @@ def _barrier(world: int):
         dist.barrier()
 
 
-def rank_workload(name: str, rank: int):
-    """The named workload; rank r > 0 gets an independent batch (seed shifted)."""
+def rank_workload(name: str, rank: int, num_seqs: int = 0, num_blocks: int = 0):
+    """The named workload; rank r > 0 gets an independent batch (seed shifted).
+
+    ``num_seqs``/``num_blocks`` (profiling only) keep the first sequences of the
+    batch in a smaller pool; the workload name then says so."""
     import workloads
     from workloads import configs
     if rank == 0:
-        return workloads.workload(name)
-    base = workloads.workload(name)
-    fn = configs.WORKLOADS[name]
-    return fn(seed=base.seed + 7919 * rank)
+        wl = workloads.workload(name)
+    else:
+        base = workloads.workload(name)
+        wl = configs.WORKLOADS[name](seed=base.seed + 7919 * rank)
+    if num_seqs or num_blocks:
+        wl = configs.truncated(wl, num_seqs or wl.num_seqs, num_blocks or wl.num_blocks)
+    return wl
 
 
 # --------------------------------------------------------------------------
@@ -337,7 +377,7 @@ def run_ours(args):
     pabuild.build()
     from paged_kv_cache_352_b200.runner import DecodeRunner, HostStep
 
-    wl = rank_workload(args.workload, rank)
+    wl = rank_workload(args.workload, rank, args.num_seqs, args.num_blocks)
     r = DecodeRunner(wl, device=device,
                      partition_tokens=args.partition_tokens if args.partition_tokens >= 0 else None)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -351,17 +391,9 @@ def run_ours(args):
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    gpu_index = device.index if device.index is not None else 0
-    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if visible:
-        try:
-            gpu_index = int(visible.split(",")[gpu_index])
-        except (ValueError, IndexError):
-            pass
     _barrier(world)
     torch.cuda.synchronize(device)
-    with ClockSampler(gpu_index) as clocks:
-        time.sleep(0.3)
+    with ClockSampler(device) as clocks:
         for k in range(K):
             flush.fill_(k & 0xFF)
             ev[k][0].record(stream)
@@ -453,13 +485,17 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--partition-tokens", type=int, default=-1,
                     help="split-KV partition size (default: the workload's / library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="profiling only: keep the first N sequences of the batch")
+    ap.add_argument("--num-blocks", type=int, default=0,
+                    help="profiling only: pool size for the truncated batch")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     args = ap.parse_args(argv)

@@ -186,6 +186,21 @@ SMALL_WORKLOADS = {
 }
 
 
+def truncated(wl, num_seqs: int, num_blocks: int):
+    """The first ``num_seqs`` sequences of an independent-sequence workload in a pool
+    of ``num_blocks`` blocks (a smaller case with the same per-sequence shapes)."""
+    if wl.kind != "decode":
+        raise ValueError("only independent-sequence workloads can be truncated")
+    ctx = wl.context_lens[:num_seqs]
+    need = int(sum(-(-int(c) // wl.block_size) for c in ctx))
+    if num_blocks < need:
+        raise ValueError(f"{num_blocks} blocks cannot hold {need}")
+    order = _meta_rng(wl.seed).permutation(num_blocks)
+    return DecodeWorkload(f"{wl.name}[:{num_seqs}]/{num_blocks}blk", wl.seed, num_seqs,
+                          wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, ctx,
+                          num_blocks, order, wl.partition_tokens, wl.block_size)
+
+
 def workload(name: str, small: bool = False):
     table = SMALL_WORKLOADS if small else WORKLOADS
     if name not in table:
