@@ -164,6 +164,40 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
                     size_t workspace_bytes, int* dev_error, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_paged_decode_noalloc — pa_paged_decode without a caller-supplied workspace.
+ *
+ * The paper has no counterpart to this call. It is a convenience of this
+ * library for callers that cannot allocate device memory: for example a plugin
+ * whose host runtime owns every allocation, or a latency-critical loop that must
+ * never reach cudaMalloc, which may synchronise the device.
+ *
+ * The result is the same as pa_paged_decode with the same arguments. The
+ * split-KV scratch comes from one array of PA_NOALLOC_WORKSPACE_BYTES compiled
+ * into the library. Every GPU that loads the library holds that array until the
+ * process exits.
+ *
+ * The call allocates nothing:
+ *   - The first call on each device looks up the array's device address and
+ *     caches it. Make that first call, with the device current, before any
+ *     stream capture on that device.
+ *   - Each call clears the array's merge counters with an async memset on
+ *     `stream`, then launches the decode kernel.
+ *   - All calls share the one array, so calls whose kernels overlap on the GPU
+ *     race. Issue them on one stream or order them with events.
+ *   - A batch whose scratch (pa_paged_decode_workspace_size) exceeds the array
+ *     returns PA_ERR_UNSUPPORTED and launches nothing. A larger partition_tokens,
+ *     or fewer sequences per call, reduces the scratch needed.
+ * ------------------------------------------------------------------------- */
+#define PA_NOALLOC_WORKSPACE_BYTES ((size_t)16 << 20) /* 16 MiB */
+
+int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int max_context_len,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float scale, int partition_tokens, int* dev_error,
+                            int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Host block manager.
  *
  * "A pre-allocated memory pool, block allocation/reclamation, and refcounts

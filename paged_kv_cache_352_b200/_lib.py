@@ -57,6 +57,9 @@ _SIGS = {
     "pa_paged_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_int, ctypes.c_float, _c_int, _vp,
                                  ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_paged_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
+                                         _c_int, _vp, _c_int, _vp]),
     "pa_bm_create": (_c_int, [_c_int, _c_int, _vp, ctypes.POINTER(_vp)]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_c_int, [_vp, _c_i64, _c_int, _vp]),
@@ -224,6 +227,35 @@ def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_co
         block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32), B,
         int(max_context_len), hq, hkv, d, bs, nb, float(scale), int(partition_tokens),
         _dev_ptr(workspace, "workspace"), ws_bytes,
+        _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
+
+
+NOALLOC_WORKSPACE_BYTES = 16 << 20
+
+
+def pa_paged_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
+                            max_context_len, scale, partition_tokens=0, dev_error=None,
+                            stream=None):
+    """Like ``pa_paged_decode`` but without a workspace argument.
+
+    For callers that cannot allocate device memory: the split-KV scratch comes
+    from a fixed array built into libpa (``NOALLOC_WORKSPACE_BYTES`` per GPU).
+    Calls share that array, so calls that overlap on the GPU must not be issued
+    (use one stream). Batches that need more scratch raise ``PAError``.
+    """
+    torch = _torch()
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    B, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or out.dtype != k_cache.dtype or q.dtype != k_cache.dtype:
+        raise PAError(PA_ERR_INVALID_ARG, "q/out must be [B, num_q_heads, head_dim] in the "
+                                          "cache's dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
+    _check(lib().pa_paged_decode_noalloc(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32), B,
+        int(max_context_len), hq, hkv, d, bs, nb, float(scale), int(partition_tokens),
         _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
 
 
