@@ -453,7 +453,7 @@ def run_ours(args):
         "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": wl.name, **{k: v for k, v in wl.describe().items()
                                            if k != "workload"},
-                   "partition_tokens": r.partition_tokens or 512,
+                   "partition_tokens": r.partition_tokens,
                    "l2": "flushed between steps (256 MiB write), outside the timed events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),

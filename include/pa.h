@@ -140,7 +140,10 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
  *   max_context_len    host-known upper bound of context_lens (sizes the grid
  *                      without a device read); longer sequences are flagged
  *   scale              softmax scale, usually 1/sqrt(head_dim)
- *   partition_tokens   0 = library default (512); else a multiple of block_size
+ *   partition_tokens   a multiple of block_size, or 0 for the library's choice:
+ *                      no split when num_seqs * num_kv_heads >= 1024, otherwise
+ *                      partitions of at least 512 tokens, as many as bring the
+ *                      number of (sequence, KV head, partition) units to ~1024
  *   workspace          device scratch of pa_paged_decode_workspace_size() bytes,
  *                      ZERO-FILLED before its first use; every completed call
  *                      leaves it zero-filled again, so it can be reused without

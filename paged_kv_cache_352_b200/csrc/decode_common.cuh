@@ -1,0 +1,114 @@
+// Shared tail of the paged-decode kernels: merging per-warp softmax states
+// into the CTA's result, and the split-KV merge across partitions.
+#pragma once
+
+#include <math.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+// After the main loop every warp w has left, in shared memory,
+//   red_m[w][g], red_l[w][g]   its running max (base 2) and sum of exponentials
+//   red_acc[w][g][D]           its unnormalised output rows
+// for the G query heads of this CTA's KV head. This merges them by rescaling
+// to the common maximum. A sequence with a single partition writes `out`
+// directly. Otherwise the CTA stores its partition state in the workspace, and
+// the CTA that completes the sequence's last partition merges all partitions
+// in logical order and returns the counter to zero.
+// `smem` (>= max_parts * G floats) is scratch once red_* have been read.
+template <typename T, int D, int G, int WARPS>
+__device__ __forceinline__ void finish_partition(const DecodeArgs& a, unsigned char* smem,
+                                                 const float* red_m, const float* red_l,
+                                                 const float* red_acc, int s, int kvh, int part,
+                                                 int nparts, T* out_rows) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool split = nparts > 1;
+  const size_t unit = (size_t)s * a.num_kv_heads + kvh;
+  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
+    const int g = item / D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_m[w * G + g]);
+    // M is finite unless every block of the partition was skipped as out of range
+    const float Mref = M == -INFINITY ? 0.f : M;
+    float L = 0.f, A = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      const float sc = exp2f(red_m[w * G + g] - Mref);
+      L = fmaf(sc, red_l[w * G + g], L);
+      A = fmaf(sc, red_acc[(w * G) * D + item], A);
+    }
+    if (!split) {
+      out_rows[item] = Storage<T>::from_f32(L > 0.f ? A / L : 0.f);
+    } else {
+      const size_t row = (unit * a.max_parts + part) * G + g;
+      a.ws_acc[row * D + (item % D)] = A;
+      if (item % D == 0) {
+        a.ws_ml[row * 2] = M;
+        a.ws_ml[row * 2 + 1] = L;
+      }
+    }
+  }
+  if (!split) return;
+
+  // ---- split-KV: the last partition to finish merges all of them.
+  // The barrier makes every thread's partial-result stores visible to thread 0,
+  // whose gpu-scope acq_rel add then publishes them (release is cumulative) and,
+  // in the last CTA, acquires the other partitions' results before the barrier
+  // hands them to the rest of the CTA. One fence per CTA instead of one per thread.
+  __syncthreads();
+  __shared__ int is_last;
+  if (threadIdx.x == 0) {
+    const int prev = atom_add_acq_rel_gpu(a.ws_count + unit, 1);
+    is_last = (prev == nparts - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+
+  // per-(partition, head) weights exp2(m_p - M) / L, staged in shared memory
+  float* wts = reinterpret_cast<float*>(smem);  // [nparts][G]
+  __shared__ float headM[G], headL[G];
+  const float* ml = a.ws_ml + unit * a.max_parts * G * 2;
+  for (int g = warp; g < G; g += WARPS) {
+    float M = -INFINITY;
+    for (int p = lane; p < nparts; p += 32) M = fmaxf(M, __ldcg(ml + (p * G + g) * 2));
+#pragma unroll
+    for (int mask = 16; mask > 0; mask >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, mask));
+    if (M == -INFINITY) M = 0.f;
+    float L = 0.f;
+    for (int p = lane; p < nparts; p += 32)
+      L += exp2f(__ldcg(ml + (p * G + g) * 2) - M) * __ldcg(ml + (p * G + g) * 2 + 1);
+#pragma unroll
+    for (int mask = 16; mask > 0; mask >>= 1) L += __shfl_xor_sync(0xffffffffu, L, mask);
+    if (lane == 0) {
+      headM[g] = M;
+      headL[g] = L;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nparts * G; idx += blockDim.x) {
+    const int g = idx % G;
+    wts[idx] = headL[g] > 0.f ? exp2f(__ldcg(ml + idx * 2) - headM[g]) / headL[g] : 0.f;
+  }
+  __syncthreads();
+  const float* accp = a.ws_acc + unit * a.max_parts * G * D;
+  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
+    const int g = item / D;
+    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+    int p = 0;
+    for (; p + 4 <= nparts; p += 4) {
+      o0 = fmaf(wts[(p + 0) * G + g], __ldcg(accp + (size_t)(p + 0) * G * D + item), o0);
+      o1 = fmaf(wts[(p + 1) * G + g], __ldcg(accp + (size_t)(p + 1) * G * D + item), o1);
+      o2 = fmaf(wts[(p + 2) * G + g], __ldcg(accp + (size_t)(p + 2) * G * D + item), o2);
+      o3 = fmaf(wts[(p + 3) * G + g], __ldcg(accp + (size_t)(p + 3) * G * D + item), o3);
+    }
+    for (; p < nparts; ++p) o0 = fmaf(wts[p * G + g], __ldcg(accp + (size_t)p * G * D + item), o0);
+    out_rows[item] = Storage<T>::from_f32((o0 + o1) + (o2 + o3));
+  }
+  if (threadIdx.x == 0) a.ws_count[unit] = 0;
+}
+
+}  // namespace pa

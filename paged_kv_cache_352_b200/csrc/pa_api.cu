@@ -51,16 +51,31 @@ int cuda_status(cudaError_t e, const char* what) {
 
 }  // namespace
 
+int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks) {
+  // One CTA per (sequence, KV head) streams best: every extra partition costs
+  // its CTA's pipeline ramp and a merge. Split only when the batch alone cannot
+  // give the GPU enough CTAs, into as many partitions as bring it to
+  // kSplitTargetUnits, never below kMinPartitionBlocks blocks each.
+  const long long units = (long long)num_seqs * num_kv_heads;
+  if (max_blocks < 1) return 1;
+  if (units >= kSplitTargetUnits) return max_blocks;
+  const long long parts = (kSplitTargetUnits + units - 1) / (units > 0 ? units : 1);
+  long long pb = (max_blocks + parts - 1) / parts;
+  if (pb < kMinPartitionBlocks) pb = kMinPartitionBlocks;
+  return (int)(pb < max_blocks ? pb : max_blocks);
+}
+
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                   int max_context_len, int partition_tokens, DecodeLayout* lay) {
-  if (partition_tokens == 0) partition_tokens = kDefaultPartitionTokens;
   if (partition_tokens < 0 || partition_tokens % kBlockSize != 0)
     return fail(PA_ERR_INVALID_ARG, "partition_tokens %d: must be 0 or a positive multiple of %d",
                 partition_tokens, kBlockSize);
   if (max_context_len < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len must be >= 0");
   const int group = num_q_heads / num_kv_heads;
-  const int part_blocks = partition_tokens / kBlockSize;
   const int max_blocks = (max_context_len + kBlockSize - 1) / kBlockSize;
+  const int part_blocks = partition_tokens == 0
+                              ? default_partition_blocks(num_seqs, num_kv_heads, max_blocks)
+                              : partition_tokens / kBlockSize;
   int max_parts = (max_blocks + part_blocks - 1) / part_blocks;
   if (max_parts < 1) max_parts = 1;
   if (max_parts > 65535)

@@ -123,6 +123,14 @@ struct Storage<__nv_bfloat16> {
   }
 };
 
+// gpu-scope fetch-and-add with acquire + release semantics.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void report(int* dev_error, int bit) {
   if (dev_error != nullptr) atomicOr(dev_error, bit);
 }

@@ -38,7 +38,10 @@
 #include <math.h>
 
 #include <atomic>
+#include <cstdlib>
+#include <cstring>
 
+#include "decode_common.cuh"
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -341,102 +344,20 @@ __global__ void __launch_bounds__(WARPS * 32)
   }
   __syncthreads();
 
-  const bool split = nparts > 1;
-  const size_t unit = (size_t)s * a.num_kv_heads + kvh;
-  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
-    const int g = item / D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_m[w * G + g]);
-    // M is finite unless every block of the partition was skipped as out of range
-    const float Mref = M == -INFINITY ? 0.f : M;
-    float L = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) {
-      const float sc = exp2f(red_m[w * G + g] - Mref);
-      L = fmaf(sc, red_l[w * G + g], L);
-      A = fmaf(sc, red_acc[(w * G) * D + item], A);
-    }
-    if (!split) {
-      out_rows[item] = Storage<T>::from_f32(L > 0.f ? A / L : 0.f);
-    } else {
-      const size_t row = (unit * a.max_parts + part) * G + g;
-      a.ws_acc[row * D + (item % D)] = A;
-      if (item % D == 0) {
-        a.ws_ml[row * 2] = M;
-        a.ws_ml[row * 2 + 1] = L;
-      }
-    }
-  }
-  if (!split) return;
-
-  // ---- split-KV: the last partition to finish merges all of them
-  __threadfence();
-  __syncthreads();
-  __shared__ int is_last;
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.ws_count + unit, 1);
-    is_last = (prev == nparts - 1);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-
-  // per-(partition, head) weights exp2(m_p - M) / L, staged in shared memory
-  float* wts = reinterpret_cast<float*>(smem);  // [nparts][G]
-  __shared__ float headM[G], headL[G];
-  const float* ml = a.ws_ml + unit * a.max_parts * G * 2;
-  for (int g = warp; g < G; g += WARPS) {
-    float M = -INFINITY;
-    for (int p = lane; p < nparts; p += 32) M = fmaxf(M, __ldcg(ml + (p * G + g) * 2));
-#pragma unroll
-    for (int mask = 16; mask > 0; mask >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, mask));
-    if (M == -INFINITY) M = 0.f;
-    float L = 0.f;
-    for (int p = lane; p < nparts; p += 32)
-      L += exp2f(__ldcg(ml + (p * G + g) * 2) - M) * __ldcg(ml + (p * G + g) * 2 + 1);
-#pragma unroll
-    for (int mask = 16; mask > 0; mask >>= 1) L += __shfl_xor_sync(0xffffffffu, L, mask);
-    if (lane == 0) {
-      headM[g] = M;
-      headL[g] = L;
-    }
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < nparts * G; idx += blockDim.x) {
-    const int g = idx % G;
-    wts[idx] = headL[g] > 0.f ? exp2f(__ldcg(ml + idx * 2) - headM[g]) / headL[g] : 0.f;
-  }
-  __syncthreads();
-  const float* accp = a.ws_acc + unit * a.max_parts * G * D;
-  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
-    const int g = item / D;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-    int p = 0;
-    for (; p + 4 <= nparts; p += 4) {
-      o0 = fmaf(wts[(p + 0) * G + g], __ldcg(accp + (size_t)(p + 0) * G * D + item), o0);
-      o1 = fmaf(wts[(p + 1) * G + g], __ldcg(accp + (size_t)(p + 1) * G * D + item), o1);
-      o2 = fmaf(wts[(p + 2) * G + g], __ldcg(accp + (size_t)(p + 2) * G * D + item), o2);
-      o3 = fmaf(wts[(p + 3) * G + g], __ldcg(accp + (size_t)(p + 3) * G * D + item), o3);
-    }
-    for (; p < nparts; ++p) o0 = fmaf(wts[p * G + g], __ldcg(accp + (size_t)p * G * D + item), o0);
-    out_rows[item] = Storage<T>::from_f32((o0 + o1) + (o2 + o3));
-  }
-  if (threadIdx.x == 0) a.ws_count[unit] = 0;
+  finish_partition<T, D, G, WARPS>(a, smem, red_m, red_l, red_acc, s, kvh, part, nparts,
+                                   out_rows);
 }
 
-constexpr int kWarps = 4;
-constexpr int kStages = 3;
 constexpr size_t kDecodeSmemLimit = 200 * 1024;
 constexpr int kMaxDevices = 64;
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int WARPS, int STAGES>
 cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
-  using Plan = SmemPlan<kWarps, kStages, D, G>;
+  using Plan = SmemPlan<WARPS, STAGES, D, G>;
   const size_t wts_bytes = (size_t)a.max_parts * G * sizeof(float);
   const size_t smem = Plan::kFixed > wts_bytes ? Plan::kFixed : wts_bytes;
   if (smem > kDecodeSmemLimit) return cudaErrorInvalidConfiguration;
-  auto kern = paged_decode_kernel<T, D, G, kWarps, kStages>;
+  auto kern = paged_decode_kernel<T, D, G, WARPS, STAGES>;
   // The opt-in limit is a ceiling, not a reservation: set it once per device.
   static std::atomic<bool> ready[kMaxDevices];
   int dev = 0;
@@ -450,25 +371,67 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
     ready[dev].store(true, std::memory_order_release);
   }
   dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
-  kern<<<grid, kWarps * 32, smem, stream>>>(a);
+  kern<<<grid, WARPS * 32, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+// Warps per CTA x stages per warp. The default is 4 x 3; PA_DECODE_TILE="WxS"
+// selects another built shape for A/B measurements (4x2, 2x3, 2x4, 8x2).
+int tile_variant() {
+  static const int v = [] {
+    const char* e = getenv("PA_DECODE_TILE");
+    if (!e) return 0;
+    if (!strcmp(e, "4x2")) return 1;
+    if (!strcmp(e, "2x3")) return 2;
+    if (!strcmp(e, "2x4")) return 3;
+    if (!strcmp(e, "8x2")) return 4;
+    return 0;
+  }();
+  return v;
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_tiles(const DecodeArgs& a, cudaStream_t stream) {
+  switch (tile_variant()) {
+    case 1: return launch_typed<T, D, G, 4, 2>(a, stream);
+    case 2: return launch_typed<T, D, G, 2, 3>(a, stream);
+    case 3: return launch_typed<T, D, G, 2, 4>(a, stream);
+    case 4: return launch_typed<T, D, G, 8, 2>(a, stream);
+    default: return launch_typed<T, D, G, 4, 3>(a, stream);
+  }
 }
 
 template <typename T, int D>
 cudaError_t launch_group(const DecodeArgs& a, int group, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_typed<T, D, 1>(a, stream);
-    case 2: return launch_typed<T, D, 2>(a, stream);
-    case 4: return launch_typed<T, D, 4>(a, stream);
-    case 8: return launch_typed<T, D, 8>(a, stream);
+    case 1: return launch_tiles<T, D, 1>(a, stream);
+    case 2: return launch_typed<T, D, 2, 4, 3>(a, stream);
+    case 4: return launch_typed<T, D, 4, 4, 3>(a, stream);
+    case 8: return launch_typed<T, D, 8, 4, 3>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
+// Which arithmetic path serves a query-head group: tensor cores from G = 4 up
+// (the q.K / P.V tiles are then real contractions), CUDA cores below.
+// PA_DECODE_PATH=cuda_cores or =tensor overrides the choice for A/B measurements.
+bool use_tensor_path(int group) {
+  static const int forced = [] {
+    const char* e = getenv("PA_DECODE_PATH");
+    if (e && !strcmp(e, "cuda_cores")) return 0;
+    if (e && !strcmp(e, "tensor")) return 1;
+    return -1;
+  }();
+  if (group < 2) return false;
+  if (forced >= 0) return forced == 1;
+  return group >= 4;
+}
+
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
                                 cudaStream_t stream) {
+  if (use_tensor_path(group)) return launch_paged_decode_mma(a, head_dim, group, dtype, stream);
   if (dtype == PA_F16) {
     if (head_dim == 64) return launch_group<__half, 64>(a, group, stream);
     if (head_dim == 128) return launch_group<__half, 128>(a, group, stream);

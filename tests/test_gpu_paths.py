@@ -1,0 +1,21 @@
+"""Both decode arithmetic paths (CUDA cores and tensor cores) against the oracle
+for every supported group size, head_dim and storage type, with NaN patterns
+planted in the unused slots of every partly filled block."""
+
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("path", ["cuda_cores", "tensor"])
+def test_decode_path_parity(path):
+    env = dict(os.environ, PA_DECODE_PATH=path)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "path_check.py")], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert "ok" in r.stdout
