@@ -11,12 +11,15 @@ Metric: KV-read GB/s (algorithmic bytes of the step / device time of the
 step; % of measured HBM peak alongside) and decode tokens/s.
 
 Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events
-on the launching stream, with an L2 flush (a 256 MiB write, more than the
-126 MB L2) between steps outside the events; a barrier + synchronize on both
-sides of the timed region; max over ranks. The decode kernel alone is timed
-the same way for the roofline. ``e2e`` repeats the step through the same
-C interface fed from pinned host buffers: every step copies its inputs
-host -> device and its output device -> host inside the timed region.
+on the launching stream; a barrier + synchronize on both sides of the timed
+region; max over ranks. Workloads whose inputs exceed 4x the 126 MB L2 run
+without a flush (a cyclic scan larger than the cache reuses nothing); smaller
+ones flush L2 between steps, outside the events, by reading a 256 MiB buffer
+(a write flush would leave dirty lines whose write-back the next kernel pays).
+The decode kernel alone is timed the same way for the roofline. ``e2e``
+repeats the step through the same C interface fed from pinned host buffers:
+every step copies its inputs host -> device and its output device -> host
+inside the timed region.
 
 Multi-GPU (torchrun, one process per GPU): the decode step has no exchange
 between GPUs, so each rank runs an independent replica with its own pool and
@@ -100,75 +103,83 @@ _REASONS = {
 }
 
 
+_NVML_POLL = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByPciBusId(sys.argv[1]) if sys.argv[1] else \
+    pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    try:
+        print(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+              pynvml.nvmlDeviceGetCurrentClocksEventReasons(h), flush=True)
+    except pynvml.NVMLError:
+        pass
+    time.sleep(0.005)
+"""
+
+
 class ClockSampler:
-    """SM clock and clock-event reasons sampled every 2 ms through NVML (read-only)
-    while a region runs; falls back to ``nvidia-smi -lms 100`` without NVML."""
+    """SM clock and clock-event reasons sampled every 5 ms through NVML (read-only)
+    by a separate process, so the sampling does not compete with the launching
+    thread; falls back to ``nvidia-smi -lms 100`` without NVML."""
 
     def __init__(self, torch_device):
         self.dev = torch_device
         self.samples = []
-        self.stop = threading.Event()
-        self.thread = None
         self.proc = None
+        self.thread = None
         self.max_mhz = None
+        self.ready = threading.Event()
 
-    def _nvml_handle(self):
-        import pynvml
+    def _bus_id(self):
         import torch
-        pynvml.nvmlInit()
-        props = torch.cuda.get_device_properties(self.dev)
         try:
-            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
-            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            p = torch.cuda.get_device_properties(self.dev)
+            return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
         except Exception:
-            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
-
-    def _poll(self, h):
-        import pynvml
-        while not self.stop.is_set():
-            try:
-                mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((float(mhz), int(bits)))
-            except Exception:
-                pass
-            time.sleep(0.002)
+            return ""
 
     def __enter__(self):
         try:
-            import pynvml
-            h = self._nvml_handle()
-            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-            self.thread = threading.Thread(target=self._poll, args=(h,), daemon=True)
-            self.thread.start()
-        except Exception:
-            self._start_smi()
-        return self
-
-    def _start_smi(self):
-        cmd = ["nvidia-smi", "-i", str(self.dev.index or 0),
-               "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
-               "--format=csv,noheader,nounits", "-lms", "100"]
+            import pynvml  # noqa: F401
+            cmd = [sys.executable, "-c", _NVML_POLL, self._bus_id(), str(self.dev.index or 0)]
+            kind = "nvml"
+        except ImportError:
+            cmd = ["nvidia-smi", "-i", str(self.dev.index or 0),
+                   "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                   "--format=csv,noheader,nounits", "-lms", "100"]
+            kind = "smi"
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
-            self.thread = threading.Thread(target=self._read_smi, daemon=True)
+            self.thread = threading.Thread(target=self._read, args=(kind,), daemon=True)
             self.thread.start()
+            self.ready.wait(timeout=20)   # the poller has started sampling
         except (OSError, ValueError):
             self.proc = None
+        return self
 
-    def _read_smi(self):
+    def _read(self, kind):
         for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
             try:
-                self.max_mhz = float(parts[1])
-                bits = int(parts[2], 16) if parts[2].startswith("0x") else int(parts[2])
-                self.samples.append((float(parts[0]), bits))
+                if kind == "nvml":
+                    parts = line.split()
+                    if parts[0] == "max":
+                        self.max_mhz = float(parts[1])
+                        continue
+                    self.samples.append((float(parts[0]), int(parts[1])))
+                else:
+                    parts = [p.strip() for p in line.split(",")]
+                    self.max_mhz = float(parts[1])
+                    bits = int(parts[2], 16) if parts[2].startswith("0x") else int(parts[2])
+                    self.samples.append((float(parts[0]), bits))
+                self.ready.set()
             except (ValueError, IndexError):
                 continue
 
     def __exit__(self, *exc):
-        self.stop.set()
+        time.sleep(0.02)  # one more sample after the region
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -205,20 +216,53 @@ def _peaks():
         return 6650.0, "fallback"
 
 
-def _traffic_for(kernel_src: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+DECODE_SOURCES = ("paged_decode_impl.cuh", "decode_policies.cuh", "decode_common.cuh",
+                  "pa_device.cuh")
+
+
+def decode_source_sha() -> str:
+    """Hash of the decode kernel's sources (ties a traffic figure to the code profiled)."""
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_352_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_for(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    on the current kernel sources for this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(workload)
-        with open(kernel_src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        sha = decode_source_sha()
     except (OSError, ValueError, AttributeError):
         return None
     if not rec or rec.get("source_sha") != sha:
         return None
     return rec.get("dram_bytes_per_launch")
+
+
+def read_stream_gbs(device, nbytes: int = 2 << 30, reps: int = 5):
+    """A read-only streaming reference: summing a 2 GiB int64 buffer (torch)."""
+    import torch
+    x = torch.ones(nbytes // 8, dtype=torch.int64, device=device)
+    x.sum()
+    torch.cuda.synchronize(device)
+    best = None
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        x.sum()
+        b.record()
+        torch.cuda.synchronize(device)
+        t = a.elapsed_time(b) / 1e3
+        best = t if best is None else min(best, t)
+    del x
+    torch.cuda.empty_cache()
+    return nbytes / best / 1e9
 
 
 def _rank_info():
@@ -380,8 +424,20 @@ def run_ours(args):
     wl = rank_workload(args.workload, rank, args.num_seqs, args.num_blocks)
     r = DecodeRunner(wl, device=device,
                      partition_tokens=args.partition_tokens if args.partition_tokens >= 0 else None)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
+    # Inputs several times larger than L2 need no flush between steps (a cyclic
+    # scan larger than the cache leaves nothing to reuse). Smaller workloads get
+    # an L2 flush that READS a buffer larger than L2: a write flush would leave
+    # dirty lines whose write-back the next kernel would pay for.
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    flush_needed = decode_bytes(wl) < 4 * l2_bytes if args.l2 == "auto" else args.l2 == "flush"
+    flush = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=device) \
+        if flush_needed else None
+    flush_sink = torch.empty(1, dtype=torch.int64, device=device)
+
+    def l2_flush():
+        if flush is not None:
+            torch.sum(flush, dim=0, out=flush_sink)
 
     for _ in range(max(3, args.warmup)):
         r.step()
@@ -395,7 +451,7 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     with ClockSampler(device) as clocks:
         for k in range(K):
-            flush.fill_(k & 0xFF)
+            l2_flush()
             ev[k][0].record(stream)
             r.copy_blocks()
             r.reshape_and_cache()
@@ -421,7 +477,7 @@ def run_ours(args):
     _barrier(world)
     torch.cuda.synchronize(device)
     for k in range(E):
-        flush.fill_(k & 0xFF)
+        l2_flush()
         ee[k][0].record(stream)
         hs()
         ee[k][1].record(stream)
@@ -435,8 +491,8 @@ def run_ours(args):
     peak, peak_kind = _peaks()
     value = world * sb / step_s / 1e9
     achieved = db / dec_s / 1e9
-    traffic = _traffic_for(os.path.join(ROOT, "paged_kv_cache_352_b200", "csrc",
-                                        "paged_decode.cu"), wl.name)
+    traffic = _traffic_for(wl.name)
+    read_ref = read_stream_gbs(device) if world == 1 else None
     csum = clocks.summary()
     launches_per_step = r.launches_per_step()
 
@@ -454,11 +510,15 @@ def run_ours(args):
         "config": {"workload": wl.name, **{k: v for k, v in wl.describe().items()
                                            if k != "workload"},
                    "partition_tokens": r.partition_tokens,
-                   "l2": "flushed between steps (256 MiB write), outside the timed events",
+                   "l2": ("flushed between steps by reading a 256 MiB buffer, outside the "
+                          "timed events" if flush_needed else
+                          f"inputs larger than L2 ({decode_bytes(wl) / 1e6:.0f} MB vs "
+                          f"{l2_bytes / 1e6:.0f} MB L2), no flush"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
         "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
+        "read_stream_ref_gbs": round(read_ref, 1) if read_ref else None,
         "decode_tokens_per_s": round(world * wl.num_seqs / step_s, 1),
         "decode_only_tokens_per_s": round(world * wl.num_seqs / dec_s, 1),
         "bytes_per_step": sb,
@@ -492,6 +552,9 @@ def main(argv=None):
     ap.add_argument("--partition-tokens", type=int, default=-1,
                     help="split-KV partition size (default: the workload's / library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--l2", choices=["auto", "flush", "none"], default="auto",
+                    help="L2 handling between steps: auto = flush (by a read) only when the "
+                         "step's inputs are smaller than 4x L2")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="profiling only: keep the first N sequences of the batch")
     ap.add_argument("--num-blocks", type=int, default=0,

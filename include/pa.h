@@ -141,9 +141,9 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
  *                      without a device read); longer sequences are flagged
  *   scale              softmax scale, usually 1/sqrt(head_dim)
  *   partition_tokens   a multiple of block_size, or 0 for the library's choice:
- *                      no split when num_seqs * num_kv_heads >= 1024, otherwise
- *                      partitions of at least 512 tokens, as many as bring the
- *                      number of (sequence, KV head, partition) units to ~1024
+ *                      partitions of at most 2048 tokens, shorter (down to 512)
+ *                      when num_seqs * num_kv_heads < 1024, so that the launch
+ *                      still has ~1024 (sequence, KV head, partition) units
  *   workspace          device scratch of pa_paged_decode_workspace_size() bytes,
  *                      ZERO-FILLED before its first use; every completed call
  *                      leaves it zero-filled again, so it can be reused without

@@ -17,9 +17,12 @@ namespace pa {
 // directly. Otherwise the CTA stores its partition state in the workspace, and
 // the CTA that completes the sequence's last partition merges all partitions
 // in logical order and returns the counter to zero.
-// `smem` (>= max_parts * G floats) is scratch once red_* have been read.
+// `wts` (>= nparts * G floats of shared memory) may alias red_*: it is written
+// only after they have been read. Every thread of the CTA must call this with
+// the same arguments; it ends with a barrier, so shared memory it used can be
+// rewritten as soon as it returns.
 template <typename T, int D, int G, int WARPS>
-__device__ __forceinline__ void finish_partition(const DecodeArgs& a, unsigned char* smem,
+__device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts,
                                                  const float* red_m, const float* red_l,
                                                  const float* red_acc, int s, int kvh, int part,
                                                  int nparts, T* out_rows) {
@@ -52,7 +55,10 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, unsigned c
       }
     }
   }
-  if (!split) return;
+  if (!split) {
+    __syncthreads();
+    return;
+  }
 
   // ---- split-KV: the last partition to finish merges all of them.
   // The barrier makes every thread's partial-result stores visible to thread 0,
@@ -66,10 +72,9 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, unsigned c
     is_last = (prev == nparts - 1);
   }
   __syncthreads();
-  if (!is_last) return;
+  if (!is_last) return;  // uniform across the CTA; the barrier above ends this call
 
-  // per-(partition, head) weights exp2(m_p - M) / L, staged in shared memory
-  float* wts = reinterpret_cast<float*>(smem);  // [nparts][G]
+  // per-(partition, head) weights exp2(m_p - M) / L, staged in shared memory [nparts][G]
   __shared__ float headM[G], headL[G];
   const float* ml = a.ws_ml + unit * a.max_parts * G * 2;
   for (int g = warp; g < G; g += WARPS) {
@@ -109,6 +114,7 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, unsigned c
     out_rows[item] = Storage<T>::from_f32((o0 + o1) + (o2 + o3));
   }
   if (threadIdx.x == 0) a.ws_count[unit] = 0;
+  __syncthreads();
 }
 
 }  // namespace pa

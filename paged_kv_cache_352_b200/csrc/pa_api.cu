@@ -52,16 +52,20 @@ int cuda_status(cudaError_t e, const char* what) {
 }  // namespace
 
 int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks) {
-  // One CTA per (sequence, KV head) streams best: every extra partition costs
-  // its CTA's pipeline ramp and a merge. Split only when the batch alone cannot
-  // give the GPU enough CTAs, into as many partitions as bring it to
-  // kSplitTargetUnits, never below kMinPartitionBlocks blocks each.
+  // A CTA streams best over a long run of blocks: every extra partition costs its
+  // CTA's pipeline ramp and a merge. Long partitions, though, leave a tail of
+  // lone CTAs at the end of the launch. Partitions are therefore capped at
+  // kMaxPartitionBlocks, and made shorter (never below kMinPartitionBlocks)
+  // when the batch alone cannot give the GPU ~kSplitTargetUnits CTAs.
   const long long units = (long long)num_seqs * num_kv_heads;
   if (max_blocks < 1) return 1;
-  if (units >= kSplitTargetUnits) return max_blocks;
-  const long long parts = (kSplitTargetUnits + units - 1) / (units > 0 ? units : 1);
-  long long pb = (max_blocks + parts - 1) / parts;
-  if (pb < kMinPartitionBlocks) pb = kMinPartitionBlocks;
+  long long pb = max_blocks;
+  if (units < kSplitTargetUnits) {
+    const long long parts = (kSplitTargetUnits + units - 1) / (units > 0 ? units : 1);
+    pb = (max_blocks + parts - 1) / parts;
+    if (pb < kMinPartitionBlocks) pb = kMinPartitionBlocks;
+  }
+  if (pb > kMaxPartitionBlocks) pb = kMaxPartitionBlocks;
   return (int)(pb < max_blocks ? pb : max_blocks);
 }
 

@@ -10,12 +10,13 @@
 namespace pa {
 
 constexpr int kBlockSize = 16;                 // tokens per cache block
-// Default split-KV rule (partition_tokens == 0): no split when the batch has at
-// least kSplitTargetUnits (sequence, KV head) pairs, else enough partitions of
-// at least kMinPartitionBlocks blocks to reach that many CTAs (148 SMs x 2
-// resident CTAs x ~3.5 waves).
+// Default split-KV rule (partition_tokens == 0): partitions of at most
+// kMaxPartitionBlocks blocks; shorter ones (down to kMinPartitionBlocks) when the
+// batch has fewer than kSplitTargetUnits (sequence, KV head) pairs, so that the
+// launch still has about that many CTAs (148 SMs x 3 resident CTAs x ~2.3 waves).
 constexpr int kSplitTargetUnits = 1024;
 constexpr int kMinPartitionBlocks = 32;
+constexpr int kMaxPartitionBlocks = 128;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // bounded on-chip waits: 1 s
 constexpr int kMaxCopyPairsPerLaunch = 1024;   // pairs carried in one kernel parameter block
 
@@ -58,9 +59,6 @@ int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
                                 cudaStream_t stream);
 
-// Tensor-core variant for grouped-query heads (group 2, 4 or 8).
-cudaError_t launch_paged_decode_mma(const DecodeArgs& a, int head_dim, int group, int dtype,
-                                    cudaStream_t stream);
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, int64_t key_stride,
                                      int64_t value_stride, void* k_cache, void* v_cache,

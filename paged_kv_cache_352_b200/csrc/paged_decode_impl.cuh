@@ -1,0 +1,298 @@
+// Paged-decode kernel template and its launcher, instantiated once per
+// (storage type, head_dim) in paged_decode_<type>_d<dim>.cu.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <type_traits>
+
+#include "decode_common.cuh"
+#include "decode_policies.cuh"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+// Register budget hint: with the default 4 x 2 tiles three CTAs fit an SM's
+// shared memory, so the kernels are compiled for three resident CTAs (at most
+// 170 registers a thread). The CUDA-core kernels for 4 and 8 query heads per KV
+// head need more and are left to the compiler (they are not the default path).
+template <class P, int G>
+constexpr int min_ctas_hint() {
+  return !P::kTensorCores && G > 2 ? 1 : 3;
+}
+
+template <class P, typename T, int D, int G, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
+    paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v) {
+  constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + P::kAlign - 1) & ~(uintptr_t)(P::kAlign - 1));
+  const int kvh = blockIdx.x;
+  const int part = blockIdx.y;
+  const int s = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Independent loads first, so their latencies overlap: the context length,
+  // this warp's first 32 block-table entries (lane i holds the entry of the
+  // warp's block i; entries past the sequence are padding, never used) and q.
+  const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+  const int b_begin = part * a.part_blocks;
+  int ctx = __ldg(a.context_lens + s);
+  int win_base = 0;  // the window covers this warp's blocks win_base .. win_base + 31
+  int win = -1;
+  {
+    const int idx = b_begin + warp + lane * WARPS;
+    if (idx < a.max_blocks_per_seq) win = __ldg(table + idx);
+  }
+  P pol;
+  pol.init(lane);
+  pol.prefetch_q(a, s, kvh);
+
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * kBS || ctx > a.max_context_len) {
+    if (part == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
+    ctx = 0;  // flagged; the sequence yields a zero output
+  }
+  const int nblk = (ctx + kBS - 1) / kBS;
+  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  if (part >= (nparts > 0 ? nparts : 1)) return;
+  T* out_rows = reinterpret_cast<T*>(a.out) + ((size_t)s * a.num_q_heads + (size_t)kvh * G) * D;
+  if (nblk == 0) {
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) out_rows[i] = Storage<T>::from_f32(0.f);
+    return;
+  }
+  const int nlocal = min(nblk, b_begin + a.part_blocks) - b_begin;
+  const int my_n = nlocal > warp ? (nlocal - warp + WARPS - 1) / WARPS : 0;
+
+  unsigned char* wring = smem + (size_t)warp * STAGES * P::kStageBytes;
+  uint64_t* wbars = reinterpret_cast<uint64_t*>(smem + kRing) + warp * STAGES;
+  int* wvalid = reinterpret_cast<int*>(smem + kRing + WARPS * STAGES * sizeof(uint64_t)) +
+                warp * STAGES;
+  float* wp = reinterpret_cast<float*>(smem + kRing + WARPS * STAGES * (sizeof(uint64_t) + 4)) +
+              warp * P::kPbufFloats;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&wbars[st], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  // Start the copies of this warp's j-th block into stage j % STAGES. Called by
+  // every lane (the table entry comes from the window by shuffle); lane 0 copies
+  // and records in wvalid whether the stage holds a block to compute.
+  auto issue = [&](int j) {
+    if (j >= win_base + 32) {
+      win_base = j & ~31;
+      const int idx = b_begin + warp + (win_base + lane) * WARPS;
+      win = win_base + lane < my_n ? __ldg(table + idx) : -1;
+    }
+    const int phys = __shfl_sync(0xffffffffu, win, j - win_base);
+    if (lane == 0) {
+      const int st = j % STAGES;
+      uint64_t* bar = &wbars[st];
+      const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
+      wvalid[st] = ok;  // published to the consumers by the arrive below
+      if (!ok) {
+        report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
+        mbar_arrive(bar);  // complete the phase without data; the block is skipped
+      } else {
+        P::issue(a, &tm_k, &tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
+      }
+    }
+  };
+  for (int j = 0; j < STAGES && j < my_n; ++j) issue(j);
+  int issued = my_n < STAGES ? my_n : STAGES;
+  pol.begin(a.scale_log2);
+
+  bool aborted = false;
+  int j = 0;
+  for (; j < my_n; ++j) {
+    const int st = j % STAGES;
+    if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
+      if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+      aborted = true;
+      break;
+    }
+    const int b = b_begin + warp + j * WARPS;
+    if (wvalid[st]) pol.block(wring + (size_t)st * P::kStageBytes, ctx - b * kBS, wp);
+    __syncwarp();
+    if (j + STAGES < my_n) {
+      if (lane == 0) fence_proxy_async_smem();  // this stage's reads precede its next copy
+      issue(j + STAGES);
+      issued = j + STAGES + 1;
+    }
+  }
+  if (aborted) {
+    // drain the copies still in flight into this warp's ring before leaving it
+    for (int k = j; k < issued; ++k)
+      mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
+  }
+
+  // merge the warps through shared memory, reusing the tile ring
+  __syncthreads();
+  float* red_m = reinterpret_cast<float*>(smem);  // [WARPS][G]
+  float* red_l = red_m + WARPS * G;                // [WARPS][G]
+  float* red_acc = red_l + WARPS * G;              // [WARPS][G][D]
+  pol.to_red(red_m, red_l, red_acc, warp, lane);
+  __syncthreads();
+  finish_partition<T, D, G, WARPS>(a, red_m, red_m, red_l, red_acc, s, kvh, part, nparts,
+                                   out_rows);
+}
+
+constexpr size_t kSmemLimit = 200 * 1024;
+constexpr int kMaxDevices = 64;
+
+template <class P, int WARPS, int STAGES, int G, int D>
+size_t smem_bytes(int max_parts) {
+  // The warp-merge buffers and the split-KV weights reuse the tile ring once
+  // the main loop is over.
+  const size_t ring = size_t(WARPS) * STAGES * P::kStageBytes;
+  const size_t red = size_t(WARPS) * G * (D + 2) * sizeof(float);
+  const size_t wts = (size_t)max_parts * G * sizeof(float);
+  size_t reuse = red > wts ? red : wts;
+  if (reuse < ring) reuse = ring;
+  return P::kAlign + reuse + size_t(WARPS) * STAGES * (sizeof(uint64_t) + sizeof(int)) +
+         size_t(WARPS) * P::kPbufFloats * sizeof(float);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// A cache array [num_blocks][Hkv][16][d] viewed as rows of d elements, read in
+// 16-row x 64-column boxes with 128-byte swizzling.
+cudaError_t make_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
+                           int dtype) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kBS};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult res = fn(
+      map, dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <class P, typename T, int D, int G, int WARPS, int STAGES>
+cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
+  const size_t smem = smem_bytes<P, WARPS, STAGES, G, D>(a.max_parts);
+  if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
+  auto kern = paged_decode_kernel<P, T, D, G, WARPS, STAGES>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // The opt-in limit is a ceiling, not a reservation: set it once per device.
+  static std::atomic<bool> ready[kMaxDevices];
+  if (!ready[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+    if (e != cudaSuccess) return e;
+    ready[dev].store(true, std::memory_order_release);
+  }
+  CUtensorMap tk, tv;
+  memset(&tk, 0, sizeof(tk));
+  memset(&tv, 0, sizeof(tv));
+  if (!std::is_same<P, CudaCorePolicy<T, D, G>>::value) {
+    const long long rows = (long long)a.num_blocks * a.num_kv_heads * kBS;
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA row coordinates are int32
+    e = make_cache_map(&tk, a.k_cache, rows, D, dtype);
+    if (e != cudaSuccess) return e;
+    e = make_cache_map(&tv, a.v_cache, rows, D, dtype);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
+  kern<<<grid, WARPS * 32, smem, stream>>>(a, tk, tv);
+  return cudaGetLastError();
+}
+
+// Warps per CTA x stages per warp. 4 x 2 (64 KiB of K/V in flight per CTA at
+// head_dim 128, three CTAs per SM) measured best or within 2% of best on every
+// workload; PA_DECODE_TILE="WxS" selects another built shape for A/B
+// measurements (4x3, 8x2, 2x3).
+int tile_variant() {
+  static const int v = [] {
+    const char* e = getenv("PA_DECODE_TILE");
+    if (!e) return 0;
+    if (!strcmp(e, "4x3")) return 1;
+    if (!strcmp(e, "8x2")) return 2;
+    if (!strcmp(e, "2x3")) return 3;
+    return 0;
+  }();
+  return v;
+}
+
+template <class P, typename T, int D, int G>
+cudaError_t launch_tiles(const DecodeArgs& a, int dtype, cudaStream_t stream) {
+  switch (tile_variant()) {
+    case 1: return launch_kernel<P, T, D, G, 4, 3>(a, dtype, stream);
+    case 2: return launch_kernel<P, T, D, G, 8, 2>(a, dtype, stream);
+    case 3: return launch_kernel<P, T, D, G, 2, 3>(a, dtype, stream);
+    default: return launch_kernel<P, T, D, G, 4, 2>(a, dtype, stream);
+  }
+}
+
+// Which arithmetic path serves a query-head group: tensor cores from G = 4 up
+// (the q.K and P.V tiles are then real contractions), CUDA cores below.
+// PA_DECODE_PATH=cuda_cores or =tensor overrides the choice for A/B measurements.
+bool use_tensor_path(int group) {
+  static const int forced = [] {
+    const char* e = getenv("PA_DECODE_PATH");
+    if (e && !strcmp(e, "cuda_cores")) return 0;
+    if (e && !strcmp(e, "tensor")) return 1;
+    return -1;
+  }();
+  if (group < 2) return false;
+  if (forced >= 0) return forced == 1;
+  return group >= 4;
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_g(const DecodeArgs& a, int dtype, cudaStream_t stream) {
+  if (use_tensor_path(G)) return launch_tiles<TensorPolicy<T, D, G>, T, D, G>(a, dtype, stream);
+  return launch_tiles<CudaCorePolicy<T, D, G>, T, D, G>(a, dtype, stream);
+}
+
+template <typename T, int D>
+cudaError_t launch_group(const DecodeArgs& a, int group, int dtype, cudaStream_t stream) {
+  switch (group) {
+    case 1: return launch_tiles<CudaCorePolicy<T, D, 1>, T, D, 1>(a, dtype, stream);
+    case 2: return launch_g<T, D, 2>(a, dtype, stream);
+    case 4: return launch_g<T, D, 4>(a, dtype, stream);
+    case 8: return launch_g<T, D, 8>(a, dtype, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+// Launches the persistent decode kernel for one storage type and head_dim.
+template <typename T, int D>
+cudaError_t launch_decode_typed(const DecodeArgs& a, int group, int dtype,
+                                cudaStream_t stream) {
+  return launch_group<T, D>(a, group, dtype, stream);
+}
+
+}  // namespace pa

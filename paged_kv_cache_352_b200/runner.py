@@ -180,37 +180,41 @@ class DecodeRunner:
 
 
 class HostStep:
-    """One step fed from pinned host buffers and read back to the host.
+    """One step fed from pinned host memory and read back to the host.
 
-    Every call copies the step's inputs (queries, new keys/values, slot
-    mapping, block tables, context lengths) host -> device, runs the step's
-    kernels, and copies the attention output device -> host, all on the
-    current stream.
+    The step's inputs (queries, new keys/values, slot mapping, block tables,
+    context lengths) live back to back in one pinned host buffer and one device
+    buffer; the runner's input tensors are views of the device buffer. Every
+    call copies the whole input buffer host -> device, runs the step's kernels,
+    and copies the attention output device -> host, all on the current stream.
     """
 
     def __init__(self, runner: DecodeRunner):
         r = self.r = runner
-        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
-        self.h_q = pin(r.q_host).view(r.dtype)
-        self.h_k = pin(r.step_k_host).view(r.dtype)
-        self.h_v = pin(r.step_v_host).view(r.dtype)
-        self.h_slots = pin(r.step_slots_host)
-        self.h_tables = pin(r.block_tables_host)
-        self.h_ctx = pin(r.context_lens_host)
+        srcs = [("q", r.q), ("step_k", r.step_k), ("step_v", r.step_v),
+                ("step_slots", r.step_slots), ("block_tables", r.block_tables),
+                ("context_lens", r.context_lens)]
+        offs, total = [], 0
+        for _, t in srcs:
+            offs.append(total)
+            total += -(-t.numel() * t.element_size() // 256) * 256
+        self.h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+        self.d_buf = torch.empty(total, dtype=torch.uint8, device=r.device)
+        for (name, t), off in zip(srcs, offs):
+            n = t.numel() * t.element_size()
+            dview = self.d_buf[off:off + n].view(t.dtype).view(t.shape)
+            hview = self.h_buf[off:off + n].view(t.dtype).view(t.shape)
+            hview.copy_(t.cpu())
+            dview.copy_(t)
+            setattr(r, name, dview)
         self.h_out = torch.empty(r.out.shape, dtype=r.dtype).pin_memory()
-        self.h2d_bytes = sum(t.numel() * t.element_size() for t in
-                             (self.h_q, self.h_k, self.h_v, self.h_slots, self.h_tables,
-                              self.h_ctx))
+        self.h2d_bytes = total
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
+        torch.cuda.synchronize(r.device)
 
     def __call__(self):
         r = self.r
-        r.q.copy_(self.h_q, non_blocking=True)
-        r.step_k.copy_(self.h_k, non_blocking=True)
-        r.step_v.copy_(self.h_v, non_blocking=True)
-        r.step_slots.copy_(self.h_slots, non_blocking=True)
-        r.block_tables.copy_(self.h_tables, non_blocking=True)
-        r.context_lens.copy_(self.h_ctx, non_blocking=True)
+        self.d_buf.copy_(self.h_buf, non_blocking=True)
         r.step()
         self.h_out.copy_(r.out, non_blocking=True)
         return self.h_out
