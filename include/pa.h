@@ -137,13 +137,24 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
  *   block_tables       device, int32 [num_seqs][max_blocks_per_seq], padded with -1
  *   context_lens       device, int32 [num_seqs], tokens per sequence including the
  *                      token written this step
+ *   seq_order          device, int32 [num_seqs], a permutation of 0..num_seqs-1
+ *                      giving the order in which sequences are scheduled, or
+ *                      NULL for 0, 1, 2, ... Listing the sequences longest first
+ *                      (pa_longest_first_order) keeps long sequences from
+ *                      finishing last and shortens the launch's tail; sequences
+ *                      that share blocks are best kept next to each other, so
+ *                      the shared blocks are read while still in L2. Results
+ *                      do not depend on the order. Entries outside
+ *                      [0, num_seqs) are flagged (PA_DEVERR_CONTEXT_RANGE) and
+ *                      skipped; a repeated entry leaves some sequence unwritten.
  *   max_context_len    host-known upper bound of context_lens (sizes the grid
  *                      without a device read); longer sequences are flagged
  *   scale              softmax scale, usually 1/sqrt(head_dim)
  *   partition_tokens   a multiple of block_size, or 0 for the library's choice:
- *                      partitions of at most 2048 tokens, shorter (down to 512)
- *                      when num_seqs * num_kv_heads < 1024, so that the launch
- *                      still has ~1024 (sequence, KV head, partition) units
+ *                      partitions of at most 2048 tokens (4096 when seq_order is
+ *                      given), shorter (down to 512) when num_seqs *
+ *                      num_kv_heads < 1024, so that the launch still has ~1024
+ *                      (sequence, KV head, partition) units
  *   workspace          device scratch of pa_paged_decode_workspace_size() bytes,
  *                      ZERO-FILLED before its first use; every completed call
  *                      leaves it zero-filled again, so it can be reused without
@@ -155,13 +166,20 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
  * bit-identical whatever the physical placement of blocks and whether blocks
  * are shared or duplicated.
  * ------------------------------------------------------------------------- */
+/* Workspace bytes pa_paged_decode needs for these sizes (enough with or
+ * without a seq_order). */
 int pa_paged_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                    int head_dim, int max_context_len, int block_size,
                                    int partition_tokens, size_t* bytes);
 
+/* Host helper: order[0..n) = sequence indices by decreasing context_lens (ties
+ * by index), the recommended seq_order. Both arrays are host memory. */
+int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order);
+
 int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int max_blocks_per_seq,
-                    const int32_t* context_lens, int num_seqs, int max_context_len,
+                    const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                    int max_context_len,
                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                     int num_blocks, float scale, int partition_tokens, void* workspace,
                     size_t workspace_bytes, int* dev_error, int dtype, void* stream);
@@ -195,7 +213,8 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
 
 int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, int max_blocks_per_seq,
-                            const int32_t* context_lens, int num_seqs, int max_context_len,
+                            const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                            int max_context_len,
                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                             int num_blocks, float scale, int partition_tokens, int* dev_error,
                             int dtype, void* stream);

@@ -20,6 +20,7 @@ from ._lib import (  # noqa: F401
     last_error,
     lib,
     pa_copy_blocks,
+    pa_longest_first_order,
     pa_paged_decode,
     pa_paged_decode_workspace_size,
     pa_reshape_and_cache,

@@ -54,12 +54,13 @@ _SIGS = {
                                 _vp]),
     "pa_paged_decode_workspace_size": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                                 _c_int, ctypes.POINTER(ctypes.c_size_t)]),
-    "pa_paged_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
-                                 _c_int, _c_int, _c_int, _c_int, ctypes.c_float, _c_int, _vp,
-                                 ctypes.c_size_t, _vp, _c_int, _vp]),
-    "pa_paged_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
-                                         _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
-                                         _c_int, _vp, _c_int, _vp]),
+    "pa_paged_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float, _c_int,
+                                 _vp, ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_paged_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                         ctypes.c_float, _c_int, _vp, _c_int, _vp]),
+    "pa_longest_first_order": (_c_int, [_vp, _c_int, _vp]),
     "pa_bm_create": (_c_int, [_c_int, _c_int, _vp, ctypes.POINTER(_vp)]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_c_int, [_vp, _c_i64, _c_int, _vp]),
@@ -203,12 +204,24 @@ def decode_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
+def pa_longest_first_order(context_lens) -> np.ndarray:
+    """Host int32 order of sequences by decreasing context length (ties by index)."""
+    ctx = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    order = np.empty(len(ctx), np.int32)
+    _check(lib().pa_longest_first_order(ctx.ctypes.data if len(ctx) else None, len(ctx),
+                                        order.ctypes.data if len(ctx) else None))
+    return order
+
+
 def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
-                    scale, partition_tokens=0, workspace=None, dev_error=None, stream=None):
+                    scale, partition_tokens=0, workspace=None, dev_error=None, stream=None,
+                    seq_order=None):
     """Decode attention through block tables; writes ``out`` ``[B, Hq, d]``.
 
     ``workspace`` must be a zero-filled uint8 CUDA tensor of at least
     ``pa_paged_decode_workspace_size(...)`` bytes when that size is non-zero.
+    ``seq_order`` (int32 CUDA tensor, a permutation) schedules sequences in that
+    order; longest first (``pa_longest_first_order``) shortens the launch's tail.
     """
     torch = _torch()
     nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
@@ -224,18 +237,26 @@ def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_co
     _check(lib().pa_paged_decode(
         _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
         _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
-        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32), B,
-        int(max_context_len), hq, hkv, d, bs, nb, float(scale), int(partition_tokens),
-        _dev_ptr(workspace, "workspace"), ws_bytes,
+        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
+        _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+        int(partition_tokens), _dev_ptr(workspace, "workspace"), ws_bytes,
         _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
 
 
 NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 
+def _order_ptr(seq_order, B):
+    if seq_order is None:
+        return None
+    if seq_order.shape != (B,):
+        raise PAError(PA_ERR_INVALID_ARG, "seq_order must be [num_seqs]")
+    return _dev_ptr(seq_order, "seq_order", _torch().int32)
+
+
 def pa_paged_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
                             max_context_len, scale, partition_tokens=0, dev_error=None,
-                            stream=None):
+                            stream=None, seq_order=None):
     """Like ``pa_paged_decode`` but without a workspace argument.
 
     For callers that cannot allocate device memory: the split-KV scratch comes
@@ -254,9 +275,10 @@ def pa_paged_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens
     _check(lib().pa_paged_decode_noalloc(
         _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
         _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
-        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32), B,
-        int(max_context_len), hq, hkv, d, bs, nb, float(scale), int(partition_tokens),
-        _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
+        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
+        _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+        int(partition_tokens), _dev_ptr(dev_error, "dev_error", torch.int32),
+        dtype_code(k_cache), _stream(stream)))
 
 
 # --------------------------------------------------------------------------

@@ -51,7 +51,7 @@ int cuda_status(cudaError_t e, const char* what) {
 
 }  // namespace
 
-int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks) {
+int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks, bool ordered) {
   // A CTA streams best over a long run of blocks: every extra partition costs its
   // CTA's pipeline ramp and a merge. Long partitions, though, leave a tail of
   // lone CTAs at the end of the launch. Partitions are therefore capped at
@@ -65,12 +65,13 @@ int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks) {
     pb = (max_blocks + parts - 1) / parts;
     if (pb < kMinPartitionBlocks) pb = kMinPartitionBlocks;
   }
-  if (pb > kMaxPartitionBlocks) pb = kMaxPartitionBlocks;
+  const int cap = ordered ? kMaxPartitionBlocksOrdered : kMaxPartitionBlocks;
+  if (pb > cap) pb = cap;
   return (int)(pb < max_blocks ? pb : max_blocks);
 }
 
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                  int max_context_len, int partition_tokens, DecodeLayout* lay) {
+                  int max_context_len, int partition_tokens, bool ordered, DecodeLayout* lay) {
   if (partition_tokens < 0 || partition_tokens % kBlockSize != 0)
     return fail(PA_ERR_INVALID_ARG, "partition_tokens %d: must be 0 or a positive multiple of %d",
                 partition_tokens, kBlockSize);
@@ -78,7 +79,8 @@ int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
   const int group = num_q_heads / num_kv_heads;
   const int max_blocks = (max_context_len + kBlockSize - 1) / kBlockSize;
   const int part_blocks = partition_tokens == 0
-                              ? default_partition_blocks(num_seqs, num_kv_heads, max_blocks)
+                              ? default_partition_blocks(num_seqs, num_kv_heads, max_blocks,
+                                                         ordered)
                               : partition_tokens / kBlockSize;
   int max_parts = (max_blocks + part_blocks - 1) / part_blocks;
   if (max_parts < 1) max_parts = 1;
@@ -107,7 +109,7 @@ extern "C" {
 
 const char* pa_last_error(void) { return g_last_error.c_str(); }
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 110; }
 
 int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_stride,
                          int64_t value_token_stride, void* k_cache, void* v_cache,
@@ -189,16 +191,31 @@ int pa_paged_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_hea
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
     return fail(PA_ERR_INVALID_ARG, "bad sequence or head counts");
   DecodeLayout lay;
+  // Without an order the default partitions are shorter, so that layout is the
+  // larger of the two.
   if (int st = decode_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                             partition_tokens, &lay))
+                             partition_tokens, false, &lay))
     return st;
   *bytes = lay.bytes;
   return PA_OK;
 }
 
+int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order) {
+  clear_error();
+  if (n < 0) return fail(PA_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return PA_OK;
+  if (!context_lens || !order) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order, order + n, [context_lens](int32_t x, int32_t y) {
+    return context_lens[x] > context_lens[y];
+  });
+  return PA_OK;
+}
+
 int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int max_blocks_per_seq,
-                    const int32_t* context_lens, int num_seqs, int max_context_len,
+                    const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                    int max_context_len,
                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                     int num_blocks, float scale, int partition_tokens, void* workspace,
                     size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
@@ -223,7 +240,7 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
     return fail(PA_ERR_INVALID_ARG, "out, q and cache pointers must be 16-byte aligned");
   DecodeLayout lay;
   if (int st = decode_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                             partition_tokens, &lay))
+                             partition_tokens, seq_order != nullptr, &lay))
     return st;
   if (lay.bytes > 0) {
     if (!workspace || workspace_bytes < lay.bytes)
@@ -239,6 +256,7 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
   a.v_cache = v_cache;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
+  a.seq_order = seq_order;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   a.ws_count = lay.bytes ? reinterpret_cast<int*>(ws + lay.count_off) : nullptr;
   a.ws_ml = lay.bytes ? reinterpret_cast<float*>(ws + lay.ml_off) : nullptr;

@@ -17,6 +17,8 @@ constexpr int kBlockSize = 16;                 // tokens per cache block
 constexpr int kSplitTargetUnits = 1024;
 constexpr int kMinPartitionBlocks = 32;
 constexpr int kMaxPartitionBlocks = 128;
+// With a longest-first seq_order the tail is short enough for longer partitions.
+constexpr int kMaxPartitionBlocksOrdered = 256;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // bounded on-chip waits: 1 s
 constexpr int kMaxCopyPairsPerLaunch = 1024;   // pairs carried in one kernel parameter block
 
@@ -31,6 +33,7 @@ struct DecodeArgs {
   const void* v_cache;
   const int32_t* block_tables;
   const int32_t* context_lens;
+  const int32_t* seq_order;  // nullable: CTA z serves sequence seq_order[z]
   float* ws_ml;      // [B][Hkv][max_parts][G][2]  (m, l) per partition
   float* ws_acc;     // [B][Hkv][max_parts][G][D]  unnormalised partition outputs
   int* ws_count;     // [B][Hkv]  partitions finished (returned to 0 by the merging CTA)
@@ -54,7 +57,7 @@ struct DecodeLayout {
 
 // Workspace layout for a decode call (bytes == 0 when no sequence can split).
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                  int max_context_len, int partition_tokens, DecodeLayout* lay);
+                  int max_context_len, int partition_tokens, bool ordered, DecodeLayout* lay);
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
                                 cudaStream_t stream);

@@ -39,9 +39,13 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
       (reinterpret_cast<uintptr_t>(smem_raw) + P::kAlign - 1) & ~(uintptr_t)(P::kAlign - 1));
   const int kvh = blockIdx.x;
   const int part = blockIdx.y;
-  const int s = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int s = a.seq_order ? __ldg(a.seq_order + blockIdx.z) : (int)blockIdx.z;
+  if ((unsigned)s >= (unsigned)a.num_seqs) {
+    if (part == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
+    return;
+  }
 
   // Independent loads first, so their latencies overlap: the context length,
   // this warp's first 32 block-table entries (lane i holds the entry of the

@@ -63,7 +63,8 @@ int scratch_address(void** out) {
 extern "C" int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache,
                                        const void* v_cache, const int32_t* block_tables,
                                        int max_blocks_per_seq, const int32_t* context_lens,
-                                       int num_seqs, int max_context_len, int num_q_heads,
+                                       const int32_t* seq_order, int num_seqs,
+                                       int max_context_len, int num_q_heads,
                                        int num_kv_heads, int head_dim, int block_size,
                                        int num_blocks, float scale, int partition_tokens,
                                        int* dev_error, int dtype, void* stream) {
@@ -92,7 +93,7 @@ extern "C" int pa_paged_decode_noalloc(void* out, const void* q, const void* k_c
       return pa::fail(PA_ERR_CUDA, "clearing the built-in scratch: %s", cudaGetErrorString(e));
   }
   return pa_paged_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                         num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
+                         seq_order, num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim,
                          block_size, num_blocks, scale, partition_tokens, scratch,
                          need > 0 ? kScratchBytes : 0, dev_error, dtype, stream);
 }

@@ -60,6 +60,14 @@ class DecodeRunner:
         self.block_tables = torch.from_numpy(self.block_tables_host).to(self.device)
         self.context_lens_host = wl.context_lens.astype(np.int32)
         self.context_lens = torch.from_numpy(self.context_lens_host).to(self.device)
+        # Schedule the longest sequences first, so they do not finish last. Samples
+        # that share a prompt's blocks stay in fork order instead: scheduled side
+        # by side they read the shared blocks while those are still in L2.
+        if wl.kind == "shared_prefix":
+            self.seq_order_host = np.arange(wl.num_seqs, dtype=np.int32)
+        else:
+            self.seq_order_host = L.pa_longest_first_order(self.context_lens_host)
+        self.seq_order = torch.from_numpy(self.seq_order_host).to(self.device)
         self.q_host = gen.query_bits(wl.seed, wl.num_seqs, wl.num_q_heads, wl.head_dim, wl.dtype)
         self.q = _to_dev(self.q_host, wl.dtype, self.device)
         self.out = torch.empty_like(self.q)
@@ -153,7 +161,7 @@ class DecodeRunner:
             L.pa_reshape_and_cache(self.step_k, self.step_v, self.k_cache, self.v_cache,
                                    self.step_slots, self.dev_error)
 
-    def decode(self, out=None, partition_tokens=None):
+    def decode(self, out=None, partition_tokens=None, ordered=True):
         out = self.out if out is None else out
         pt = self.partition_tokens if partition_tokens is None else partition_tokens
         ws = self.workspace
@@ -162,7 +170,7 @@ class DecodeRunner:
                                     self.wl.head_dim, self.wl.max_context_len, pt, self.device)
         L.pa_paged_decode(out, self.q, self.k_cache, self.v_cache, self.block_tables,
                           self.context_lens, self.wl.max_context_len, self.wl.scale, pt, ws,
-                          self.dev_error)
+                          self.dev_error, seq_order=self.seq_order if ordered else None)
         return out
 
     def step(self):
@@ -183,7 +191,7 @@ class HostStep:
     """One step fed from pinned host memory and read back to the host.
 
     The step's inputs (queries, new keys/values, slot mapping, block tables,
-    context lengths) live back to back in one pinned host buffer and one device
+    context lengths, scheduling order) live back to back in one pinned host buffer and one device
     buffer; the runner's input tensors are views of the device buffer. Every
     call copies the whole input buffer host -> device, runs the step's kernels,
     and copies the attention output device -> host, all on the current stream.
@@ -193,7 +201,7 @@ class HostStep:
         r = self.r = runner
         srcs = [("q", r.q), ("step_k", r.step_k), ("step_v", r.step_v),
                 ("step_slots", r.step_slots), ("block_tables", r.block_tables),
-                ("context_lens", r.context_lens)]
+                ("context_lens", r.context_lens), ("seq_order", r.seq_order)]
         offs, total = [], 0
         for _, t in srcs:
             offs.append(total)

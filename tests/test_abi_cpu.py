@@ -27,7 +27,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert len(names) >= 18
     missing = [n for n in names if not hasattr(h, n)]
     assert not missing, missing
-    assert h.pa_version() == 100
+    assert h.pa_version() == 110
 
 
 def test_binding_covers_every_declared_symbol():
@@ -98,7 +98,7 @@ def test_decode_argument_checks():
                  err=None, dt=L.PA_BF16)
         a.update(kw)
         return lib.pa_paged_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["mb"], a["ctx"],
-                                   a["B"], a["maxctx"], a["hq"], a["hkv"], a["d"], a["bs"],
+                                   None, a["B"], a["maxctx"], a["hq"], a["hkv"], a["d"], a["bs"],
                                    a["nb"], a["scale"], a["pt"], a["ws"], a["wsb"], a["err"],
                                    a["dt"], None)
 
@@ -112,6 +112,12 @@ def test_decode_argument_checks():
     assert call(q=ctypes.c_void_p(4100)) == L.PA_ERR_INVALID_ARG
     assert call(B=0) == L.PA_OK                         # nothing to do
     assert call(scale=float("nan")) == L.PA_ERR_INVALID_ARG
+
+
+def test_longest_first_order():
+    ctx = [5, 90, 90, 1, 300, 0]
+    assert pa.pa_longest_first_order(ctx).tolist() == [4, 1, 2, 0, 3, 5]
+    assert pa.pa_longest_first_order([]).tolist() == []
 
 
 def test_workspace_size_formula():

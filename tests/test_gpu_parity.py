@@ -297,3 +297,38 @@ def test_full_size_sampled_parity(name):
     again = r.step().clone()
     _sync()
     assert torch.equal(again.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["gqa_32_8_bf16", "long_ctx_split_kv", "mha_7b_fp16"])
+def test_scheduling_order_does_not_change_results(name):
+    wl = workloads.workload(name, small=True)
+    r = DecodeRunner(wl)
+    r.step()
+    outs = []
+    for order in (None, "longest", "random"):
+        out = torch.empty_like(r.out)
+        if order is None:
+            r.decode(out, ordered=False)
+        else:
+            if order == "random":
+                perm = np.random.default_rng(5).permutation(wl.num_seqs).astype(np.int32)
+                r.seq_order.copy_(torch.from_numpy(perm))
+            r.decode(out, ordered=True)
+        outs.append(out)
+    _sync()
+    assert r.error_bits() == 0
+    for o in outs[1:]:
+        assert torch.equal(outs[0].view(torch.int16), o.view(torch.int16))
+
+
+def test_bad_order_entries_are_flagged():
+    ctx = [40, 70]
+    q, kc, vc, tables, cl = _manual_case(ctx)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(q)
+    order = torch.tensor([1, 7], dtype=torch.int32, device="cuda")
+    pa.pa_paged_decode(out, q, kc, vc, tables, cl, 70, 0.1, 0, None, err, seq_order=order)
+    _sync()
+    assert err.item() & pa.PA_DEVERR_CONTEXT_RANGE
+    ref = _oracle_manual(q, kc, vc, tables, cl, 0.1, torch.bfloat16)
+    assert_close(out_to_f64(out[1:], "bf16"), ref[1:])   # sequence 1 was still computed
