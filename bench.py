@@ -363,6 +363,42 @@ def oracle_sample_setup_range(wl, first: int, n: int):
 # arms
 # --------------------------------------------------------------------------
 
+def measure_swap(wl, r, device, nblocks: int = 2048, reps: int = 5):
+    """Host-link rate of pa_swap_blocks: ``nblocks`` whole blocks (all KV heads,
+    K and V) from the workload's pool to a pinned host pool and back, in a
+    shuffled order, timed with CUDA events (best of ``reps``)."""
+    import torch
+    from paged_kv_cache_352_b200 import _lib as L
+    nblocks = min(nblocks, wl.num_blocks)
+    shape = (nblocks,) + tuple(r.k_cache.shape[1:])
+    hk = torch.empty(shape, dtype=r.dtype).pin_memory()
+    hv = torch.empty(shape, dtype=r.dtype).pin_memory()
+    rng = np.random.default_rng(7)
+    src = rng.permutation(wl.num_blocks)[:nblocks]
+    out_pairs = np.stack([src, np.arange(nblocks)], 1)
+    in_pairs = np.stack([np.arange(nblocks), src], 1)
+    nbytes = 2 * r.k_cache[0].numel() * r.k_cache.element_size() * nblocks
+    res = {}
+    for name, fn in (("d2h", lambda: L.pa_swap_blocks(r.k_cache, r.v_cache, hk, hv, out_pairs)),
+                     ("h2d", lambda: L.pa_swap_blocks(hk, hv, r.k_cache, r.v_cache, in_pairs))):
+        fn()
+        torch.cuda.synchronize(device)
+        best = None
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize(device)
+            t = a.elapsed_time(b) / 1e3
+            best = t if best is None else min(best, t)
+        res[name + "_gbs"] = round(nbytes / best / 1e9, 2)
+    res.update(blocks=int(nblocks), bytes=int(nbytes), unit="GB/s",
+               what="pa_swap_blocks, shuffled whole blocks, device pool <-> pinned host pool")
+    return res
+
+
 def run_reference(args):
     rank, world, _ = _rank_info()
     if rank != 0:
@@ -486,6 +522,8 @@ def run_ours(args):
     e2e_s = _max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ee]) / 1e3), world,
                             device)
 
+    swap = measure_swap(wl, r, device) if world == 1 else None
+
     sb = step_bytes(wl, r)
     db = decode_bytes(wl)
     peak, peak_kind = _peaks()
@@ -531,6 +569,7 @@ def run_ours(args):
                 "h2d_bytes_per_step": hs.h2d_bytes, "d2h_bytes_per_step": hs.d2h_bytes,
                 "ms_per_step": round(e2e_s * 1e3, 4)},
         "gpu_launches": K * launches_per_step,
+        "swap": swap,
         "clocks": csum,
     }
     if world == 1 and not args.no_cpu_baseline:

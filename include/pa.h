@@ -17,7 +17,8 @@
  * Conventions for every call
  *   - Return value: a pa_status (0 = PA_OK). On failure, pa_last_error() holds a
  *     message for the calling thread until its next libpa call.
- *   - Device calls (pa_reshape_and_cache, pa_copy_blocks, pa_paged_decode) take
+ *   - Device calls (pa_reshape_and_cache, pa_copy_blocks, pa_swap_blocks,
+ *     pa_paged_decode) take
  *     device pointers owned by the caller, enqueue kernels on the caller's CUDA
  *     stream (`stream` is a cudaStream_t; NULL = legacy default stream), never
  *     synchronise, never allocate device memory, and return after the launch.
@@ -53,7 +54,8 @@ typedef enum pa_status {
   PA_ERR_UNKNOWN_SEQ = 3,    /* sequence id not registered */
   PA_ERR_CUDA = 4,           /* a CUDA runtime call failed */
   PA_ERR_UNSUPPORTED = 5,    /* shape or type outside the supported set */
-  PA_ERR_SEQ_EXISTS = 6      /* sequence id already registered */
+  PA_ERR_SEQ_EXISTS = 6,     /* sequence id already registered */
+  PA_ERR_SEQ_SWAPPED = 7     /* sequence is swapped out (or, for swap-in, is not) */
 } pa_status;
 
 typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
@@ -115,6 +117,32 @@ int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_s
 int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                    void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_swap_blocks — move whole blocks between two pools: the device pool and a
+ * pool of pinned host memory, for preemption by swapping.
+ *
+ * When memory runs short a low-priority request's blocks are swapped to CPU
+ * memory and brought back later ("PagedAttention: The vLLM Paper",
+ * "Implementation Essentials"; "The OS paging analogy", swapping). For each
+ * pair i: block pairs[2i+1] of the destination pool (K and V) becomes a copy of
+ * block pairs[2i] of the source pool. pa_bm_swap_out / pa_bm_swap_in emit the
+ * pairs.
+ *
+ *   src_k, src_v / dst_k, dst_v   pools in the cache layout above with
+ *                 src_num_blocks / dst_num_blocks blocks. Each is device memory
+ *                 or pinned host memory the GPU can address (cudaHostAlloc /
+ *                 cudaHostRegister); pageable host memory is refused. Source and
+ *                 destination must be different pools.
+ *   pairs         HOST int64 [num_pairs][2] = (src block, dst block); ids in
+ *                 range of their pools and destination ids distinct, else
+ *                 PA_ERR_INVALID_ARG and nothing is launched.
+ * The copy runs on `stream`; after a swap-out, it must run before the freed
+ * device blocks are written again (enqueue it first on the same stream).
+ * ------------------------------------------------------------------------- */
+int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, void* dst_k,
+                   void* dst_v, int dst_num_blocks, const int64_t* pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
  * pa_paged_decode — decode-step attention through the block tables.
@@ -266,6 +294,26 @@ int pa_bm_free_seq(pa_bm* bm, int64_t seq_id);
  * PA_ERR_INVALID_ARG if a table is longer than max_blocks. */
 int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* out,
                        int max_blocks);
+
+/* Swapping. pa_bm_set_host_pool sizes the host pool (host blocks 0..n-1, handed
+ * out 0 first; refused while any sequence is swapped out). pa_bm_swap_out moves
+ * seq_id's blocks to host blocks: pairs_out[capacity][2] receives one
+ * (device block, host block) pair per block in logical order and *n_pairs their
+ * count; device refcounts drop by one and blocks reaching zero return to the
+ * free list, last logical block first. A block still shared with resident
+ * sequences stays on the device for them. pa_bm_swap_in reverses it with
+ * (host block, device block) pairs. While swapped, the sequence cannot append,
+ * fork or appear in block tables (PA_ERR_SEQ_SWAPPED); pa_bm_free_seq releases
+ * its host blocks. Both calls are all-or-nothing (PA_ERR_NO_FREE_BLOCKS when
+ * the target pool is short). */
+int pa_bm_set_host_pool(pa_bm* bm, int num_host_blocks);
+int pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int64_t* pairs_out, int capacity, int* n_pairs);
+int pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int64_t* pairs_out, int capacity, int* n_pairs);
+/* 1 if swapped out, 0 if resident, -1 for an unknown sequence. */
+int pa_bm_is_swapped(const pa_bm* bm, int64_t seq_id);
+int pa_bm_num_free_host(const pa_bm* bm);
+/* Free host blocks in hand-out order into out[capacity]; returns the count or -1. */
+int pa_bm_host_free_list(const pa_bm* bm, int32_t* out, int capacity);
 
 /* Queries. pa_bm_refcount and pa_bm_seq_len return -1 for an unknown block or
  * sequence (and set pa_last_error). */

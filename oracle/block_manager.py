@@ -28,6 +28,23 @@ rules so that tables can be compared bit for bit):
     drops by one. A sequence whose last block has refcount one writes in place.
   * Every call is all-or-nothing: when the pool cannot cover it, nothing changes.
   * Block tables are padded with -1.
+
+Swapping (preemption when the pool runs short: a request's blocks move to CPU
+memory and come back later — "PagedAttention: The vLLM Paper", "Implementation
+Essentials" and "The OS paging analogy", swapping), read as:
+  * A host pool of equal blocks with its own stack free list, set once.
+  * ``swap_out`` gives each of the sequence's blocks a host block, in logical
+    order, and emits ``(device block, host block)`` pairs; the device
+    refcounts drop by one and blocks reaching zero return to the device free
+    list, last logical block first (as ``free_seq``). A block still shared with
+    resident sequences stays on the device for them; the swapped sequence takes
+    its own host copy. The caller copies the pairs before the freed device
+    blocks are written again.
+  * ``swap_in`` gives each host block a fresh device block, in logical order,
+    emits ``(host block, device block)`` pairs, and returns the host blocks to
+    the host free list, last logical block first.
+  * A swapped sequence cannot append, fork, be swapped out again or appear in
+    block tables; ``free_seq`` releases its host blocks.
 """
 
 from __future__ import annotations
@@ -40,6 +57,7 @@ ERR_INVALID_ARG = 1
 ERR_NO_FREE_BLOCKS = 2
 ERR_UNKNOWN_SEQ = 3
 ERR_SEQ_EXISTS = 6
+ERR_SEQ_SWAPPED = 7
 
 
 class BlockManagerError(Exception):
@@ -70,6 +88,65 @@ class BlockManager:
         self._ref = [0] * num_blocks
         self._tables: dict[int, list[int]] = {}
         self._lens: dict[int, int] = {}
+        self._host_free: list[int] = []
+        self.num_host_blocks = 0
+        self._swapped: dict[int, list[int]] = {}   # seq -> host blocks in logical order
+
+    def set_host_pool(self, num_host_blocks: int) -> None:
+        if num_host_blocks < 0:
+            raise BlockManagerError(ERR_INVALID_ARG, "num_host_blocks must be >= 0")
+        if self._swapped:
+            raise BlockManagerError(ERR_INVALID_ARG, "host blocks are in use")
+        self.num_host_blocks = num_host_blocks
+        self._host_free = list(reversed(range(num_host_blocks)))
+
+    def num_free_host(self) -> int:
+        return len(self._host_free)
+
+    def is_swapped(self, seq_id: int) -> bool:
+        self._need(seq_id)
+        return seq_id in self._swapped
+
+    def swap_out(self, seq_id: int):
+        """Move the sequence to host blocks; return ``(device, host)`` copy pairs."""
+        self._need(seq_id)
+        self._resident(seq_id)
+        table = self._tables[seq_id]
+        if len(table) > len(self._host_free):
+            raise BlockManagerError(ERR_NO_FREE_BLOCKS, "host pool exhausted")
+        host = [self._host_free.pop() for _ in table]
+        pairs = list(zip(table, host))
+        for b in reversed(table):
+            self._ref[b] -= 1
+            if self._ref[b] == 0:
+                self._free.append(b)
+        self._tables[seq_id] = []
+        self._swapped[seq_id] = host
+        return pairs
+
+    def swap_in(self, seq_id: int):
+        """Bring a swapped sequence back; return ``(host, device)`` copy pairs."""
+        self._need(seq_id)
+        if seq_id not in self._swapped:
+            raise BlockManagerError(ERR_SEQ_SWAPPED, f"sequence {seq_id} is not swapped out")
+        host = self._swapped[seq_id]
+        if len(host) > len(self._free):
+            raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
+        table = []
+        for _ in host:
+            b = self._free.pop()
+            self._ref[b] = 1
+            table.append(b)
+        pairs = list(zip(host, table))
+        for h in reversed(host):
+            self._host_free.append(h)
+        del self._swapped[seq_id]
+        self._tables[seq_id] = table
+        return pairs
+
+    def _resident(self, seq_id):
+        if seq_id in self._swapped:
+            raise BlockManagerError(ERR_SEQ_SWAPPED, f"sequence {seq_id} is swapped out")
 
     # -- queries ---------------------------------------------------------
     def num_free(self) -> int:
@@ -87,6 +164,13 @@ class BlockManager:
     def table(self, seq_id: int) -> list[int]:
         self._need(seq_id)
         return list(self._tables[seq_id])
+
+    def host_table(self, seq_id: int) -> list[int]:
+        self._need(seq_id)
+        return list(self._swapped.get(seq_id, []))
+
+    def host_free_list(self) -> list[int]:
+        return list(reversed(self._host_free))
 
     def seq_ids(self):
         return list(self._tables)
@@ -125,6 +209,7 @@ class BlockManager:
     def fork(self, parent: int, child: int) -> None:
         """Child starts as a copy of the parent's table; every block is shared."""
         self._need(parent)
+        self._resident(parent)
         if child in self._tables:
             raise BlockManagerError(ERR_SEQ_EXISTS, f"sequence {child} exists")
         table = list(self._tables[parent])
@@ -136,6 +221,7 @@ class BlockManager:
     def append_slots(self, seq_id: int, n: int):
         """Append ``n`` tokens; return ``(slots, cow_pairs)``."""
         self._need(seq_id)
+        self._resident(seq_id)
         if n < 0:
             raise BlockManagerError(ERR_INVALID_ARG, "n must be >= 0")
         table = self._tables[seq_id]
@@ -165,6 +251,8 @@ class BlockManager:
 
     def free_seq(self, seq_id: int) -> None:
         self._need(seq_id)
+        for h in reversed(self._swapped.pop(seq_id, [])):
+            self._host_free.append(h)
         for b in reversed(self._tables[seq_id]):
             self._ref[b] -= 1
             if self._ref[b] == 0:
@@ -178,6 +266,7 @@ class BlockManager:
         out = np.full((len(seq_ids), max_blocks), -1, dtype=np.int32)
         for i, s in enumerate(seq_ids):
             self._need(s)
+            self._resident(s)
             t = self._tables[s]
             if len(t) > max_blocks:
                 raise BlockManagerError(ERR_INVALID_ARG, "table longer than max_blocks")

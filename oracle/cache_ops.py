@@ -39,3 +39,11 @@ def copy_blocks(k_cache, v_cache, pairs):
     for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2).tolist():
         k_cache[dst] = k_cache[src].copy()
         v_cache[dst] = v_cache[src].copy()
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, pairs):
+    """Copy block ``src`` of the source pool over block ``dst`` of the destination
+    pool (device -> host on swap-out, host -> device on swap-in), K and V."""
+    for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2).tolist():
+        dst_k[dst] = src_k[src].copy()
+        dst_v[dst] = src_v[src].copy()

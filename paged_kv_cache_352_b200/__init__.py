@@ -24,4 +24,5 @@ from ._lib import (  # noqa: F401
     pa_paged_decode,
     pa_paged_decode_workspace_size,
     pa_reshape_and_cache,
+    pa_swap_blocks,
 )

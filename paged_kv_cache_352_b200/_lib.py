@@ -24,6 +24,7 @@ PA_ERR_UNKNOWN_SEQ = 3
 PA_ERR_CUDA = 4
 PA_ERR_UNSUPPORTED = 5
 PA_ERR_SEQ_EXISTS = 6
+PA_ERR_SEQ_SWAPPED = 7
 
 PA_F16 = 0
 PA_BF16 = 1
@@ -73,6 +74,14 @@ _SIGS = {
     "pa_bm_seq_len": (_c_int, [_vp, _c_i64]),
     "pa_bm_num_seqs": (_c_int, [_vp]),
     "pa_bm_free_list": (_c_int, [_vp, _vp, _c_int]),
+    "pa_swap_blocks": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
+                                _c_int, _c_int, _vp]),
+    "pa_bm_set_host_pool": (_c_int, [_vp, _c_int]),
+    "pa_bm_swap_out": (_c_int, [_vp, _c_i64, _vp, _c_int, ctypes.POINTER(_c_int)]),
+    "pa_bm_swap_in": (_c_int, [_vp, _c_i64, _vp, _c_int, ctypes.POINTER(_c_int)]),
+    "pa_bm_is_swapped": (_c_int, [_vp, _c_i64]),
+    "pa_bm_num_free_host": (_c_int, [_vp]),
+    "pa_bm_host_free_list": (_c_int, [_vp, _vp, _c_int]),
 }
 
 _LIB = None
@@ -182,6 +191,29 @@ def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
     _check(lib().pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
                                 p.ctypes.data if len(p) else None, len(p), hkv, d, bs, nb,
                                 dtype_code(k_cache), _stream(stream)))
+
+
+def _pool_ptr(t, name):
+    """Address of a pool tensor on the GPU or in pinned host memory."""
+    if not t.is_contiguous():
+        raise PAError(PA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if not t.is_cuda and not t.is_pinned():
+        raise PAError(PA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor or pinned host memory")
+    return t.data_ptr()
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, pairs, stream=None):
+    """Copy blocks ``pairs[i, 0]`` of the source pool over ``pairs[i, 1]`` of the
+    destination pool; pools are CUDA tensors or pinned host tensors."""
+    s_nb, hkv, bs, d = _cache_dims(src_k, src_v)
+    d_nb, hkv2, bs2, d2 = _cache_dims(dst_k, dst_v)
+    if (hkv, bs, d) != (hkv2, bs2, d2) or src_k.dtype != dst_k.dtype:
+        raise PAError(PA_ERR_INVALID_ARG, "source and destination pools differ in layout")
+    p = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    _check(lib().pa_swap_blocks(_pool_ptr(src_k, "src_k"), _pool_ptr(src_v, "src_v"), s_nb,
+                                _pool_ptr(dst_k, "dst_k"), _pool_ptr(dst_v, "dst_v"), d_nb,
+                                p.ctypes.data if len(p) else None, len(p), hkv, d, bs,
+                                dtype_code(src_k), _stream(stream)))
 
 
 def pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
@@ -368,5 +400,42 @@ class BlockManager:
         return out[:n].tolist()
 
     def table(self, seq_id: int) -> list:
+        if self.is_swapped(seq_id):
+            return []
         n = -(-self.seq_len(seq_id) // self.block_size)
         return self.block_tables([seq_id], max(n, 1))[0, :n].tolist()
+
+    # -- swapping ----------------------------------------------------------------
+    def set_host_pool(self, num_host_blocks: int) -> None:
+        _check(self._lib.pa_bm_set_host_pool(self._h, num_host_blocks))
+        self.num_host_blocks = num_host_blocks
+
+    def _swap(self, fn, seq_id):
+        n = -(-self.seq_len(seq_id) // self.block_size)
+        pairs = np.empty((max(n, 1), 2), np.int64)
+        cnt = ctypes.c_int(0)
+        _check(fn(self._h, seq_id, pairs.ctypes.data, n, ctypes.byref(cnt)))
+        return pairs[:cnt.value].copy()
+
+    def swap_out(self, seq_id: int) -> np.ndarray:
+        """(device block, host block) copy pairs, in logical order."""
+        return self._swap(self._lib.pa_bm_swap_out, seq_id)
+
+    def swap_in(self, seq_id: int) -> np.ndarray:
+        """(host block, device block) copy pairs, in logical order."""
+        return self._swap(self._lib.pa_bm_swap_in, seq_id)
+
+    def is_swapped(self, seq_id: int) -> bool:
+        r = self._lib.pa_bm_is_swapped(self._h, seq_id)
+        if r < 0:
+            raise PAError(PA_ERR_UNKNOWN_SEQ, last_error())
+        return bool(r)
+
+    def num_free_host(self) -> int:
+        return self._lib.pa_bm_num_free_host(self._h)
+
+    def host_free_list(self) -> list:
+        n = max(self.num_free_host(), 1)
+        out = np.empty(n, np.int32)
+        m = self._lib.pa_bm_host_free_list(self._h, out.ctypes.data, n)
+        return out[:m].tolist()

@@ -7,6 +7,13 @@
 // paging analogy"; "PagedAttention and Continuous Batching", "Pages, from
 // operating systems").
 //
+// Preemption by swapping: a sequence's blocks can move to a host pool and back
+// ("PagedAttention: The vLLM Paper", "Implementation Essentials" and "The OS
+// paging analogy", swapping). The host pool is a stack like the device pool;
+// swap-out emits (device, host) copy pairs in logical order and releases device
+// blocks last first, swap-in emits (host, device) pairs and releases host blocks
+// last first. A swapped sequence cannot grow, fork or appear in block tables.
+//
 // Every mutating call first works out how many free blocks it needs and fails
 // before touching any state when the pool cannot cover it.
 #include <stdint.h>
@@ -19,14 +26,19 @@
 
 struct pa_bm {
   struct Seq {
-    std::vector<int32_t> table;
+    std::vector<int32_t> table;  // device blocks (empty while swapped out)
+    std::vector<int32_t> host;   // host blocks while swapped out
     int64_t len = 0;
+    bool swapped = false;
   };
   int num_blocks = 0;
   int block_size = 0;
   std::vector<int32_t> free_stack;  // back() is handed out next
   std::vector<int32_t> ref;
   std::unordered_map<int64_t, Seq> seqs;
+  std::vector<int32_t> host_free;  // back() is handed out next
+  int num_host_blocks = 0;
+  int num_swapped = 0;
 
   int32_t pop() {
     const int32_t b = free_stack.back();
@@ -44,6 +56,10 @@ using pa::fail;
 namespace {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int swapped_error(int64_t seq_id) {
+  return fail(PA_ERR_SEQ_SWAPPED, "sequence %lld is swapped out", (long long)seq_id);
+}
 
 }  // namespace
 
@@ -108,6 +124,7 @@ int pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child) {
   auto it = bm->seqs.find(parent);
   if (it == bm->seqs.end())
     return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)parent);
+  if (it->second.swapped) return swapped_error(parent);
   if (bm->seqs.count(child))
     return fail(PA_ERR_SEQ_EXISTS, "sequence %lld exists", (long long)child);
   pa_bm::Seq s = it->second;
@@ -127,6 +144,7 @@ int pa_bm_append_slots(pa_bm* bm, int64_t seq_id, int n, int64_t* slots_out,
   if (it == bm->seqs.end())
     return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
   pa_bm::Seq& s = it->second;
+  if (s.swapped) return swapped_error(seq_id);
   const int bs = bm->block_size;
   const int64_t new_blocks = ceil_div(s.len + n, bs) - (int64_t)s.table.size();
   const bool cow = n > 0 && s.len % bs != 0 && bm->ref[s.table.back()] > 1;
@@ -157,6 +175,9 @@ int pa_bm_free_seq(pa_bm* bm, int64_t seq_id) {
   auto it = bm->seqs.find(seq_id);
   if (it == bm->seqs.end())
     return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+  const std::vector<int32_t>& h = it->second.host;
+  for (auto b = h.rbegin(); b != h.rend(); ++b) bm->host_free.push_back(*b);
+  if (it->second.swapped) --bm->num_swapped;
   const std::vector<int32_t>& t = it->second.table;
   for (auto b = t.rbegin(); b != t.rend(); ++b)
     if (--bm->ref[*b] == 0) bm->free_stack.push_back(*b);
@@ -175,6 +196,7 @@ int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* 
     auto it = bm->seqs.find(seq_ids[i]);
     if (it == bm->seqs.end())
       return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_ids[i]);
+    if (it->second.swapped) return swapped_error(seq_ids[i]);
     if ((int64_t)it->second.table.size() > max_blocks)
       return fail(PA_ERR_INVALID_ARG, "sequence %lld holds %zu blocks > max_blocks %d",
                   (long long)seq_ids[i], it->second.table.size(), max_blocks);
@@ -210,6 +232,94 @@ int pa_bm_seq_len(const pa_bm* bm, int64_t seq_id) {
 }
 
 int pa_bm_num_seqs(const pa_bm* bm) { return bm ? (int)bm->seqs.size() : -1; }
+
+int pa_bm_set_host_pool(pa_bm* bm, int num_host_blocks) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  if (num_host_blocks < 0) return fail(PA_ERR_INVALID_ARG, "num_host_blocks must be >= 0");
+  if (bm->num_swapped > 0) return fail(PA_ERR_INVALID_ARG, "host blocks are in use");
+  bm->num_host_blocks = num_host_blocks;
+  bm->host_free.resize(num_host_blocks);
+  for (int i = 0; i < num_host_blocks; ++i) bm->host_free[num_host_blocks - 1 - i] = i;
+  return PA_OK;
+}
+
+int pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int64_t* pairs_out, int capacity, int* n_pairs) {
+  pa::clear_error();
+  if (!bm || !n_pairs) return fail(PA_ERR_INVALID_ARG, "null argument");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+  pa_bm::Seq& s = it->second;
+  if (s.swapped) return swapped_error(seq_id);
+  const int n = (int)s.table.size();
+  if (n > capacity || (n > 0 && !pairs_out))
+    return fail(PA_ERR_INVALID_ARG, "pairs_out holds %d pairs, %d needed", capacity, n);
+  if (n > (int)bm->host_free.size())
+    return fail(PA_ERR_NO_FREE_BLOCKS, "need %d host blocks, %zu free", n, bm->host_free.size());
+  s.host.resize(n);
+  for (int i = 0; i < n; ++i) {
+    s.host[i] = bm->host_free.back();
+    bm->host_free.pop_back();
+    pairs_out[2 * i] = s.table[i];
+    pairs_out[2 * i + 1] = s.host[i];
+  }
+  for (int i = n - 1; i >= 0; --i)
+    if (--bm->ref[s.table[i]] == 0) bm->free_stack.push_back(s.table[i]);
+  s.table.clear();
+  s.swapped = true;
+  ++bm->num_swapped;
+  *n_pairs = n;
+  return PA_OK;
+}
+
+int pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int64_t* pairs_out, int capacity, int* n_pairs) {
+  pa::clear_error();
+  if (!bm || !n_pairs) return fail(PA_ERR_INVALID_ARG, "null argument");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+  pa_bm::Seq& s = it->second;
+  if (!s.swapped)
+    return fail(PA_ERR_SEQ_SWAPPED, "sequence %lld is not swapped out", (long long)seq_id);
+  const int n = (int)s.host.size();
+  if (n > capacity || (n > 0 && !pairs_out))
+    return fail(PA_ERR_INVALID_ARG, "pairs_out holds %d pairs, %d needed", capacity, n);
+  if (n > (int)bm->free_stack.size())
+    return fail(PA_ERR_NO_FREE_BLOCKS, "need %d blocks, %zu free", n, bm->free_stack.size());
+  s.table.resize(n);
+  for (int i = 0; i < n; ++i) {
+    s.table[i] = bm->pop();
+    pairs_out[2 * i] = s.host[i];
+    pairs_out[2 * i + 1] = s.table[i];
+  }
+  for (int i = n - 1; i >= 0; --i) bm->host_free.push_back(s.host[i]);
+  s.host.clear();
+  s.swapped = false;
+  --bm->num_swapped;
+  *n_pairs = n;
+  return PA_OK;
+}
+
+int pa_bm_is_swapped(const pa_bm* bm, int64_t seq_id) {
+  if (!bm) return -1;
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) {
+    fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_id);
+    return -1;
+  }
+  return it->second.swapped ? 1 : 0;
+}
+
+int pa_bm_num_free_host(const pa_bm* bm) { return bm ? (int)bm->host_free.size() : -1; }
+
+int pa_bm_host_free_list(const pa_bm* bm, int32_t* out, int capacity) {
+  if (!bm || (!out && capacity > 0) || capacity < 0) return -1;
+  const int n = (int)bm->host_free.size();
+  const int m = n < capacity ? n : capacity;
+  for (int i = 0; i < m; ++i) out[i] = bm->host_free[n - 1 - i];
+  return m;
+}
 
 int pa_bm_free_list(const pa_bm* bm, int32_t* out, int capacity) {
   if (!bm || (!out && capacity > 0) || capacity < 0) return -1;

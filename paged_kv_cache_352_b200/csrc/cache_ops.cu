@@ -10,6 +10,10 @@
 // copy_blocks: a shared block is duplicated only when one sharer must write to
 // it, as with fork and copy-on-write ("Pages, from operating systems"; "The OS
 // paging analogy", page sharing).
+//
+// swap_blocks: the same copy between two pools, the device pool and a pinned
+// host pool, to preempt a request by swapping its blocks to CPU memory ("The OS
+// paging analogy", swapping).
 #include <cuda_runtime.h>
 
 #include "pa_device.cuh"
@@ -52,10 +56,14 @@ constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;
 
 // grid = (chunks of one pair's K+V bytes, pair). Each thread copies kCopyUnroll
-// 16-byte vectors; the first half of the index space is the K block, the second V.
+// 16-byte vectors from block src of the source pool to block dst of the
+// destination pool; the first half of the index space is the K block, the
+// second V. The two pools are the same for copy-on-write copies and differ
+// (device <-> pinned host) for swapping; plain loads, since host memory may be
+// on either side.
 __global__ void __launch_bounds__(kCopyThreads)
-    copy_blocks_kernel(uint4* k_cache, uint4* v_cache, const __grid_constant__ CopyPairs pairs,
-                       int64_t vecs_per_block) {
+    copy_pool_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* dst_v,
+                            const __grid_constant__ CopyPairs pairs, int64_t vecs_per_block) {
   const int pair = blockIdx.y;
   const int64_t src = pairs.src[pair];
   const int64_t dst = pairs.dst[pair];
@@ -68,9 +76,9 @@ __global__ void __launch_bounds__(kCopyThreads)
     live[u] = i < 2 * vecs_per_block;
     if (live[u]) {
       const bool is_v = i >= vecs_per_block;
-      const uint4* cache = is_v ? v_cache : k_cache;
+      const uint4* pool = is_v ? src_v : src_k;
       const int64_t off = is_v ? i - vecs_per_block : i;
-      buf[u] = __ldg(cache + src * vecs_per_block + off);
+      buf[u] = pool[src * vecs_per_block + off];
     }
   }
 #pragma unroll
@@ -78,9 +86,9 @@ __global__ void __launch_bounds__(kCopyThreads)
     const int64_t i = base + (int64_t)u * kCopyThreads;
     if (live[u]) {
       const bool is_v = i >= vecs_per_block;
-      uint4* cache = is_v ? v_cache : k_cache;
+      uint4* pool = is_v ? dst_v : dst_k;
       const int64_t off = is_v ? i - vecs_per_block : i;
-      cache[dst * vecs_per_block + off] = buf[u];
+      pool[dst * vecs_per_block + off] = buf[u];
     }
   }
 }
@@ -105,15 +113,17 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, int64_t
   return cudaGetLastError();
 }
 
-cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const CopyPairs& pairs, int n,
-                               int64_t block_bytes, cudaStream_t stream) {
+cudaError_t launch_copy_pool_blocks(const void* src_k, const void* src_v, void* dst_k,
+                                    void* dst_v, const CopyPairs& pairs, int n,
+                                    int64_t block_bytes, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
   const int64_t vecs = block_bytes / 16;
   const int64_t per_cta = (int64_t)kCopyThreads * kCopyUnroll;
   const int64_t gx = (2 * vecs + per_cta - 1) / per_cta;
   dim3 grid((unsigned)gx, (unsigned)n);
-  copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(static_cast<uint4*>(k_cache),
-                                                        static_cast<uint4*>(v_cache), pairs, vecs);
+  copy_pool_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(
+      static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v),
+      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), pairs, vecs);
   return cudaGetLastError();
 }
 

@@ -44,6 +44,28 @@ int check_cache_shape(int num_kv_heads, int head_dim, int block_size, int num_bl
   return PA_OK;
 }
 
+// Device-addressable form of a pool pointer: device or managed memory as is,
+// pinned host memory through its device alias; pageable memory is refused.
+int device_view(const void* p, const char* name, void** out) {
+  cudaPointerAttributes attr;
+  const cudaError_t e = cudaPointerGetAttributes(&attr, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // the query's error is not sticky: clear it
+    return fail(PA_ERR_INVALID_ARG, "%s: not memory the GPU can address (%s)", name,
+                cudaGetErrorString(e));
+  }
+  if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+    *out = const_cast<void*>(p);
+    return PA_OK;
+  }
+  if (attr.type == cudaMemoryTypeHost && attr.devicePointer != nullptr) {
+    *out = attr.devicePointer;
+    return PA_OK;
+  }
+  return fail(PA_ERR_INVALID_ARG,
+              "%s: not memory the GPU can address (pageable host memory must be pinned)", name);
+}
+
 int cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return PA_OK;
   return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -172,9 +194,56 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
       cp.src[i] = (int32_t)pairs[2 * (first + i)];
       cp.dst[i] = (int32_t)pairs[2 * (first + i) + 1];
     }
-    if (int st = cuda_status(launch_copy_blocks(k_cache, v_cache, cp, n, block_bytes,
-                                                static_cast<cudaStream_t>(stream)),
+    if (int st = cuda_status(launch_copy_pool_blocks(k_cache, v_cache, k_cache, v_cache, cp, n,
+                                                     block_bytes, static_cast<cudaStream_t>(stream)),
                              "copy_blocks launch"))
+      return st;
+  }
+  return PA_OK;
+}
+
+int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, void* dst_k,
+                   void* dst_v, int dst_num_blocks, const int64_t* pairs, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int dtype, void* stream) {
+  clear_error();
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, src_num_blocks, dtype))
+    return st;
+  if (dst_num_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "dst_num_blocks must be positive");
+  if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs must be >= 0");
+  if (num_pairs == 0) return PA_OK;
+  if (!src_k || !src_v || !dst_k || !dst_v || !pairs)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (src_k == dst_k || src_v == dst_v || src_k == dst_v || src_v == dst_k)
+    return fail(PA_ERR_INVALID_ARG, "source and destination must be different pools");
+  if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v))
+    return fail(PA_ERR_INVALID_ARG, "pool pointers must be 16-byte aligned");
+  std::unordered_set<int64_t> dsts;
+  dsts.reserve(num_pairs * 2);
+  for (int i = 0; i < num_pairs; ++i) {
+    const int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+    if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks)
+      return fail(PA_ERR_INVALID_ARG, "pair %d (%lld -> %lld) outside the pools (%d, %d blocks)",
+                  i, (long long)s, (long long)d, src_num_blocks, dst_num_blocks);
+    if (!dsts.insert(d).second)
+      return fail(PA_ERR_INVALID_ARG, "destination block %lld appears twice", (long long)d);
+  }
+  void *sk, *sv, *dk, *dv;
+  if (int st = device_view(src_k, "src_k", &sk)) return st;
+  if (int st = device_view(src_v, "src_v", &sv)) return st;
+  if (int st = device_view(dst_k, "dst_k", &dk)) return st;
+  if (int st = device_view(dst_v, "dst_v", &dv)) return st;
+  const int64_t block_bytes = (int64_t)num_kv_heads * kBlockSize * head_dim * 2;
+  for (int first = 0; first < num_pairs; first += kMaxCopyPairsPerLaunch) {
+    const int n = std::min(kMaxCopyPairsPerLaunch, num_pairs - first);
+    CopyPairs cp;
+    for (int i = 0; i < n; ++i) {
+      cp.src[i] = (int32_t)pairs[2 * (first + i)];
+      cp.dst[i] = (int32_t)pairs[2 * (first + i) + 1];
+    }
+    if (int st = cuda_status(
+            launch_copy_pool_blocks(sk, sv, dk, dv, cp, n, block_bytes,
+                                    static_cast<cudaStream_t>(stream)),
+            "swap_blocks launch"))
       return st;
   }
   return PA_OK;

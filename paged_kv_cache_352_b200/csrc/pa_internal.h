@@ -74,7 +74,10 @@ struct CopyPairs {
   int32_t dst[kMaxCopyPairsPerLaunch];
 };
 
-cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const CopyPairs& pairs, int n,
-                               int64_t block_bytes, cudaStream_t stream);
+// Copies block pairs.src[i] of the source pool over block pairs.dst[i] of the
+// destination pool (K and V); the pools may be the same (copy-on-write).
+cudaError_t launch_copy_pool_blocks(const void* src_k, const void* src_v, void* dst_k,
+                                    void* dst_v, const CopyPairs& pairs, int n,
+                                    int64_t block_bytes, cudaStream_t stream);
 
 }  // namespace pa

@@ -85,6 +85,46 @@ def test_copy_blocks_rejects_bad_pairs(pairs, why):
     assert st == L.PA_ERR_INVALID_ARG and why in L.last_error()
 
 
+@pytest.mark.parametrize("pairs,why", [
+    ([(0, 10)], "outside"),        # destination pool has 10 blocks
+    ([(64, 1)], "outside"),        # source pool has 64 blocks
+    ([(0, 3), (1, 3)], "twice"),
+])
+def test_swap_blocks_rejects_bad_pairs(pairs, why):
+    arr, ptr = _pairs(pairs)
+    other = ctypes.c_void_p(8192)
+    st = L.lib().pa_swap_blocks(FAKE, FAKE, 64, other, other, 10, ptr, len(arr), 8, 128, 16,
+                                L.PA_F16, None)
+    assert st == L.PA_ERR_INVALID_ARG and why in L.last_error()
+
+
+def test_swap_blocks_refuses_same_pool():
+    arr, ptr = _pairs([(0, 1)])
+    st = L.lib().pa_swap_blocks(FAKE, FAKE, 64, FAKE, FAKE, 64, ptr, 1, 8, 128, 16, L.PA_F16,
+                                None)
+    assert st == L.PA_ERR_INVALID_ARG and "different pools" in L.last_error()
+
+
+def test_block_manager_swap_errors():
+    bm = pa.BlockManager(8, 16)
+    bm.set_host_pool(2)
+    bm.add_seq(1, 40)                      # 3 blocks > 2 host blocks
+    with pytest.raises(pa.PAError) as e:
+        bm.swap_out(1)
+    assert e.value.code == L.PA_ERR_NO_FREE_BLOCKS and not bm.is_swapped(1)
+    bm.add_seq(2, 20)
+    bm.swap_out(2)
+    for op in (lambda: bm.append_slots(2, 1), lambda: bm.fork(2, 3),
+               lambda: bm.block_tables([2], 4), lambda: bm.swap_out(2)):
+        with pytest.raises(pa.PAError) as e:
+            op()
+        assert e.value.code == L.PA_ERR_SEQ_SWAPPED
+    with pytest.raises(pa.PAError):
+        bm.set_host_pool(8)                # host blocks in use
+    bm.free_seq(2)
+    assert bm.num_free_host() == 2
+
+
 def test_copy_blocks_zero_pairs_is_noop():
     assert L.lib().pa_copy_blocks(FAKE, FAKE, None, 0, 8, 128, 16, 64, L.PA_F16, None) == L.PA_OK
 
@@ -138,6 +178,10 @@ def test_workspace_size_formula():
 def _same_state(cbm, obm, seqs):
     assert cbm.num_free() == obm.num_free()
     assert cbm.free_list() == obm.free_list()
+    assert cbm.num_free_host() == obm.num_free_host()
+    assert cbm.host_free_list() == obm.host_free_list()
+    for s in seqs:
+        assert cbm.is_swapped(s) == obm.is_swapped(s)
     for b in range(obm.num_blocks):
         assert cbm.refcount(b) == obm.refcount(b)
     for s in seqs:
@@ -152,9 +196,11 @@ def test_block_manager_matches_oracle(seed):
     order = rng.permutation(nb)
     cbm = pa.BlockManager(nb, bs, order)
     obm = OBM.BlockManager(nb, bs, order)
+    cbm.set_host_pool(40)
+    obm.set_host_pool(40)
     live, nid = [], 1000
-    for it in range(800):
-        op = int(rng.integers(0, 5))
+    for it in range(1200):
+        op = int(rng.integers(0, 7))
         if op == 0 or not live:
             n = int(rng.integers(0, 70))
             args = ("add_seq", nid, n)
@@ -162,8 +208,12 @@ def test_block_manager_matches_oracle(seed):
             args = ("fork", live[int(rng.integers(len(live)))], nid)
         elif op in (2, 3):
             args = ("append_slots", live[int(rng.integers(len(live)))], int(rng.integers(0, 25)))
-        else:
+        elif op == 4:
             args = ("free_seq", live[int(rng.integers(len(live)))])
+        elif op == 5:
+            args = ("swap_out", live[int(rng.integers(len(live)))])
+        else:
+            args = ("swap_in", live[int(rng.integers(len(live)))])
         oerr = cerr = None
         try:
             ores = getattr(obm, args[0])(*args[1:])
@@ -187,9 +237,12 @@ def test_block_manager_matches_oracle(seed):
                 assert [tuple(p) for p in cres[1].tolist()] == [tuple(p) for p in ores[1]]
             elif args[0] == "free_seq":
                 live.remove(args[1])
+            elif args[0] in ("swap_out", "swap_in"):
+                assert [tuple(p) for p in cres.tolist()] == [tuple(p) for p in ores]
         _same_state(cbm, obm, live)
-    mb = max([len(obm.table(s)) for s in live] + [1])
-    assert np.array_equal(cbm.block_tables(live, mb + 2), obm.block_tables(live, mb + 2))
+    resident = [s for s in live if not obm.is_swapped(s)]
+    mb = max([len(obm.table(s)) for s in resident] + [1])
+    assert np.array_equal(cbm.block_tables(resident, mb + 2), obm.block_tables(resident, mb + 2))
 
 
 def test_block_manager_errors_and_queries():

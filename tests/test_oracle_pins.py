@@ -211,6 +211,61 @@ def pin_no_two_writers_share_a_slot():
         seen |= set(slots)
 
 
+def pin_swap_bookkeeping():
+    bm = BMmod.BlockManager(8, 16, [3, 1, 4, 0, 5, 2, 7, 6])
+    bm.set_host_pool(5)
+    bm.add_seq(1, 40)                     # blocks 3, 1, 4
+    bm.fork(1, 2)                         # shared
+    pairs = bm.swap_out(1)
+    assert pairs == [(3, 0), (1, 1), (4, 2)] and bm.is_swapped(1)
+    assert bm.table(2) == [3, 1, 4] and all(bm.refcount(b) == 1 for b in (3, 1, 4))
+    assert bm.num_free() == 5 and bm.num_free_host() == 2 and bm.seq_len(1) == 40
+    for op in (lambda: bm.append_slots(1, 1), lambda: bm.fork(1, 9), lambda: bm.swap_out(1),
+               lambda: bm.block_tables([1], 4)):
+        with pytest.raises(BMmod.BlockManagerError) as e:
+            op()
+        assert e.value.code == BMmod.ERR_SEQ_SWAPPED
+    with pytest.raises(BMmod.BlockManagerError) as e:
+        bm.swap_in(2)                     # resident
+    assert e.value.code == BMmod.ERR_SEQ_SWAPPED
+    bm.free_seq(2)                        # releases 4, 1, 3 (last first) -> 3 on top
+    pairs = bm.swap_in(1)
+    assert pairs == [(0, 3), (1, 1), (2, 4)] and not bm.is_swapped(1)
+    assert bm.num_free_host() == 5 and bm.host_free_list() == [0, 1, 2, 3, 4]
+    # host pool exhaustion leaves everything unchanged
+    bm.add_seq(5, 80)                     # 5 blocks -> 0 device blocks left
+    with pytest.raises(BMmod.BlockManagerError) as e:
+        bm.swap_out(5) if bm.num_free_host() < 5 else (bm.set_host_pool(0), bm.swap_out(5))
+    assert e.value.code in (BMmod.ERR_NO_FREE_BLOCKS, BMmod.ERR_INVALID_ARG)
+    assert not bm.is_swapped(5) and len(bm.table(5)) == 5
+
+
+def pin_swap_round_trip():
+    """Swap out, let another sequence overwrite the freed blocks, swap in: the
+    sequence's logical keys/values and its decode output are unchanged."""
+    rng = np.random.default_rng(17)
+    nb, hkv, d = 12, 2, 8
+    kc = gen.f32_to_bits(rng.standard_normal((nb, hkv, 16, d)).astype(np.float32), "f16")
+    vc = gen.f32_to_bits(rng.standard_normal((nb, hkv, 16, d)).astype(np.float32), "f16")
+    hk = np.zeros((6, hkv, 16, d), np.uint16)
+    hv = np.zeros_like(hk)
+    q = gen.f32_to_bits(rng.standard_normal((1, hkv, d)).astype(np.float32), "f16")
+    bm = BMmod.BlockManager(nb, 16, rng.permutation(nb))
+    bm.set_host_pool(6)
+    bm.add_seq(0, 37)
+    before_k = A.gather_sequence(kc, bm.table(0), 37, 1, 16).copy()
+    before = A.paged_decode(q, kc, vc, bm.block_tables([0], 3), [37], 0.3, "f16")
+    C.swap_blocks(kc, vc, hk, hv, bm.swap_out(0))
+    bm.add_seq(1, 16 * nb)                 # takes every device block, including the freed ones
+    noise = gen.f32_to_bits(rng.standard_normal((16 * nb, hkv, d)).astype(np.float32), "f16")
+    C.reshape_and_cache(kc, vc, noise, noise, list(range(16 * nb)), 16)
+    bm.free_seq(1)
+    C.swap_blocks(hk, hv, kc, vc, bm.swap_in(0))
+    assert np.array_equal(A.gather_sequence(kc, bm.table(0), 37, 1, 16), before_k)
+    after = A.paged_decode(q, kc, vc, bm.block_tables([0], 3), [37], 0.3, "f16")
+    assert np.array_equal(before, after)
+
+
 # --------------------------------------------------------------------------
 # cache writes and block copies
 # --------------------------------------------------------------------------
@@ -518,7 +573,18 @@ def _free_first_to_last(self, seq_id):
     del self._lens[seq_id]
 
 
+def _swap_in_reversed(self, seq_id):
+    pairs = _ORIG_SWAP_IN(self, seq_id)
+    table = self._tables[seq_id]
+    table.reverse()
+    return [(h, b) for (h, _), b in zip(pairs, table)]
+
+
+_ORIG_SWAP_IN = BMmod.BlockManager.swap_in
+
+
 MISTAKES = {
+    "swap_in_reversed": (BMmod.BlockManager, "swap_in", _swap_in_reversed),
     "dropped_scale": (A, "softmax_attention", _softmax_no_scale),
     "k_v_swapped": (A, "softmax_attention", _softmax_kv_swapped),
     "gather_block_offset_transposed": (A, "gather_sequence", _gather_transposed),
