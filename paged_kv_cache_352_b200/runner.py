@@ -226,3 +226,74 @@ class HostStep:
         r.step()
         self.h_out.copy_(r.out, non_blocking=True)
         return self.h_out
+
+
+class HostPipeline:
+    """Steps fed from pinned host memory with the copies overlapped.
+
+    Two slots each hold a step's inputs (pinned host and device copies) and its
+    output. Step k uses slot k % 2: an upload stream copies the slot's inputs
+    host -> device, the current stream waits for them and runs the step's
+    kernels into the slot's output, and a download stream copies that output
+    device -> host. Step k + 1's upload thus runs while step k computes, and
+    step k's download while step k + 1 computes. Every step still moves all of
+    its inputs and its output across the host link; a slot is reused only after
+    its previous output has reached the host.
+    """
+
+    FIELDS = ("q", "step_k", "step_v", "step_slots", "block_tables", "context_lens", "seq_order")
+
+    def __init__(self, runner: DecodeRunner):
+        r = self.r = runner
+        self.compute = torch.cuda.current_stream(r.device)
+        self.upload = torch.cuda.Stream(r.device)
+        self.download = torch.cuda.Stream(r.device)
+        self.slots = []
+        for _ in range(2):
+            offs, total = [], 0
+            for name in self.FIELDS:
+                t = getattr(r, name)
+                offs.append(total)
+                total += -(-t.numel() * t.element_size() // 256) * 256
+            h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+            d_buf = torch.empty(total, dtype=torch.uint8, device=r.device)
+            views = {}
+            for name, off in zip(self.FIELDS, offs):
+                t = getattr(r, name)
+                n = t.numel() * t.element_size()
+                h_buf[off:off + n].view(t.dtype).view(t.shape).copy_(t.cpu())
+                views[name] = d_buf[off:off + n].view(t.dtype).view(t.shape)
+            self.slots.append({
+                "h_buf": h_buf, "d_buf": d_buf, "views": views,
+                "out": torch.empty_like(r.out),
+                "h_out": torch.empty(r.out.shape, dtype=r.dtype).pin_memory(),
+                "in_ready": torch.cuda.Event(), "out_ready": torch.cuda.Event(),
+                "free": torch.cuda.Event(),
+            })
+            self.h2d_bytes = total
+        self.d2h_bytes = self.slots[0]["h_out"].numel() * self.slots[0]["h_out"].element_size()
+        for sl in self.slots:
+            sl["free"].record(self.download)
+        self.k = 0
+        torch.cuda.synchronize(r.device)
+
+    def __call__(self):
+        r = self.r
+        sl = self.slots[self.k % 2]
+        self.k += 1
+        with torch.cuda.stream(self.upload):
+            self.upload.wait_event(sl["free"])
+            sl["d_buf"].copy_(sl["h_buf"], non_blocking=True)
+            sl["in_ready"].record(self.upload)
+        self.compute.wait_event(sl["in_ready"])
+        for name, v in sl["views"].items():
+            setattr(r, name, v)
+        r.copy_blocks()
+        r.reshape_and_cache()
+        r.decode(out=sl["out"])
+        sl["out_ready"].record(self.compute)
+        with torch.cuda.stream(self.download):
+            self.download.wait_event(sl["out_ready"])
+            sl["h_out"].copy_(sl["out"], non_blocking=True)
+            sl["free"].record(self.download)
+        return sl["h_out"]

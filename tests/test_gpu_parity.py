@@ -332,3 +332,16 @@ def test_bad_order_entries_are_flagged():
     assert err.item() & pa.PA_DEVERR_CONTEXT_RANGE
     ref = _oracle_manual(q, kc, vc, tables, cl, 0.1, torch.bfloat16)
     assert_close(out_to_f64(out[1:], "bf16"), ref[1:])   # sequence 1 was still computed
+
+
+def test_host_pipeline_returns_each_steps_output():
+    from paged_kv_cache_352_b200.runner import HostPipeline
+    wl = workloads.workload("gqa_32_8_bf16", small=True)
+    r = DecodeRunner(wl)
+    ref = r.step().clone()
+    hp = HostPipeline(r)
+    outs = [hp() for _ in range(4)]
+    _sync()
+    for o in outs[-2:]:
+        assert torch.equal(o.view(torch.int16), ref.cpu().view(torch.int16))
+    assert hp.h2d_bytes >= (r.q.numel() + r.step_k.numel() + r.step_v.numel()) * 2
