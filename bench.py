@@ -400,6 +400,64 @@ def measure_swap(wl, r, device, nblocks: int = 2048, reps: int = 5):
     return res
 
 
+def measure_prefix_cache(wl, device, requests: int = 64, prompts: int = 4,
+                         prompt_len: int = 1024, own_len: int = 256, reps: int = 5):
+    """Prefix caching on a synthetic request trace: ``requests`` requests, each a
+    ``prompt_len``-token prompt drawn from ``prompts`` shared system prompts plus
+    ``own_len`` tokens of its own, admitted through the block manager's prefix
+    cache. Reports the share of prompt tokens found cached, and the device time
+    of the one cache-write launch that stores every admitted request's new
+    tokens, with the cache (suffixes only) and without it (whole prompts)."""
+    import torch
+    from paged_kv_cache_352_b200 import _lib as L
+    rng = np.random.default_rng(11)
+    sys_toks = [rng.integers(0, 32000, prompt_len).tolist() for _ in range(prompts)]
+    own = [rng.integers(0, 32000, own_len).tolist() for _ in range(requests)]
+    nblk = requests * (-(-(prompt_len + own_len) // 16))
+    shape = (nblk, wl.num_kv_heads, 16, wl.head_dim)
+    dt = torch.float16 if wl.dtype == "f16" else torch.bfloat16
+    kc = torch.zeros(shape, dtype=dt, device=device)
+    vc = torch.zeros_like(kc)
+    row_bytes = wl.num_kv_heads * wl.head_dim * 2
+
+    def admit(cached_mode):
+        bm = L.BlockManager(nblk, 16)
+        slots_all, total, hit = [], 0, 0
+        for r in range(requests):
+            toks = sys_toks[r % prompts] + own[r]
+            if cached_mode:
+                slots, c = bm.add_seq_cached(r, toks)
+            else:
+                slots, c = bm.add_seq(r, len(toks)), 0
+            slots_all.append(np.asarray(slots[c:], np.int64))
+            total += len(toks)
+            hit += c
+        sl = torch.from_numpy(np.concatenate(slots_all)).to(device)
+        kv = torch.randn((sl.numel(), wl.num_kv_heads, wl.head_dim), device=device).to(dt)
+        L.pa_reshape_and_cache(kv, kv, kc, vc, sl)             # warm-up
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(reps):
+            L.pa_reshape_and_cache(kv, kv, kc, vc, sl)
+        ev[1].record()
+        torch.cuda.synchronize(device)
+        ms = ev[0].elapsed_time(ev[1]) / reps
+        return hit, total, sl.numel(), ms
+
+    hit, total, n_c, t_c = admit(True)
+    _, _, n_p, t_p = admit(False)
+    # bytes moved by one write launch: K and V rows read and written once each
+    gbs = lambda n, ms: round(4 * n * row_bytes / (ms * 1e6), 1)
+    return {"requests": requests, "prompt_tokens": total, "cached_tokens": hit,
+            "hit_rate": round(hit / total, 4),
+            "written_tokens_with_cache": n_c, "written_tokens_without_cache": n_p,
+            "write_ms_with_cache": round(t_c, 4), "write_ms_without_cache": round(t_p, 4),
+            "write_gbs_with_cache": gbs(n_c, t_c), "write_gbs_without_cache": gbs(n_p, t_p),
+            "what": f"{requests} requests = one of {prompts} shared {prompt_len}-token prompts "
+                    f"+ {own_len} own tokens, admitted through pa_bm_add_seq_cached; "
+                    f"one pa_reshape_and_cache launch stores all new tokens"}
+
+
 def run_reference(args):
     rank, world, _ = _rank_info()
     if rank != 0:
@@ -525,6 +583,7 @@ def run_ours(args):
     e2e_s = _max_over_ranks(e_start.elapsed_time(e_end) / 1e3 / E, world, device)
 
     swap = measure_swap(wl, r, device) if world == 1 else None
+    prefix_cache = measure_prefix_cache(wl, device) if world == 1 else None
 
     sb = step_bytes(wl, r)
     db = decode_bytes(wl)
@@ -572,6 +631,7 @@ def run_ours(args):
                 "ms_per_step": round(e2e_s * 1e3, 4)},
         "gpu_launches": K * launches_per_step,
         "swap": swap,
+        "prefix_cache": prefix_cache,
         "clocks": csum,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -315,8 +315,30 @@ int pa_bm_num_free_host(const pa_bm* bm);
 /* Free host blocks in hand-out order into out[capacity]; returns the count or -1. */
 int pa_bm_host_free_list(const pa_bm* bm, int32_t* out, int capacity);
 
+/* Prefix caching across requests: the KV of shared prompt prefixes is kept and
+ * reused by later requests, so a hit makes prefill nearly free
+ * ("PagedAttention: The vLLM Paper", "Impact and Follow-Ups", item 1).
+ * pa_bm_add_seq_cached registers seq_id from its prompt's token_ids. Every full
+ * block of the prompt is identified exactly by (physical block of the previous
+ * logical block or -1, its block_size token ids); the leading full blocks found
+ * in the cache are shared (refcount + 1), the rest get fresh blocks, and the new
+ * full blocks join the cache. The partly filled last block is never cached, so
+ * no write ever touches a cached block. slots_out[num_tokens] receives every
+ * token's slot; *num_cached_tokens = the leading tokens whose keys and values
+ * are already in the pool (only the rest need pa_reshape_and_cache).
+ * A cached block whose refcount falls to 0 is kept for reuse on a queue, least
+ * recently released first, and counts as free; blocks are taken from the free
+ * list first, then by evicting the queue's head (with any cached descendants).
+ * All-or-nothing like the other calls. */
+int pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* token_ids, int num_tokens,
+                         int64_t* slots_out, int* num_cached_tokens);
+int pa_bm_num_cached(const pa_bm* bm);
+/* Evictable cached blocks, oldest first, into out[capacity]; returns the count or -1. */
+int pa_bm_evictable_list(const pa_bm* bm, int32_t* out, int capacity);
+
 /* Queries. pa_bm_refcount and pa_bm_seq_len return -1 for an unknown block or
- * sequence (and set pa_last_error). */
+ * sequence (and set pa_last_error). pa_bm_num_free counts free blocks plus cached
+ * blocks kept for reuse. */
 int pa_bm_num_free(const pa_bm* bm);
 int pa_bm_refcount(const pa_bm* bm, int32_t block);
 int pa_bm_seq_len(const pa_bm* bm, int64_t seq_id);

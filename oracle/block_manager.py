@@ -45,6 +45,26 @@ Essentials" and "The OS paging analogy", swapping), read as:
     the host free list, last logical block first.
   * A swapped sequence cannot append, fork, be swapped out again or appear in
     block tables; ``free_seq`` releases its host blocks.
+
+Prefix caching across requests (the KV of shared prompt prefixes is kept and
+reused by later requests, so a hit makes prefill nearly free — "PagedAttention:
+The vLLM Paper", "Impact and Follow-Ups", item 1), read as:
+  * ``add_seq_cached`` takes the prompt's token ids. Every full block of the
+    prompt is identified exactly by (physical block of the previous logical
+    block, or -1 for the first; the block's 16 token ids). Leading full blocks
+    found in the cache are shared (refcount + 1); the first miss and everything
+    after it get fresh blocks, and the new full blocks join the cache. The
+    partly filled last block is never cached, so writes never touch a cached
+    block. The call reports how many leading tokens need no write.
+  * A cached block whose refcount falls to 0 is not freed but kept for reuse,
+    queued least recently released first. Blocks are taken from the free list
+    first and, when it is empty, by evicting the head of that queue. Tables are
+    released last block first and a table holding a block holds its whole
+    prefix, so a block is never queued before its cached descendants and
+    eviction takes leaves first; evicting a block nevertheless also evicts any
+    cached descendant, so no cache key can name a block that now holds other
+    tokens.
+  * ``num_free`` counts free plus evictable blocks.
 """
 
 from __future__ import annotations
@@ -91,6 +111,10 @@ class BlockManager:
         self._host_free: list[int] = []
         self.num_host_blocks = 0
         self._swapped: dict[int, list[int]] = {}   # seq -> host blocks in logical order
+        self._cache: dict = {}          # (parent block, tokens) -> block
+        self._key_of: dict = {}         # cached block -> its key
+        self._children: dict = {}       # cached block -> set of cached child blocks
+        self._evictable: list[int] = [] # cached blocks with refcount 0, oldest first
 
     def set_host_pool(self, num_host_blocks: int) -> None:
         if num_host_blocks < 0:
@@ -117,9 +141,7 @@ class BlockManager:
         host = [self._host_free.pop() for _ in table]
         pairs = list(zip(table, host))
         for b in reversed(table):
-            self._ref[b] -= 1
-            if self._ref[b] == 0:
-                self._free.append(b)
+            self._release(b)
         self._tables[seq_id] = []
         self._swapped[seq_id] = host
         return pairs
@@ -130,13 +152,9 @@ class BlockManager:
         if seq_id not in self._swapped:
             raise BlockManagerError(ERR_SEQ_SWAPPED, f"sequence {seq_id} is not swapped out")
         host = self._swapped[seq_id]
-        if len(host) > len(self._free):
+        if len(host) > self.num_free():
             raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
-        table = []
-        for _ in host:
-            b = self._free.pop()
-            self._ref[b] = 1
-            table.append(b)
+        table = [self._take() for _ in host]
         pairs = list(zip(host, table))
         for h in reversed(host):
             self._host_free.append(h)
@@ -150,7 +168,13 @@ class BlockManager:
 
     # -- queries ---------------------------------------------------------
     def num_free(self) -> int:
-        return len(self._free)
+        return len(self._free) + len(self._evictable)
+
+    def num_cached(self) -> int:
+        return len(self._key_of)
+
+    def evictable_list(self) -> list[int]:
+        return list(self._evictable)
 
     def refcount(self, block: int) -> int:
         if not 0 <= block < self.num_blocks:
@@ -184,6 +208,33 @@ class BlockManager:
         if seq_id not in self._tables:
             raise BlockManagerError(ERR_UNKNOWN_SEQ, f"unknown sequence {seq_id}")
 
+    def _take(self) -> int:
+        """A block for new tokens: the free list first, else evict the oldest
+        released cached block (with its cached descendants)."""
+        if not self._free:
+            self._evict(self._evictable[0])
+        b = self._free.pop()
+        self._ref[b] = 1
+        return b
+
+    def _evict(self, b: int) -> None:
+        for c in sorted(self._children.pop(b, ())):
+            self._evict(c)
+        key = self._key_of.pop(b)
+        del self._cache[key]
+        if key[0] >= 0:
+            self._children[key[0]].discard(b)
+        self._evictable.remove(b)
+        self._free.append(b)
+
+    def _release(self, b: int) -> None:
+        self._ref[b] -= 1
+        if self._ref[b] == 0:
+            if b in self._key_of:
+                self._evictable.append(b)
+            else:
+                self._free.append(b)
+
     def _slot(self, table, pos):
         return table[pos // self.block_size] * self.block_size + pos % self.block_size
 
@@ -195,16 +246,52 @@ class BlockManager:
         if seq_id in self._tables:
             raise BlockManagerError(ERR_SEQ_EXISTS, f"sequence {seq_id} exists")
         need = _ceil_div(num_tokens, self.block_size)
-        if need > len(self._free):
+        if need > self.num_free():
             raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
-        table = []
-        for _ in range(need):
-            b = self._free.pop()
-            self._ref[b] = 1
-            table.append(b)
+        table = [self._take() for _ in range(need)]
         self._tables[seq_id] = table
         self._lens[seq_id] = num_tokens
         return [self._slot(table, p) for p in range(num_tokens)]
+
+    def add_seq_cached(self, seq_id: int, token_ids):
+        """Register a sequence from its prompt's token ids, sharing the leading
+        full blocks already cached. Returns ``(slots, num_cached_tokens)``; the
+        first ``num_cached_tokens`` tokens' keys and values are already in place."""
+        tokens = [int(t) for t in token_ids]
+        n = len(tokens)
+        if seq_id in self._tables:
+            raise BlockManagerError(ERR_SEQ_EXISTS, f"sequence {seq_id} exists")
+        bs = self.block_size
+        full = n // bs
+        hits, parent = [], -1
+        for i in range(full):
+            b = self._cache.get((parent, tuple(tokens[i * bs:(i + 1) * bs])))
+            if b is None:
+                break
+            hits.append(b)
+            parent = b
+        need = _ceil_div(n, bs) - len(hits)
+        revived = sum(1 for b in hits if self._ref[b] == 0)
+        if need > self.num_free() - revived:
+            raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
+        for b in hits:
+            if self._ref[b] == 0:
+                self._evictable.remove(b)
+            self._ref[b] += 1
+        table = list(hits)
+        for i in range(len(hits), _ceil_div(n, bs)):
+            b = self._take()
+            table.append(b)
+            if i < full:
+                key = (parent, tuple(tokens[i * bs:(i + 1) * bs]))
+                self._cache[key] = b
+                self._key_of[b] = key
+                if parent >= 0:
+                    self._children.setdefault(parent, set()).add(b)
+                parent = b
+        self._tables[seq_id] = table
+        self._lens[seq_id] = n
+        return [self._slot(table, p) for p in range(n)], len(hits) * bs
 
     def fork(self, parent: int, child: int) -> None:
         """Child starts as a copy of the parent's table; every block is shared."""
@@ -229,22 +316,19 @@ class BlockManager:
         bs = self.block_size
         new_blocks = _ceil_div(length + n, bs) - len(table)
         cow = n > 0 and length % bs != 0 and self._ref[table[-1]] > 1
-        if new_blocks + int(cow) > len(self._free):
+        if new_blocks + int(cow) > self.num_free():
             raise BlockManagerError(ERR_NO_FREE_BLOCKS, "pool exhausted")
         pairs = []
         if cow:
             old = table[-1]
-            new = self._free.pop()
-            self._ref[old] -= 1
-            self._ref[new] = 1
+            new = self._take()
+            self._ref[old] -= 1   # still held by its other sharers
             table[-1] = new
             pairs.append((old, new))
         slots = []
         for p in range(length, length + n):
             if p % bs == 0:
-                b = self._free.pop()
-                self._ref[b] = 1
-                table.append(b)
+                table.append(self._take())
             slots.append(self._slot(table, p))
         self._lens[seq_id] = length + n
         return slots, pairs
@@ -254,9 +338,7 @@ class BlockManager:
         for h in reversed(self._swapped.pop(seq_id, [])):
             self._host_free.append(h)
         for b in reversed(self._tables[seq_id]):
-            self._ref[b] -= 1
-            if self._ref[b] == 0:
-                self._free.append(b)
+            self._release(b)
         del self._tables[seq_id]
         del self._lens[seq_id]
 

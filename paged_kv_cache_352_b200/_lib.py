@@ -82,6 +82,9 @@ _SIGS = {
     "pa_bm_is_swapped": (_c_int, [_vp, _c_i64]),
     "pa_bm_num_free_host": (_c_int, [_vp]),
     "pa_bm_host_free_list": (_c_int, [_vp, _vp, _c_int]),
+    "pa_bm_add_seq_cached": (_c_int, [_vp, _c_i64, _vp, _c_int, _vp, ctypes.POINTER(_c_int)]),
+    "pa_bm_num_cached": (_c_int, [_vp]),
+    "pa_bm_evictable_list": (_c_int, [_vp, _vp, _c_int]),
 }
 
 _LIB = None
@@ -404,6 +407,24 @@ class BlockManager:
             return []
         n = -(-self.seq_len(seq_id) // self.block_size)
         return self.block_tables([seq_id], max(n, 1))[0, :n].tolist()
+
+    # -- prefix caching ----------------------------------------------------------
+    def add_seq_cached(self, seq_id: int, token_ids):
+        """Register from prompt token ids; returns (slots, num_cached_tokens)."""
+        toks = np.ascontiguousarray(np.asarray(list(token_ids), dtype=np.int32))
+        slots = np.empty(max(len(toks), 1), np.int64)
+        cached = ctypes.c_int(0)
+        _check(self._lib.pa_bm_add_seq_cached(self._h, seq_id, toks.ctypes.data, len(toks),
+                                              slots.ctypes.data, ctypes.byref(cached)))
+        return slots[:len(toks)].copy(), cached.value
+
+    def num_cached(self) -> int:
+        return self._lib.pa_bm_num_cached(self._h)
+
+    def evictable_list(self) -> list:
+        out = np.empty(max(self.num_blocks, 1), np.int32)
+        n = self._lib.pa_bm_evictable_list(self._h, out.ctypes.data, self.num_blocks)
+        return out[:n].tolist()
 
     # -- swapping ----------------------------------------------------------------
     def set_host_pool(self, num_host_blocks: int) -> None:

@@ -14,11 +14,23 @@
 // blocks last first, swap-in emits (host, device) pairs and releases host blocks
 // last first. A swapped sequence cannot grow, fork or appear in block tables.
 //
+// Prefix caching across requests: the KV of shared prompt prefixes is kept and
+// reused by later requests ("PagedAttention: The vLLM Paper", "Impact and
+// Follow-Ups", item 1). A full prompt block is identified exactly by
+// (physical block of the previous logical block or -1, its token ids); a
+// sequence added with its token ids shares every leading block found. Cached
+// blocks whose refcount falls to 0 stay reusable on a queue, least recently
+// released first; blocks come from the free list first, then by evicting the
+// queue's head together with any cached descendants.
+//
 // Every mutating call first works out how many free blocks it needs and fails
 // before touching any state when the pool cannot cover it.
 #include <stdint.h>
 
+#include <list>
+#include <map>
 #include <new>
+#include <set>
 #include <unordered_map>
 #include <vector>
 
@@ -40,11 +52,53 @@ struct pa_bm {
   int num_host_blocks = 0;
   int num_swapped = 0;
 
+  // prefix cache: key = {parent block or -1, token ids of the block}
+  std::map<std::vector<int32_t>, int32_t> cache;
+  std::unordered_map<int32_t, std::vector<int32_t>> key_of;
+  std::unordered_map<int32_t, std::set<int32_t>> children;
+  std::list<int32_t> evictable;  // cached blocks with refcount 0, oldest first
+  std::unordered_map<int32_t, std::list<int32_t>::iterator> evictable_pos;
+
+  size_t num_free() const { return free_stack.size() + evictable.size(); }
+
+  void evict(int32_t b) {
+    auto ch = children.find(b);
+    if (ch != children.end()) {
+      const std::set<int32_t> kids = ch->second;  // ascending block ids
+      children.erase(ch);
+      for (int32_t c : kids) evict(c);
+    }
+    auto k = key_of.find(b);
+    const int32_t parent = k->second[0];
+    cache.erase(k->second);
+    key_of.erase(k);
+    if (parent >= 0) {
+      auto pc = children.find(parent);
+      if (pc != children.end()) pc->second.erase(b);
+    }
+    auto pos = evictable_pos.find(b);
+    evictable.erase(pos->second);
+    evictable_pos.erase(pos);
+    free_stack.push_back(b);
+  }
+
+  // A block for new tokens: the free list first, else the oldest released cached block.
   int32_t pop() {
+    if (free_stack.empty()) evict(evictable.front());
     const int32_t b = free_stack.back();
     free_stack.pop_back();
     ref[b] = 1;
     return b;
+  }
+
+  void release(int32_t b) {
+    if (--ref[b] != 0) return;
+    if (key_of.count(b)) {
+      evictable.push_back(b);
+      evictable_pos[b] = std::prev(evictable.end());
+    } else {
+      free_stack.push_back(b);
+    }
   }
   int64_t slot(const Seq& s, int64_t pos) const {
     return (int64_t)s.table[pos / block_size] * block_size + pos % block_size;
@@ -106,9 +160,9 @@ int pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int num_tokens, int64_t* slots_out)
   if (bm->seqs.count(seq_id))
     return fail(PA_ERR_SEQ_EXISTS, "sequence %lld exists", (long long)seq_id);
   const int64_t need = ceil_div(num_tokens, bm->block_size);
-  if (need > (int64_t)bm->free_stack.size())
+  if (need > (int64_t)bm->num_free())
     return fail(PA_ERR_NO_FREE_BLOCKS, "need %lld blocks, %zu free", (long long)need,
-                bm->free_stack.size());
+                bm->num_free());
   pa_bm::Seq s;
   s.table.reserve(need);
   for (int64_t i = 0; i < need; ++i) s.table.push_back(bm->pop());
@@ -148,9 +202,9 @@ int pa_bm_append_slots(pa_bm* bm, int64_t seq_id, int n, int64_t* slots_out,
   const int bs = bm->block_size;
   const int64_t new_blocks = ceil_div(s.len + n, bs) - (int64_t)s.table.size();
   const bool cow = n > 0 && s.len % bs != 0 && bm->ref[s.table.back()] > 1;
-  if (new_blocks + (cow ? 1 : 0) > (int64_t)bm->free_stack.size())
+  if (new_blocks + (cow ? 1 : 0) > (int64_t)bm->num_free())
     return fail(PA_ERR_NO_FREE_BLOCKS, "need %lld blocks, %zu free",
-                (long long)(new_blocks + (cow ? 1 : 0)), bm->free_stack.size());
+                (long long)(new_blocks + (cow ? 1 : 0)), bm->num_free());
   *n_cow = 0;
   if (cow) {
     const int32_t old = s.table.back();
@@ -179,8 +233,7 @@ int pa_bm_free_seq(pa_bm* bm, int64_t seq_id) {
   for (auto b = h.rbegin(); b != h.rend(); ++b) bm->host_free.push_back(*b);
   if (it->second.swapped) --bm->num_swapped;
   const std::vector<int32_t>& t = it->second.table;
-  for (auto b = t.rbegin(); b != t.rend(); ++b)
-    if (--bm->ref[*b] == 0) bm->free_stack.push_back(*b);
+  for (auto b = t.rbegin(); b != t.rend(); ++b) bm->release(*b);
   bm->seqs.erase(it);
   return PA_OK;
 }
@@ -211,7 +264,75 @@ int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* 
   return PA_OK;
 }
 
-int pa_bm_num_free(const pa_bm* bm) { return bm ? (int)bm->free_stack.size() : -1; }
+int pa_bm_num_free(const pa_bm* bm) { return bm ? (int)bm->num_free() : -1; }
+
+int pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* token_ids, int num_tokens,
+                         int64_t* slots_out, int* num_cached_tokens) {
+  pa::clear_error();
+  if (!bm || !num_cached_tokens) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0");
+  if (num_tokens > 0 && (!slots_out || !token_ids))
+    return fail(PA_ERR_INVALID_ARG, "null token_ids or slots_out");
+  if (bm->seqs.count(seq_id))
+    return fail(PA_ERR_SEQ_EXISTS, "sequence %lld exists", (long long)seq_id);
+  const int bs = bm->block_size;
+  const int full = num_tokens / bs;
+  std::vector<int32_t> hits;
+  std::vector<int32_t> key(bs + 1);
+  int32_t parent = -1;
+  for (int i = 0; i < full; ++i) {
+    key[0] = parent;
+    for (int t = 0; t < bs; ++t) key[1 + t] = token_ids[i * bs + t];
+    auto c = bm->cache.find(key);
+    if (c == bm->cache.end()) break;
+    hits.push_back(c->second);
+    parent = c->second;
+  }
+  const int64_t need = ceil_div(num_tokens, bs) - (int64_t)hits.size();
+  int64_t revived = 0;
+  for (int32_t b : hits) revived += bm->ref[b] == 0;
+  if (need > (int64_t)bm->num_free() - revived)
+    return fail(PA_ERR_NO_FREE_BLOCKS, "need %lld blocks, %lld free", (long long)need,
+                (long long)(bm->num_free() - revived));
+  for (int32_t b : hits) {
+    if (bm->ref[b] == 0) {
+      auto pos = bm->evictable_pos.find(b);
+      bm->evictable.erase(pos->second);
+      bm->evictable_pos.erase(pos);
+    }
+    ++bm->ref[b];
+  }
+  pa_bm::Seq s;
+  s.table = hits;
+  const int64_t nblk = ceil_div(num_tokens, bs);
+  for (int64_t i = (int64_t)hits.size(); i < nblk; ++i) {
+    const int32_t b = bm->pop();
+    s.table.push_back(b);
+    if (i < full) {
+      key[0] = parent;
+      for (int t = 0; t < bs; ++t) key[1 + t] = token_ids[i * bs + t];
+      bm->cache[key] = b;
+      bm->key_of[b] = key;
+      if (parent >= 0) bm->children[parent].insert(b);
+      parent = b;
+    }
+  }
+  s.len = num_tokens;
+  for (int64_t p = 0; p < num_tokens; ++p) slots_out[p] = bm->slot(s, p);
+  bm->seqs.emplace(seq_id, std::move(s));
+  *num_cached_tokens = (int)hits.size() * bs;
+  return PA_OK;
+}
+
+int pa_bm_num_cached(const pa_bm* bm) { return bm ? (int)bm->key_of.size() : -1; }
+
+int pa_bm_evictable_list(const pa_bm* bm, int32_t* out, int capacity) {
+  if (!bm || (!out && capacity > 0) || capacity < 0) return -1;
+  int i = 0;
+  for (auto it = bm->evictable.begin(); it != bm->evictable.end() && i < capacity; ++it)
+    out[i++] = *it;
+  return i;
+}
 
 int pa_bm_refcount(const pa_bm* bm, int32_t block) {
   if (!bm || block < 0 || block >= bm->num_blocks) {
@@ -264,8 +385,7 @@ int pa_bm_swap_out(pa_bm* bm, int64_t seq_id, int64_t* pairs_out, int capacity, 
     pairs_out[2 * i] = s.table[i];
     pairs_out[2 * i + 1] = s.host[i];
   }
-  for (int i = n - 1; i >= 0; --i)
-    if (--bm->ref[s.table[i]] == 0) bm->free_stack.push_back(s.table[i]);
+  for (int i = n - 1; i >= 0; --i) bm->release(s.table[i]);
   s.table.clear();
   s.swapped = true;
   ++bm->num_swapped;
@@ -285,8 +405,8 @@ int pa_bm_swap_in(pa_bm* bm, int64_t seq_id, int64_t* pairs_out, int capacity, i
   const int n = (int)s.host.size();
   if (n > capacity || (n > 0 && !pairs_out))
     return fail(PA_ERR_INVALID_ARG, "pairs_out holds %d pairs, %d needed", capacity, n);
-  if (n > (int)bm->free_stack.size())
-    return fail(PA_ERR_NO_FREE_BLOCKS, "need %d blocks, %zu free", n, bm->free_stack.size());
+  if (n > (int)bm->num_free())
+    return fail(PA_ERR_NO_FREE_BLOCKS, "need %d blocks, %zu free", n, bm->num_free());
   s.table.resize(n);
   for (int i = 0; i < n; ++i) {
     s.table[i] = bm->pop();

@@ -179,6 +179,8 @@ def _same_state(cbm, obm, seqs):
     assert cbm.num_free() == obm.num_free()
     assert cbm.free_list() == obm.free_list()
     assert cbm.num_free_host() == obm.num_free_host()
+    assert cbm.num_cached() == obm.num_cached()
+    assert cbm.evictable_list() == obm.evictable_list()
     assert cbm.host_free_list() == obm.host_free_list()
     for s in seqs:
         assert cbm.is_swapped(s) == obm.is_swapped(s)
@@ -199,9 +201,15 @@ def test_block_manager_matches_oracle(seed):
     cbm.set_host_pool(40)
     obm.set_host_pool(40)
     live, nid = [], 1000
-    for it in range(1200):
-        op = int(rng.integers(0, 7))
-        if op == 0 or not live:
+    prefixes = [rng.integers(0, 50, 64).tolist() for _ in range(3)]
+    for it in range(1500):
+        op = int(rng.integers(0, 8))
+        if op == 7:
+            base = prefixes[int(rng.integers(0, 3))]
+            keep = int(rng.integers(0, 65))
+            toks = base[:keep] + rng.integers(0, 50, int(rng.integers(0, 40))).tolist()
+            args = ("add_seq_cached", nid, toks)
+        elif op == 0 or not live:
             n = int(rng.integers(0, 70))
             args = ("add_seq", nid, n)
         elif op == 1:
@@ -229,6 +237,10 @@ def test_block_manager_matches_oracle(seed):
                 assert list(cres) == ores
                 live.append(nid)
                 nid += 1
+            elif args[0] == "add_seq_cached":
+                assert list(cres[0]) == ores[0] and cres[1] == ores[1]
+                live.append(nid)
+                nid += 1
             elif args[0] == "fork":
                 live.append(nid)
                 nid += 1
@@ -243,6 +255,18 @@ def test_block_manager_matches_oracle(seed):
     resident = [s for s in live if not obm.is_swapped(s)]
     mb = max([len(obm.table(s)) for s in resident] + [1])
     assert np.array_equal(cbm.block_tables(resident, mb + 2), obm.block_tables(resident, mb + 2))
+
+
+def test_prefix_cache_reuse_counts():
+    bm = pa.BlockManager(64, 16)
+    prompt = list(range(1000, 1100))                 # 6 full blocks + 4 tokens
+    _, c1 = bm.add_seq_cached(1, prompt)
+    _, c2 = bm.add_seq_cached(2, prompt + [5, 6])
+    assert (c1, c2) == (0, 96) and bm.table(2)[:6] == bm.table(1)[:6]
+    assert bm.num_cached() == 6
+    bm.free_seq(1)
+    bm.free_seq(2)
+    assert bm.num_free() == 64 and len(bm.evictable_list()) == 6
 
 
 def test_block_manager_errors_and_queries():

@@ -266,6 +266,86 @@ def pin_swap_round_trip():
     assert np.array_equal(before, after)
 
 
+def pin_prefix_cache_hits():
+    bm = BMmod.BlockManager(32, 16)
+    P = list(range(100, 140))                       # 40 tokens: 2 full blocks + 8
+    s1, c1 = bm.add_seq_cached(1, P)
+    assert c1 == 0 and bm.num_cached() == 2
+    s2, c2 = bm.add_seq_cached(2, P)
+    assert c2 == 32 and bm.table(2)[:2] == bm.table(1)[:2] and bm.table(2)[2] != bm.table(1)[2]
+    assert s2[:32] == s1[:32] and s2[32:] != s1[32:]
+    assert [bm.refcount(b) for b in bm.table(1)[:2]] == [2, 2]
+    _, c3 = bm.add_seq_cached(3, P[:16] + list(range(7, 30)))
+    assert c3 == 16 and bm.table(3)[0] == bm.table(1)[0] and bm.table(3)[1] != bm.table(1)[1]
+    _, c4 = bm.add_seq_cached(4, [5] + P[1:])        # first block differs: no hit at all
+    assert c4 == 0
+    _, c5 = bm.add_seq_cached(5, P[:15])             # no full block
+    assert c5 == 0 and bm.num_cached() == 2 + 1 + 2
+
+
+def pin_prefix_cache_eviction_is_exact():
+    """Freed cached blocks stay reusable; when evicted (oldest first) their cached
+    descendants go too, so a reused block id never matches a stale key."""
+    bm = BMmod.BlockManager(6, 16)
+    A = list(range(32))                              # 2 full blocks
+    bm.add_seq_cached(1, A)
+    a0, a1 = bm.table(1)
+    bm.free_seq(1)
+    assert bm.num_free() == 6 and bm.evictable_list() == [a1, a0]
+    _, c = bm.add_seq_cached(2, A)                   # revived from the evictable list
+    assert c == 32 and bm.table(2) == [a0, a1]
+    bm.free_seq(2)
+    bm.add_seq(3, 16 * 4)                            # takes the 4 free blocks
+    bm.add_seq(4, 16)                                # evicts the oldest released: a1
+    assert bm.table(4) == [a1] and bm.num_cached() == 1
+    bm.free_seq(3)
+    bm.free_seq(4)
+    # a0 is evicted next and then reused for different tokens B; the old child key
+    # (a0, A[16:]) must not match B followed by A[16:]
+    bm.add_seq(5, 16 * 5)                            # every free block: evicts a0 last
+    bm.free_seq(5)
+    B = list(range(500, 516)) + A[16:]
+    _, c = bm.add_seq_cached(6, B)
+    assert c == 0
+    bm2 = BMmod.BlockManager(3, 16)
+    bm2.add_seq_cached(1, A)                         # a0 -> a1 cached
+    p0, p1 = bm2.table(1)
+    bm2.free_seq(1)                                  # evictable: [p1, p0]
+    bm2.add_seq(2, 16)                               # free block
+    bm2.add_seq(3, 16)                               # evicts p1 (a leaf)
+    bm2.free_seq(2)
+    bm2.free_seq(3)
+    bm2.add_seq(4, 48)                               # needs p0 too: evicted with descendants
+    bm2.free_seq(4)
+    _, c = bm2.add_seq_cached(5, list(range(900, 916)) + A[16:])
+    assert c == 0 and bm2.num_cached() == 2          # only the new request's own blocks
+
+
+def pin_prefix_cache_decode():
+    """A request reading a cached prefix equals attention over its own tokens."""
+    rng = np.random.default_rng(8)
+    nb, hkv, d = 16, 2, 8
+    kc = np.zeros((nb, hkv, 16, d), np.uint16)
+    vc = np.zeros_like(kc)
+    bm = BMmod.BlockManager(nb, 16, rng.permutation(nb))
+    prompt = list(range(40))
+    kv = gen.f32_to_bits(rng.standard_normal((2, 60, hkv, d)).astype(np.float32), "f16")
+    slots, c = bm.add_seq_cached(1, prompt)
+    C.reshape_and_cache(kc, vc, kv[0, :40], kv[1, :40], slots, 16)
+    tail = list(range(40)) + [77] * 12                 # same 40 tokens, then 12 of its own
+    slots2, c2 = bm.add_seq_cached(2, tail)
+    assert c2 == 32
+    own_k = np.concatenate([kv[0, :32], kv[0, 40:60]])   # token 32.. are the request's own
+    own_v = np.concatenate([kv[1, :32], kv[1, 40:60]])
+    C.reshape_and_cache(kc, vc, own_k[32:], own_v[32:], slots2[32:], 16)
+    q = gen.f32_to_bits(rng.standard_normal((1, hkv, d)).astype(np.float32), "f16")
+    out = A.paged_decode(q, kc, vc, bm.block_tables([2], 4), [52], 0.4, "f16")
+    for h in range(hkv):
+        ref = A.softmax_attention(bits_to_f64(q[0, h], "f16"), bits_to_f64(own_k[:, h], "f16"),
+                                  bits_to_f64(own_v[:, h], "f16"), 0.4)
+        np.testing.assert_allclose(out[0, h], ref, rtol=1e-14, atol=0)
+
+
 # --------------------------------------------------------------------------
 # cache writes and block copies
 # --------------------------------------------------------------------------
@@ -583,7 +663,13 @@ def _swap_in_reversed(self, seq_id):
 _ORIG_SWAP_IN = BMmod.BlockManager.swap_in
 
 
+def _no_cache_hits(self, seq_id, token_ids):
+    slots = self.add_seq(seq_id, len(list(token_ids)))
+    return slots, 0
+
+
 MISTAKES = {
+    "prefix_cache_never_hits": (BMmod.BlockManager, "add_seq_cached", _no_cache_hits),
     "swap_in_reversed": (BMmod.BlockManager, "swap_in", _swap_in_reversed),
     "dropped_scale": (A, "softmax_attention", _softmax_no_scale),
     "k_v_swapped": (A, "softmax_attention", _softmax_kv_swapped),
