@@ -27,6 +27,27 @@ FIXTURES = {
         "block_size": 16, "tokens": 70, "blocks": 5, "full_blocks": 4, "last_block_used": 6,
         "max_waste_per_request": 15,
     },
+    "iteration_level_example.json": {
+        "source": "PagedAttention: The vLLM Paper (ai.zenoagi.com), section 'Continuous "
+                  "Batching: Request-Level vs. Iteration-Level Scheduling', side-by-side figure; "
+                  "also PagedAttention and Continuous Batching (roadtointelligence.com), section "
+                  "'Batch by step, not by request'",
+        "statement": "with A, B and C in the batch, A finishing lets the waiting D join at the "
+                     "next iteration, giving the batch B, C, D; under request-level scheduling D "
+                     "would wait until the whole batch is done",
+        "reading": "batch of at most 3 sequences; A generates 2 tokens, B and C 4 each, D "
+                   "arrives at step 1 and generates 2; one token per request per step",
+        "max_num_seqs": 3,
+        "requests": [
+            {"name": "A", "arrival": 0, "output_len": 2},
+            {"name": "B", "arrival": 0, "output_len": 4},
+            {"name": "C", "arrival": 0, "output_len": 4},
+            {"name": "D", "arrival": 1, "output_len": 2},
+        ],
+        "iteration_level_batches": [["A", "B", "C"], ["A", "B", "C"], ["B", "C", "D"],
+                                    ["B", "C", "D"]],
+        "request_level_first_step_of_D": 4,
+    },
     "block_table_figure.json": {
         "source": "PagedAttention: The vLLM Paper (ai.zenoagi.com), section 'The Core Idea', GPU "
                   "block pool and block-table figure",
