@@ -35,6 +35,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import subprocess
 import sys
@@ -458,6 +459,97 @@ def measure_prefix_cache(wl, device, requests: int = 64, prompts: int = 4,
                     f"one pa_reshape_and_cache launch stores all new tokens"}
 
 
+def continuous_batching_trace(num_requests: int = 1000, seed: int = 352, rate: float = 1.0):
+    """Seeded request trace for the continuous-batching loop: Poisson arrivals
+    (``rate`` requests per step; at 1.0 the 8192-block pool binds and requests
+    are preempted), lognormal prompt (median 400, clipped to 8..1536)
+    and output (median 200, clipped to 4..512) lengths, and 1, 2 or 4 parallel
+    samples with probabilities 0.85, 0.10, 0.05."""
+    rng = np.random.default_rng(seed)
+    arrival = np.floor(np.cumsum(rng.exponential(1 / rate, num_requests))).astype(np.int64)
+    prompt = np.clip(np.rint(rng.lognormal(np.log(400), 0.8, num_requests)), 8, 1536)
+    output = np.clip(np.rint(rng.lognormal(np.log(200), 0.8, num_requests)), 4, 512)
+    samples = rng.choice([1, 2, 4], num_requests, p=[0.85, 0.10, 0.05])
+    return [(i, int(prompt[i]), int(output[i]), int(samples[i]), int(arrival[i]))
+            for i in range(num_requests)]
+
+
+def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks: int = 8192,
+                                max_num_seqs: int = 256, host_blocks: int = 4096,
+                                max_model_len: int = 2048):
+    """The iteration-level batching loop end to end on one GPU: the library's
+    scheduler plans each step and its executor runs swap-out/in, prefill writes,
+    copy-on-write, new-token writes and decode (7B-like heads of ``wl``). Keys,
+    values and queries are rows of a random device bank (no model). Reports
+    generated tokens per second over the whole trace (CUDA events around the
+    loop; host planning included), and KV occupancy sampled every 16 steps next
+    to what a contiguous ``max_model_len`` reservation per sequence would give."""
+    import torch
+    from paged_kv_cache_352_b200 import _lib as L
+    trace = continuous_batching_trace(num_requests)
+    dt = torch.float16 if wl.dtype == "f16" else torch.bfloat16
+    hq, hkv, d = wl.num_q_heads, wl.num_kv_heads, wl.head_dim
+    sched = L.Scheduler(num_blocks, 16, np.random.default_rng(7).permutation(num_blocks),
+                        max_num_seqs=max_num_seqs, num_host_blocks=host_blocks)
+    for t in trace:
+        sched.submit(*t)
+    sched.attach(hq, hkv, d, dt, max_model_len)
+    kc = torch.zeros(num_blocks, hkv, 16, d, dtype=dt, device=device)
+    vc = torch.zeros_like(kc)
+    hk = torch.zeros(host_blocks, hkv, 16, d, dtype=dt).pin_memory()
+    hv = torch.zeros_like(hk).pin_memory()
+    bank = torch.randn(num_blocks * 16, hkv, d, device=device).to(dt)
+    qbank = torch.randn(max_num_seqs, hq, d, device=device).to(dt)
+    out = torch.empty(max_num_seqs, hq, d, dtype=dt, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    scale = 1.0 / math.sqrt(d)
+    tot = {"steps": 0, "tokens": 0, "prefill_tokens": 0, "preempt": 0, "swap_blocks": 0,
+           "cow": 0, "kv_bytes": 0}
+    util, contiguous = [], []
+    row_bytes = hkv * d * 2
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record()
+    while not sched.idle():
+        c = sched.step()
+        sched.execute(kc, vc, hk, hv, bank, bank, bank, bank, qbank, out, scale, dev_error=err)
+        tot["steps"] += 1
+        tot["tokens"] += c.num_seqs
+        tot["prefill_tokens"] += c.num_prefill
+        tot["preempt"] += c.num_preempted
+        tot["swap_blocks"] += c.num_swap_out + c.num_swap_in
+        tot["cow"] += c.num_copies
+        if tot["steps"] % 16 == 0 and c.num_seqs:
+            filled, alloc = sched.kv_usage()
+            util.append(filled / alloc)
+            contiguous.append(filled / (c.num_seqs * max_model_len))
+    b.record()
+    torch.cuda.synchronize(device)
+    host_s = time.perf_counter() - t0
+    ms = a.elapsed_time(b)
+    if int(err.item()):
+        raise RuntimeError(f"continuous batching: device error bits {int(err.item())}")
+    return {
+        "metric": "generated_tokens_per_s", "value": round(tot["tokens"] / (ms / 1e3), 1),
+        "unit": "tokens/s", "requests": num_requests, "steps": tot["steps"],
+        "ms_per_step": round(ms / tot["steps"], 4),
+        "host_ms_per_step": round(1e3 * host_s / tot["steps"], 4),
+        "mean_batch": round(tot["tokens"] / tot["steps"], 1),
+        "generated_tokens": tot["tokens"], "prefill_tokens": tot["prefill_tokens"],
+        "preemptions": tot["preempt"], "swapped_blocks": tot["swap_blocks"],
+        "cow_copies": tot["cow"],
+        "kv_utilization": round(float(np.mean(util)), 4) if util else None,
+        "contiguous_reservation_utilization": (round(float(np.mean(contiguous)), 4)
+                                               if contiguous else None),
+        "what": f"{num_requests} requests (Poisson 1.0/step, lognormal prompts/outputs, "
+                f"1/2/4 samples), pool {num_blocks} blocks, batch cap {max_num_seqs}, "
+                f"host pool {host_blocks} blocks; utilization vs a {max_model_len}-token "
+                f"contiguous reservation per sequence",
+    }
+
+
 def run_reference(args):
     rank, world, _ = _rank_info()
     if rank != 0:
@@ -584,6 +676,7 @@ def run_ours(args):
 
     swap = measure_swap(wl, r, device) if world == 1 else None
     prefix_cache = measure_prefix_cache(wl, device) if world == 1 else None
+    batching = measure_continuous_batching(wl, device) if world == 1 else None
 
     sb = step_bytes(wl, r)
     db = decode_bytes(wl)
@@ -632,6 +725,7 @@ def run_ours(args):
         "gpu_launches": K * launches_per_step,
         "swap": swap,
         "prefix_cache": prefix_cache,
+        "continuous_batching": batching,
         "clocks": csum,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -346,6 +346,151 @@ int pa_bm_num_seqs(const pa_bm* bm);
 /* Free blocks in hand-out order into out[capacity]; returns the count written or -1. */
 int pa_bm_free_list(const pa_bm* bm, int32_t* out, int capacity);
 
+/* ---------------------------------------------------------------------------
+ * Continuous (iteration-level) batching: a scheduler over the block manager and
+ * an executor that runs one planned step through the kernels above.
+ *
+ * Requests join and leave the batch at every decoding step instead of waiting
+ * for a whole batch to finish ("PagedAttention and Continuous Batching", "Batch
+ * by step, not by request"; "PagedAttention: The vLLM Paper", "Continuous
+ * Batching: Request-Level vs. Iteration-Level Scheduling"); when the pool runs
+ * short a request is preempted by swapping its blocks to host memory or by
+ * dropping them for recomputation ("Implementation Essentials", block manager);
+ * parallel samples of one prompt share its blocks (same section, prefix sharing).
+ *
+ * A request is (request_id >= 0, prompt_len >= 1, output_len >= 1,
+ * 1 <= num_samples <= PA_SCHED_MAX_SAMPLES, arrival_step). There is no model:
+ * every sample generates exactly output_len tokens, one per step, and the keys,
+ * values and queries of the tokens are the caller's inputs. Sample s of request
+ * r is block-manager sequence r * PA_SCHED_MAX_SAMPLES + s.
+ *
+ * pa_sched_step plans one step, in this order (rules the pages leave open):
+ *   1. requests that finished in the previous step are freed;
+ *   2. running requests, oldest admission first, append one token per sample.
+ *      Before a request appends, the blocks its appends take (one per sample
+ *      whose last block is full, one per copy-on-write of a shared partly
+ *      filled block) are checked against the free count; while short, the
+ *      newest running request is preempted (the request itself if it is the
+ *      newest). Preemption swaps every sample out when the host pool has room
+ *      for a copy of each sample's table, else drops a one-sample request for
+ *      recomputation (it rejoins the waiting queue in arrival order, and on
+ *      readmission its prompt and generated tokens are written again); a
+ *      many-sample request that cannot be swapped makes the step fail;
+ *   3. if nothing was preempted in this step: swapped requests resume in
+ *      arrival order while the batch (max_num_seqs sequences) and the pool
+ *      have room for them and their appends;
+ *   4. if nothing was preempted and nothing is swapped out: waiting requests
+ *      whose arrival_step has come are admitted in arrival order (arrival_step,
+ *      then submission order), stopping at the first that does not fit. The
+ *      prompt is registered for sample 0, samples 1.. fork it.
+ *   Resumed and admitted requests append in the same step. The decode batch is
+ *   every running sample, in running order then sample order, each with its
+ *   new token in its context. A request whose samples have generated
+ *   output_len tokens finishes with this step.
+ *
+ * Device order of a step (pa_sched_execute): swap-out pairs (device -> host),
+ * swap-in pairs (host -> device), prefill writes (prompts and recomputed
+ * tokens of admitted requests), copy-on-write pairs, new-token writes, decode.
+ * ------------------------------------------------------------------------- */
+#define PA_SCHED_MAX_SAMPLES 64
+#define PA_PREEMPT_SWAP 0
+#define PA_PREEMPT_RECOMPUTE 1
+
+typedef struct pa_sched pa_sched;
+
+/* Counts of the last planned step. */
+typedef struct {
+  int64_t step;            /* 0 for the first step */
+  int num_finished;        /* requests freed at the start of the step */
+  int num_preempted;
+  int num_resumed;
+  int num_admitted;
+  int num_swap_out;        /* (device block, host block) pairs */
+  int num_swap_in;         /* (host block, device block) pairs */
+  int num_copies;          /* copy-on-write (src, dst) pairs */
+  int num_prefill;         /* tokens written before the copies */
+  int num_writes;          /* new tokens written after the copies */
+  int num_seqs;            /* decode batch */
+  int max_blocks_per_seq;  /* widest block table in the batch (>= 1) */
+  int max_context_len;
+} pa_sched_plan;
+
+/* num_blocks / block_size / initial_free_order as pa_bm_create. max_num_seqs
+ * caps the decode batch (sequences). num_host_blocks sizes the host pool used
+ * by swap preemption (0: none). preempt_mode PA_PREEMPT_RECOMPUTE takes no host
+ * pool and only one-sample requests. */
+int pa_sched_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                    int max_num_seqs, int num_host_blocks, int preempt_mode, pa_sched** out);
+void pa_sched_destroy(pa_sched* s);
+
+/* PA_ERR_INVALID_ARG for bad sizes, a duplicate or negative id, or several
+ * samples in recompute mode; PA_ERR_NO_FREE_BLOCKS when the request could never
+ * fit (num_samples > max_num_seqs, or num_samples * ceil((prompt_len +
+ * output_len) / block_size) > num_blocks). */
+int pa_sched_submit(pa_sched* s, int64_t request_id, int prompt_len, int output_len,
+                    int num_samples, int64_t arrival_step);
+
+/* Plans the next step and writes its counts to *plan. PA_ERR_NO_FREE_BLOCKS if
+ * a many-sample request could not be preempted (host pool full); the scheduler
+ * is then failed and every later step returns that error. */
+int pa_sched_step(pa_sched* s, pa_sched_plan* plan);
+
+/* 1 when nothing is pending, waiting, running, swapped or left to free. */
+int pa_sched_idle(const pa_sched* s);
+
+/* Detail of the last planned step. Every output pointer may be NULL; arrays
+ * are sized by the counts in pa_sched_plan.
+ *   requests: finished[num_finished], preempted[num_preempted] with
+ *     preempt_modes[num_preempted] (PA_PREEMPT_*), resumed[num_resumed],
+ *     admitted[num_admitted] (request ids, in planning order);
+ *   pairs: swap_out[num_swap_out][2], swap_in[num_swap_in][2],
+ *     copies[num_copies][2];
+ *   writes (which = 0: prefill, 1: new tokens): per token its request, sample,
+ *     position in the sample's sequence and slot;
+ *   batch: per decoded sequence its request, sample and context length, and
+ *     block_tables[num_seqs][max_blocks_per_seq] padded with -1. */
+int pa_sched_plan_requests(const pa_sched* s, int64_t* finished, int64_t* preempted,
+                           int32_t* preempt_modes, int64_t* resumed, int64_t* admitted);
+int pa_sched_plan_pairs(const pa_sched* s, int64_t* swap_out, int64_t* swap_in,
+                        int64_t* copies);
+int pa_sched_plan_writes(const pa_sched* s, int which, int64_t* request, int32_t* sample,
+                         int32_t* position, int64_t* slot);
+int pa_sched_plan_batch(const pa_sched* s, int64_t* request, int32_t* sample,
+                        int32_t* context_lens, int32_t* block_tables);
+
+/* KV occupancy now: *filled = slots holding tokens and *allocated = block_size x device
+ * blocks held by resident requests (running, and finished in the last step);
+ * a shared block counts once, at the fill of its fullest holder. */
+int pa_sched_kv_usage(const pa_sched* s, int64_t* filled, int64_t* allocated);
+
+/* The scheduler's block manager (owned by the scheduler; read-only use). */
+const pa_bm* pa_sched_block_manager(const pa_sched* s);
+
+/* Executor. pa_sched_attach allocates, once, the executor's device metadata
+ * buffers, a ring of pinned host staging buffers and the decode workspace, for
+ * the given head shape and a largest context of max_context_len tokens (on the
+ * current device). Planning works without it. */
+int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim, int dtype,
+                    int max_context_len);
+
+/* Runs the last planned step on `stream` in device order: pa_swap_blocks for
+ * the swap pairs (device pool k_cache/v_cache <-> pinned host pool
+ * host_k/host_v, [num_host_blocks][Hkv][16][d]; may be NULL when the plan has
+ * no swap pair), pa_reshape_and_cache of prefill_key/prefill_value
+ * ([num_prefill][Hkv][d], contiguous, device), pa_copy_blocks, pa_reshape_and_cache
+ * of key/value ([num_writes][Hkv][d]), then pa_paged_decode of q
+ * ([num_seqs][Hq][d]) into out ([num_seqs][Hq][d]) through the plan's tables,
+ * longest context first. Row i of each input belongs to write / sequence i of
+ * the plan. Block tables, context lengths, slots and the order reach the device
+ * through the pinned ring with one host-to-device copy per step; the call
+ * waits only for the copy that last used the ring slot. Never synchronises the
+ * stream otherwise. dev_error as pa_paged_decode. A step may be executed at
+ * most once, and before the next pa_sched_step. */
+int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, void* host_v,
+                     const void* prefill_key, const void* prefill_value, const void* key,
+                     const void* value, const void* q, void* out, float scale, int* dev_error,
+                     void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,6 +16,9 @@ from ._lib import (  # noqa: F401
     PA_DEVERR_SLOT_RANGE,
     PA_DEVERR_WAIT_TIMEOUT,
     PA_F16,
+    PA_PREEMPT_RECOMPUTE,
+    PA_PREEMPT_SWAP,
+    Scheduler,
     decode_workspace,
     last_error,
     lib,

@@ -85,6 +85,20 @@ _SIGS = {
     "pa_bm_add_seq_cached": (_c_int, [_vp, _c_i64, _vp, _c_int, _vp, ctypes.POINTER(_c_int)]),
     "pa_bm_num_cached": (_c_int, [_vp]),
     "pa_bm_evictable_list": (_c_int, [_vp, _vp, _c_int]),
+    "pa_sched_create": (_c_int, [_c_int, _c_int, _vp, _c_int, _c_int, _c_int, ctypes.POINTER(_vp)]),
+    "pa_sched_destroy": (None, [_vp]),
+    "pa_sched_submit": (_c_int, [_vp, _c_i64, _c_int, _c_int, _c_int, _c_i64]),
+    "pa_sched_step": (_c_int, [_vp, _vp]),
+    "pa_sched_idle": (_c_int, [_vp]),
+    "pa_sched_plan_requests": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "pa_sched_plan_pairs": (_c_int, [_vp, _vp, _vp, _vp]),
+    "pa_sched_plan_writes": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp]),
+    "pa_sched_plan_batch": (_c_int, [_vp, _vp, _vp, _vp, _vp]),
+    "pa_sched_kv_usage": (_c_int, [_vp, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64)]),
+    "pa_sched_block_manager": (_vp, [_vp]),
+    "pa_sched_attach": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "pa_sched_execute": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  ctypes.c_float, _vp, _vp]),
 }
 
 _LIB = None
@@ -327,6 +341,17 @@ def _i64p(a):
 class BlockManager:
     """Owner of one ``pa_bm`` handle (the pa_bm_* calls as methods)."""
 
+    @classmethod
+    def _borrow(cls, handle, num_blocks: int, block_size: int):
+        """A view of a manager owned elsewhere (never destroyed by this object)."""
+        self = cls.__new__(cls)
+        self._lib = lib()
+        self._h = ctypes.c_void_p(handle)
+        self._owned = False
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        return self
+
     def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE, initial_free_order=None):
         self._lib = lib()
         order = None
@@ -339,11 +364,12 @@ class BlockManager:
                                       order.ctypes.data if order is not None else None,
                                       ctypes.byref(h)))
         self._h = h
+        self._owned = True
         self.num_blocks = num_blocks
         self.block_size = block_size
 
     def close(self):
-        if getattr(self, "_h", None):
+        if getattr(self, "_owned", False) and self._h:
             self._lib.pa_bm_destroy(self._h)
             self._h = None
 
@@ -460,3 +486,147 @@ class BlockManager:
         out = np.empty(n, np.int32)
         m = self._lib.pa_bm_host_free_list(self._h, out.ctypes.data, n)
         return out[:m].tolist()
+
+
+# --------------------------------------------------------------------------
+# continuous batching
+# --------------------------------------------------------------------------
+
+PA_SCHED_MAX_SAMPLES = 64
+PA_PREEMPT_SWAP = 0
+PA_PREEMPT_RECOMPUTE = 1
+
+
+class SchedPlanCounts(ctypes.Structure):
+    _fields_ = [("step", ctypes.c_int64), ("num_finished", ctypes.c_int),
+                ("num_preempted", ctypes.c_int), ("num_resumed", ctypes.c_int),
+                ("num_admitted", ctypes.c_int), ("num_swap_out", ctypes.c_int),
+                ("num_swap_in", ctypes.c_int), ("num_copies", ctypes.c_int),
+                ("num_prefill", ctypes.c_int), ("num_writes", ctypes.c_int),
+                ("num_seqs", ctypes.c_int), ("max_blocks_per_seq", ctypes.c_int),
+                ("max_context_len", ctypes.c_int)]
+
+
+def _p(a):
+    return a.ctypes.data if a is not None and a.size else None
+
+
+class Scheduler:
+    """Owner of one ``pa_sched`` handle: iteration-level batching over a block
+    manager (pa_sched_* calls as methods) and the executor of planned steps."""
+
+    def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE, initial_free_order=None,
+                 max_num_seqs: int = 256, num_host_blocks: int = 0,
+                 preempt_mode: int = PA_PREEMPT_SWAP):
+        self._lib = lib()
+        order = None
+        if initial_free_order is not None:
+            order = np.ascontiguousarray(np.asarray(initial_free_order, dtype=np.int32))
+            if order.shape != (num_blocks,):
+                raise PAError(PA_ERR_INVALID_ARG, "initial_free_order must have num_blocks ids")
+        h = ctypes.c_void_p()
+        _check(self._lib.pa_sched_create(num_blocks, block_size,
+                                         order.ctypes.data if order is not None else None,
+                                         max_num_seqs, num_host_blocks, preempt_mode,
+                                         ctypes.byref(h)))
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.max_num_seqs = max_num_seqs
+        self.num_host_blocks = num_host_blocks
+        self.bm = BlockManager._borrow(self._lib.pa_sched_block_manager(h), num_blocks,
+                                       block_size)
+        self.counts = None
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pa_sched_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def submit(self, request_id: int, prompt_len: int, output_len: int, num_samples: int = 1,
+               arrival: int = 0) -> None:
+        _check(self._lib.pa_sched_submit(self._h, request_id, prompt_len, output_len,
+                                         num_samples, arrival))
+
+    def step(self) -> SchedPlanCounts:
+        c = SchedPlanCounts()
+        _check(self._lib.pa_sched_step(self._h, ctypes.byref(c)))
+        self.counts = c
+        return c
+
+    def idle(self) -> bool:
+        return bool(self._lib.pa_sched_idle(self._h))
+
+    def kv_usage(self):
+        f, a = ctypes.c_int64(0), ctypes.c_int64(0)
+        _check(self._lib.pa_sched_kv_usage(self._h, ctypes.byref(f), ctypes.byref(a)))
+        return f.value, a.value
+
+    def plan(self) -> dict:
+        """The last planned step in full, as plain lists (the oracle's Plan fields)."""
+        c = self.counts
+        fin = np.empty(c.num_finished, np.int64)
+        pre = np.empty(c.num_preempted, np.int64)
+        mode = np.empty(c.num_preempted, np.int32)
+        res = np.empty(c.num_resumed, np.int64)
+        adm = np.empty(c.num_admitted, np.int64)
+        _check(self._lib.pa_sched_plan_requests(self._h, _p(fin), _p(pre), _p(mode), _p(res),
+                                                _p(adm)))
+        so = np.empty((c.num_swap_out, 2), np.int64)
+        si = np.empty((c.num_swap_in, 2), np.int64)
+        cp = np.empty((c.num_copies, 2), np.int64)
+        _check(self._lib.pa_sched_plan_pairs(self._h, _p(so), _p(si), _p(cp)))
+        writes = {}
+        for which, n in ((0, c.num_prefill), (1, c.num_writes)):
+            r = np.empty(n, np.int64)
+            sm = np.empty(n, np.int32)
+            pos = np.empty(n, np.int32)
+            sl = np.empty(n, np.int64)
+            _check(self._lib.pa_sched_plan_writes(self._h, which, _p(r), _p(sm), _p(pos), _p(sl)))
+            writes[which] = [tuple(int(x) for x in t) for t in zip(r, sm, pos, sl)]
+        br = np.empty(c.num_seqs, np.int64)
+        bsm = np.empty(c.num_seqs, np.int32)
+        ctx = np.empty(c.num_seqs, np.int32)
+        tables = np.empty((c.num_seqs, c.max_blocks_per_seq), np.int32)
+        _check(self._lib.pa_sched_plan_batch(self._h, _p(br), _p(bsm), _p(ctx), _p(tables)))
+        pairs = lambda a: [tuple(int(x) for x in row) for row in a]
+        return {
+            "step": int(c.step),
+            "finished": fin.tolist(),
+            "preempted": list(zip(pre.tolist(), mode.tolist())),
+            "resumed": res.tolist(),
+            "admitted": adm.tolist(),
+            "swap_out": pairs(so), "swap_in": pairs(si), "copies": pairs(cp),
+            "prefill": writes[0], "writes": writes[1],
+            "batch": list(zip(br.tolist(), bsm.tolist(), ctx.tolist())),
+            "tables": tables,
+        }
+
+    def attach(self, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype,
+               max_context_len: int) -> None:
+        code = dtype if isinstance(dtype, int) else (
+            PA_F16 if dtype == _torch().float16 else PA_BF16)
+        _check(self._lib.pa_sched_attach(self._h, num_q_heads, num_kv_heads, head_dim, code,
+                                         max_context_len))
+
+    def execute(self, k_cache, v_cache, host_k, host_v, prefill_key, prefill_value, key, value,
+                q, out, scale: float, dev_error=None, stream=None) -> None:
+        """Run the last planned step (pa_sched_execute). Inputs are device tensors
+        whose leading dimension covers the plan's counts; host_k/host_v are the
+        pinned host pool (or None)."""
+        torch = _torch()
+        dt = k_cache.dtype
+        host = lambda t, n: None if t is None else _pool_ptr(t, n)
+        _check(self._lib.pa_sched_execute(
+            self._h, _dev_ptr(k_cache, "k_cache", dt), _dev_ptr(v_cache, "v_cache", dt),
+            host(host_k, "host_k"), host(host_v, "host_v"),
+            _dev_ptr(prefill_key, "prefill_key", dt), _dev_ptr(prefill_value, "prefill_value", dt),
+            _dev_ptr(key, "key", dt), _dev_ptr(value, "value", dt), _dev_ptr(q, "q", dt),
+            _dev_ptr(out, "out", dt), scale, _dev_ptr(dev_error, "dev_error", torch.int32),
+            _stream(stream)))

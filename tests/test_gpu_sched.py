@@ -1,0 +1,109 @@
+"""Continuous batching on a B200: the library's scheduler plans every step, the
+executor runs it through the swap, cache-write, copy-on-write and decode
+kernels, and each step's outputs are compared with the oracle's attention over
+every decoded sample's logical keys and values (prompt + its own tokens), with
+the plans checked bit for bit against the oracle scheduler."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_352_b200 as pa
+from oracle import scheduler as SCH
+from oracle.attention import softmax_attention
+from oracle.fpbits import bits_to_f64
+from tests.parity import assert_close, out_to_f64
+from workloads import gen
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed):
+    tdt = torch.float16 if dt == "f16" else torch.bfloat16
+    order = np.random.default_rng(seed).permutation(nb)
+    c = pa.Scheduler(nb, 16, order, max_num_seqs=cap, num_host_blocks=host, preempt_mode=mode)
+    o = SCH.Scheduler(nb, 16, order, max_num_seqs=cap, num_host_blocks=host, preempt_mode=mode)
+    for t in trace:
+        c.submit(*t)
+        o.submit(*t)
+    max_ctx = max(p + n for _, p, n, _, _ in trace)
+    c.attach(hq, hkv, d, tdt, max_ctx)
+    kc = torch.zeros(nb, hkv, 16, d, dtype=tdt, device="cuda")
+    vc = torch.zeros_like(kc)
+    hk = torch.zeros(max(host, 1), hkv, 16, d, dtype=tdt).pin_memory() if host else None
+    hv = torch.zeros_like(hk).pin_memory() if host else None
+    toks = gen.RequestTokens(seed, {r: p for r, p, *_ in trace}, hkv, d, dt)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scale = 1 / math.sqrt(d)
+    G = hq // hkv
+    stats = {"steps": 0, "preempt": 0, "swap": 0, "cow": 0, "seqs": 0}
+    while not o.idle():
+        c.step()
+        op = o.step()
+        cp = c.plan()
+        for f in ("preempted", "swap_out", "swap_in", "copies", "prefill", "writes", "batch"):
+            assert [tuple(x) for x in cp[f]] == [tuple(x) for x in getattr(op, f)], (op.step, f)
+
+        def rows(ws):
+            k = np.zeros((len(ws), hkv, d), np.uint16)
+            v = np.zeros_like(k)
+            for i, (r, s, p, _) in enumerate(ws):
+                k[i], v[i] = toks.row(r, s, p)
+            return (torch.from_numpy(k.view(np.int16)).view(tdt).cuda(),
+                    torch.from_numpy(v.view(np.int16)).view(tdt).cuda())
+
+        pk, pv = rows(op.prefill)
+        wk, wv = rows(op.writes)
+        q_bits = np.stack([gen.step_query_bits(seed, r, s, op.step, hq, d, dt)
+                           for r, s, _ in op.batch]) if op.batch else np.zeros((0, hq, d), np.uint16)
+        q = torch.from_numpy(q_bits.view(np.int16)).view(tdt).cuda()
+        out = torch.empty(len(op.batch), hq, d, dtype=tdt, device="cuda")
+        c.execute(kc, vc, hk, hv, pk, pv, wk, wv, q, out, scale, dev_error=err)
+        torch.cuda.synchronize()
+        got = out_to_f64(out, dt)
+        for i, (r, s, ctx) in enumerate(op.batch):
+            K, V = toks.rows(r, s, range(ctx))
+            ref = np.stack([softmax_attention(bits_to_f64(q_bits[i, h], dt),
+                                              bits_to_f64(K[:, h // G], dt),
+                                              bits_to_f64(V[:, h // G], dt), scale)
+                            for h in range(hq)])
+            assert_close(got[i], ref, f"step {op.step} request {r} sample {s}")
+        stats["steps"] += 1
+        stats["preempt"] += len(op.preempted)
+        stats["swap"] += len(op.swap_out) + len(op.swap_in)
+        stats["cow"] += len(op.copies)
+        stats["seqs"] += len(op.batch)
+    assert int(err.item()) == 0
+    return stats
+
+
+def _trace(seed, n, max_samples, prompt=(1, 70), out=(1, 40), arrive=25):
+    rng = np.random.default_rng(seed)
+    return [(i, int(rng.integers(*prompt)), int(rng.integers(*out)),
+             int(rng.integers(1, max_samples + 1)), int(rng.integers(0, arrive)))
+            for i in range(n)]
+
+
+def test_swap_mode_trace_gqa_bf16():
+    st = _run_trace(_trace(11, 24, 3), nb=26, cap=12, host=400, mode=pa.PA_PREEMPT_SWAP,
+                    hq=8, hkv=2, d=128, dt="bf16", seed=41)
+    assert st["preempt"] > 0 and st["swap"] > 0 and st["cow"] > 0, st
+
+
+def test_recompute_mode_trace_mha_f16():
+    st = _run_trace(_trace(12, 24, 1), nb=24, cap=10, host=0, mode=pa.PA_PREEMPT_RECOMPUTE,
+                    hq=4, hkv=4, d=64, dt="f16", seed=42)
+    assert st["preempt"] > 0, st
+
+
+def test_long_prompts_split_kv():
+    """Contexts of 600 to 2500 tokens, long enough for the decode's default split
+    into partitions, through the loop."""
+    rng = np.random.default_rng(13)
+    trace = [(i, int(rng.integers(600, 2500)), int(rng.integers(1, 30)), 1,
+              int(rng.integers(0, 6))) for i in range(8)]
+    st = _run_trace(trace, nb=600, cap=8, host=0, mode=pa.PA_PREEMPT_SWAP,
+                    hq=16, hkv=2, d=128, dt="bf16", seed=43)
+    assert st["steps"] > 0

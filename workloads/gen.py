@@ -23,6 +23,8 @@ STREAM_SEQ_KV = 1      # per-sequence key/value rows (prompt + generated tokens)
 STREAM_QUERY = 2       # the decode step's queries
 STREAM_OWN_KV = 3      # per-sample tokens appended after a fork (shared-prefix workload)
 STREAM_META = 4        # context lengths and block placement
+STREAM_REQUEST_KV = 5  # request traces: one key/value row per (request, branch, position)
+STREAM_STEP_QUERY = 6  # request traces: one query per (request, sample, step)
 
 _DTYPES = ("f16", "bf16")
 
@@ -97,3 +99,45 @@ def own_token_kv_bits(seed: int, sample: int, ntok: int, num_kv_heads: int, head
     k = f32_to_bits(rng.standard_normal(shape, dtype=np.float32), dtype)
     v = f32_to_bits(rng.standard_normal(shape, dtype=np.float32), dtype)
     return k, v
+
+
+def request_token_kv_bits(seed: int, request: int, branch: int, position: int,
+                          num_kv_heads: int, head_dim: int, dtype: str):
+    """Key and value rows ``[num_kv_heads, head_dim]`` of one token of a request
+    trace. ``branch`` 0 holds the prompt (shared by every sample); branch
+    ``1 + s`` holds the tokens sample ``s`` generates."""
+    b = normal_bits([seed, STREAM_REQUEST_KV, request, branch, position],
+                    (2, num_kv_heads, head_dim), dtype)
+    return b[0], b[1]
+
+
+def step_query_bits(seed: int, request: int, sample: int, step: int, num_q_heads: int,
+                    head_dim: int, dtype: str) -> np.ndarray:
+    """The query ``[num_q_heads, head_dim]`` of one sample at one step of a trace."""
+    return normal_bits([seed, STREAM_STEP_QUERY, request, sample, step],
+                       (num_q_heads, head_dim), dtype)
+
+
+class RequestTokens:
+    """Memoised token rows of a request trace: position ``p`` of sample ``s`` of
+    request ``r`` is a prompt row when ``p < prompt_len[r]``, else sample ``s``'s own."""
+
+    def __init__(self, seed: int, prompt_len: dict, num_kv_heads: int, head_dim: int,
+                 dtype: str):
+        self.seed, self.prompt_len = seed, prompt_len
+        self.hkv, self.d, self.dtype = num_kv_heads, head_dim, dtype
+        self._rows = {}
+
+    def row(self, request: int, sample: int, position: int):
+        branch = 0 if position < self.prompt_len[request] else 1 + sample
+        key = (request, branch, position)
+        if key not in self._rows:
+            self._rows[key] = request_token_kv_bits(self.seed, request, branch, position,
+                                                    self.hkv, self.d, self.dtype)
+        return self._rows[key]
+
+    def rows(self, request: int, sample: int, positions):
+        ks, vs = zip(*(self.row(request, sample, p) for p in positions)) if len(positions) else ((), ())
+        shape = (0, self.hkv, self.d)
+        return (np.stack(ks) if ks else np.zeros(shape, np.uint16),
+                np.stack(vs) if vs else np.zeros(shape, np.uint16))
