@@ -58,7 +58,11 @@ typedef enum pa_status {
   PA_ERR_SEQ_SWAPPED = 7     /* sequence is swapped out (or, for swap-in, is not) */
 } pa_status;
 
-typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+/* PA_FP8_E4M3 is a cache element type only: pa_reshape_and_cache_fp8 writes it,
+ * pa_paged_decode_fp8 reads it, pa_copy_blocks and pa_swap_blocks move it (one
+ * byte per element). Queries, outputs and the 16-bit inputs of the cache write
+ * are PA_F16 or PA_BF16. */
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 /* Bits OR-ed into *dev_error by device calls. */
 #define PA_DEVERR_SLOT_RANGE 1    /* slot >= num_blocks * block_size: token not written */
@@ -112,7 +116,7 @@ int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_s
  *           src of the same call (so the copies are independent). Violations
  *           return PA_ERR_INVALID_ARG and launch nothing.
  * The pairs travel in the kernel's parameter block: no device buffer is needed.
- * num_pairs == 0 is a no-op.
+ * num_pairs == 0 is a no-op. dtype PA_FP8_E4M3 copies 8-bit caches.
  * ------------------------------------------------------------------------- */
 int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
@@ -143,6 +147,42 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
 int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, void* dst_k,
                    void* dst_v, int dst_num_blocks, const int64_t* pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 8-bit KV cache: pa_reshape_and_cache_fp8 and pa_paged_decode_fp8.
+ *
+ * Quantizing the KV cache shrinks the bytes a bandwidth-bound decode reads
+ * ("PagedAttention: The vLLM Paper", "Impact and Follow-Ups" and "Limitations");
+ * the pages fix no format. Format taken: OCP FP8 E4M3 (bias 7, no infinities,
+ * largest finite 448, codes 0x7F / 0xFF NaN), one scale per cache tensor.
+ * Caches are uint8 arrays in the layout above ([num_blocks][Hkv][16][d], one
+ * byte per element); copy and swap them with dtype PA_FP8_E4M3.
+ *
+ * pa_reshape_and_cache_fp8: as pa_reshape_and_cache, but element x of key
+ * (value) is stored as the E4M3 code nearest to float32(x) / k_scale
+ * (v_scale), the division rounded to nearest in fp32, ties of the conversion
+ * to the even code, magnitudes past 448 saturating to 448, the sign kept.
+ * src_dtype is the type of key/value (PA_F16 or PA_BF16). k_scale and v_scale
+ * must be finite and positive (else PA_ERR_INVALID_ARG).
+ *
+ * pa_paged_decode_fp8: as pa_paged_decode over E4M3 caches, attending to the
+ * dequantized keys code * k_scale and values code * v_scale; q and out are of
+ * type dtype (PA_F16 or PA_BF16). The workspace is sized by
+ * pa_paged_decode_workspace_size exactly as for pa_paged_decode.
+ * ------------------------------------------------------------------------- */
+int pa_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_token_stride,
+                             int64_t value_token_stride, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                             int head_dim, int block_size, int num_blocks, int src_dtype,
+                             float k_scale, float v_scale, int* dev_error, void* stream);
+
+int pa_paged_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, int max_blocks_per_seq,
+                        const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                        int max_context_len, int num_q_heads, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, float scale, float k_scale,
+                        float v_scale, int partition_tokens, void* workspace,
+                        size_t workspace_bytes, int* dev_error, int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
  * pa_paged_decode — decode-step attention through the block tables.

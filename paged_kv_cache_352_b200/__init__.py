@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     PA_DEVERR_SLOT_RANGE,
     PA_DEVERR_WAIT_TIMEOUT,
     PA_F16,
+    PA_FP8_E4M3,
     PA_PREEMPT_RECOMPUTE,
     PA_PREEMPT_SWAP,
     Scheduler,
@@ -25,7 +26,9 @@ from ._lib import (  # noqa: F401
     pa_copy_blocks,
     pa_longest_first_order,
     pa_paged_decode,
+    pa_paged_decode_fp8,
     pa_paged_decode_workspace_size,
     pa_reshape_and_cache,
+    pa_reshape_and_cache_fp8,
     pa_swap_blocks,
 )

@@ -28,6 +28,7 @@ PA_ERR_SEQ_SWAPPED = 7
 
 PA_F16 = 0
 PA_BF16 = 1
+PA_FP8_E4M3 = 2
 
 PA_DEVERR_SLOT_RANGE = 1
 PA_DEVERR_BLOCK_RANGE = 2
@@ -62,6 +63,13 @@ _SIGS = {
                                          _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                          ctypes.c_float, _c_int, _vp, _c_int, _vp]),
     "pa_longest_first_order": (_c_int, [_vp, _c_int, _vp]),
+    "pa_reshape_and_cache_fp8": (_c_int, [_vp, _vp, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int,
+                                          _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
+                                          ctypes.c_float, _vp, _vp]),
+    "pa_paged_decode_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int,
+                                     _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
+                                     ctypes.c_float, ctypes.c_float, _c_int, _vp, ctypes.c_size_t,
+                                     _vp, _c_int, _vp]),
     "pa_bm_create": (_c_int, [_c_int, _c_int, _vp, ctypes.POINTER(_vp)]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_c_int, [_vp, _c_i64, _c_int, _vp]),
@@ -144,6 +152,8 @@ def dtype_code(t) -> int:
         return PA_F16
     if t.dtype == torch.bfloat16:
         return PA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return PA_FP8_E4M3
     raise PAError(PA_ERR_UNSUPPORTED, f"storage type {t.dtype}: expected float16 or bfloat16")
 
 
@@ -290,6 +300,53 @@ def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_co
         _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
         int(partition_tokens), _dev_ptr(workspace, "workspace"), ws_bytes,
         _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             dev_error=None, stream=None):
+    """Quantize ``key``/``value`` ``[T, num_kv_heads, head_dim]`` (float16/bfloat16)
+    into the E4M3 caches (uint8 or float8_e4m3fn tensors) at ``slot_mapping``."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    if dtype_code(k_cache) != PA_FP8_E4M3:
+        raise PAError(PA_ERR_INVALID_ARG, "k_cache/v_cache must be uint8 or float8_e4m3fn")
+    T = key.shape[0]
+    if key.shape[1:] != (hkv, d) or value.shape[1:] != (hkv, d) or value.shape[0] != T:
+        raise PAError(PA_ERR_INVALID_ARG, "key/value must be [T, num_kv_heads, head_dim]")
+    if key.stride(2) != 1 or key.stride(1) != d or value.stride(2) != 1 or value.stride(1) != d:
+        raise PAError(PA_ERR_INVALID_ARG, "key/value rows must be dense per token")
+    if value.dtype != key.dtype or slot_mapping.shape != (T,):
+        raise PAError(PA_ERR_INVALID_ARG, "value must match key; slot_mapping must be [T]")
+    _check(lib().pa_reshape_and_cache_fp8(
+        _dev_ptr(key, "key", contiguous=False), _dev_ptr(value, "value", contiguous=False),
+        key.stride(0), value.stride(0), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, hkv, d, bs, nb, dtype_code(key),
+        float(k_scale), float(v_scale), _dev_ptr(dev_error, "dev_error", torch.int32),
+        _stream(stream)))
+
+
+def pa_paged_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                        scale, k_scale, v_scale, partition_tokens=0, workspace=None,
+                        dev_error=None, stream=None, seq_order=None):
+    """pa_paged_decode over E4M3 caches (uint8 / float8_e4m3fn) with key and value
+    scales; ``q``/``out`` are float16 or bfloat16."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    if dtype_code(k_cache) != PA_FP8_E4M3:
+        raise PAError(PA_ERR_INVALID_ARG, "k_cache/v_cache must be uint8 or float8_e4m3fn")
+    B, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or out.dtype != q.dtype:
+        raise PAError(PA_ERR_INVALID_ARG, "q/out must be [B, num_q_heads, head_dim], one dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pa_paged_decode_fp8(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
+        _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+        float(k_scale), float(v_scale), int(partition_tokens), _dev_ptr(workspace, "workspace"),
+        ws_bytes, _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(q), _stream(stream)))
 
 
 NOALLOC_WORKSPACE_BYTES = 16 << 20

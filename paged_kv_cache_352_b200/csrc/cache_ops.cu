@@ -11,6 +11,10 @@
 // it, as with fork and copy-on-write ("Pages, from operating systems"; "The OS
 // paging analogy", page sharing).
 //
+// reshape_and_cache_fp8: the same write into 8-bit E4M3 caches, quantizing each
+// element by the tensor's scale (KV-cache quantization, "PagedAttention: The
+// vLLM Paper", "Impact and Follow-Ups" and "Limitations").
+//
 // swap_blocks: the same copy between two pools, the device pool and a pinned
 // host pool, to preempt a request by swapping its blocks to CPU memory ("The OS
 // paging analogy", swapping).
@@ -50,6 +54,56 @@ __global__ void __launch_bounds__(256)
   const int64_t dst = ((block * num_kv_heads + h) * kBlockSize + offset) * chunks_per_row + c;
   k_cache[dst] = kv;
   v_cache[dst] = vv;
+}
+
+// E4M3 caches: one thread per 16 codes (16 bytes of the cache row) of a
+// (token, KV head) row; it reads the matching 16 elements of the 16-bit input,
+// divides each by the tensor's scale in fp32 (round to nearest) and stores the
+// nearest E4M3 codes, saturating at +-448.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_fp8_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                                 int64_t key_stride_v, int64_t value_stride_v, uint4* k_cache,
+                                 uint4* v_cache, const int64_t* __restrict__ slot_mapping,
+                                 int64_t total_chunks, int chunks_per_row, int num_kv_heads,
+                                 int64_t num_slots, float k_scale, float v_scale,
+                                 int* dev_error) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= total_chunks) return;
+  const int64_t per_token = (int64_t)chunks_per_row * num_kv_heads;
+  const int64_t t = idx / per_token;
+  const int r = (int)(idx - t * per_token);
+  const int h = r / chunks_per_row;
+  const int c = r - h * chunks_per_row;
+  const int64_t slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (c == 0 && h == 0) report(dev_error, PA_DEVERR_SLOT_RANGE);
+    return;
+  }
+  const int64_t block = slot / kBlockSize;
+  const int64_t offset = slot - block * kBlockSize;
+  const int64_t dst = ((block * num_kv_heads + h) * kBlockSize + offset) * chunks_per_row + c;
+  const uint4* srcs[2] = {key + t * key_stride_v + 2 * r, value + t * value_stride_v + 2 * r};
+  uint4* caches[2] = {k_cache, v_cache};
+  const float scales[2] = {k_scale, v_scale};
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    float f[2][8];  // elements 0-7 and 8-15 of the chunk
+    Storage<T>::to_f32(__ldg(srcs[kv]), f[0]);
+    Storage<T>::to_f32(__ldg(srcs[kv] + 1), f[1]);
+    uint32_t w[4];  // w[i]: codes of elements 4i .. 4i+3, lowest byte first
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float* g = f[i >> 1] + 4 * (i & 1);
+      const uint32_t p0 =
+          f32x2_to_e4m3x2(__fdiv_rn(g[0], scales[kv]), __fdiv_rn(g[1], scales[kv]));
+      const uint32_t p1 =
+          f32x2_to_e4m3x2(__fdiv_rn(g[2], scales[kv]), __fdiv_rn(g[3], scales[kv]));
+      w[i] = (p0 & 0xffffu) | (p1 << 16);
+    }
+    caches[kv][dst] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 constexpr int kCopyThreads = 256;
@@ -110,6 +164,28 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, int64_t
       static_cast<const uint4*>(key), static_cast<const uint4*>(value), key_stride / 8,
       value_stride / 8, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping,
       total, chunks_per_row, num_kv_heads, (int64_t)num_blocks * kBlockSize, dev_error);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_stride,
+                                         int64_t value_stride, void* k_cache, void* v_cache,
+                                         const int64_t* slot_mapping, int num_tokens,
+                                         int num_kv_heads, int head_dim, int num_blocks,
+                                         int src_dtype, float k_scale, float v_scale,
+                                         int* dev_error, cudaStream_t stream) {
+  const int chunks_per_row = head_dim / 16;
+  const int64_t total = (int64_t)num_tokens * num_kv_heads * chunks_per_row;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  auto kern = src_dtype == PA_F16 ? reshape_and_cache_fp8_kernel<__half>
+                                  : reshape_and_cache_fp8_kernel<__nv_bfloat16>;
+  kern<<<(unsigned)blocks, threads, 0, stream>>>(
+      static_cast<const uint4*>(key), static_cast<const uint4*>(value), key_stride / 8,
+      value_stride / 8, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping,
+      total, chunks_per_row, num_kv_heads, (int64_t)num_blocks * kBlockSize, k_scale, v_scale,
+      dev_error);
   return cudaGetLastError();
 }
 

@@ -9,6 +9,7 @@
 
 namespace pa {
 
+// Outputs are multiplied by a.out_scale (the value scale of an E4M3 cache, else 1).
 // After the main loop every warp w has left, in shared memory,
 //   red_m[w][g], red_l[w][g]   its running max (base 2) and sum of exponentials
 //   red_acc[w][g][D]           its unnormalised output rows
@@ -45,7 +46,7 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
       A = fmaf(sc, red_acc[(w * G) * D + item], A);
     }
     if (!split) {
-      out_rows[item] = Storage<T>::from_f32(L > 0.f ? A / L : 0.f);
+      out_rows[item] = Storage<T>::from_f32(L > 0.f ? (A / L) * a.out_scale : 0.f);
     } else {
       const size_t row = (unit * a.max_parts + part) * G + g;
       a.ws_acc[row * D + (item % D)] = A;
@@ -111,7 +112,7 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
       o3 = fmaf(wts[(p + 3) * G + g], __ldcg(accp + (size_t)(p + 3) * G * D + item), o3);
     }
     for (; p < nparts; ++p) o0 = fmaf(wts[p * G + g], __ldcg(accp + (size_t)p * G * D + item), o0);
-    out_rows[item] = Storage<T>::from_f32((o0 + o1) + (o2 + o3));
+    out_rows[item] = Storage<T>::from_f32(((o0 + o1) + (o2 + o3)) * a.out_scale);
   }
   if (threadIdx.x == 0) a.ws_count[unit] = 0;
   __syncthreads();

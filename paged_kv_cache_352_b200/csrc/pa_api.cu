@@ -31,9 +31,14 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_cache_shape(int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype) {
-  if (dtype != PA_F16 && dtype != PA_BF16)
-    return fail(PA_ERR_UNSUPPORTED, "dtype %d: expected PA_F16 or PA_BF16", dtype);
+// Element bytes of a cache type (PA_F16, PA_BF16: 2; PA_FP8_E4M3: 1).
+int64_t elem_bytes(int dtype) { return dtype == PA_FP8_E4M3 ? 1 : 2; }
+
+int check_cache_shape(int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                      bool allow_fp8 = false) {
+  if (dtype != PA_F16 && dtype != PA_BF16 && !(allow_fp8 && dtype == PA_FP8_E4M3))
+    return fail(PA_ERR_UNSUPPORTED, "dtype %d: expected PA_F16 or PA_BF16%s", dtype,
+                allow_fp8 ? " or PA_FP8_E4M3" : "");
   if (block_size != kBlockSize)
     return fail(PA_ERR_UNSUPPORTED, "block_size %d: only %d is supported", block_size,
                 kBlockSize);
@@ -70,6 +75,8 @@ int cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return PA_OK;
   return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
+
+bool positive_finite(float x) { return x > 0.f && x <= 3.4028234663852886e38f; }
 
 }  // namespace
 
@@ -164,7 +171,8 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                    void* stream) {
   clear_error();
-  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype, true))
+    return st;
   if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs must be >= 0");
   if (num_pairs == 0) return PA_OK;
   if (!k_cache || !v_cache || !pairs) return fail(PA_ERR_INVALID_ARG, "null pointer argument");
@@ -186,7 +194,7 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
     if (srcs.count(d))
       return fail(PA_ERR_INVALID_ARG, "block %lld is both a source and a destination",
                   (long long)d);
-  const int64_t block_bytes = (int64_t)num_kv_heads * kBlockSize * head_dim * 2;
+  const int64_t block_bytes = (int64_t)num_kv_heads * kBlockSize * head_dim * elem_bytes(dtype);
   for (int first = 0; first < num_pairs; first += kMaxCopyPairsPerLaunch) {
     const int n = std::min(kMaxCopyPairsPerLaunch, num_pairs - first);
     CopyPairs cp;
@@ -206,7 +214,7 @@ int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, voi
                    void* dst_v, int dst_num_blocks, const int64_t* pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int dtype, void* stream) {
   clear_error();
-  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, src_num_blocks, dtype))
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, src_num_blocks, dtype, true))
     return st;
   if (dst_num_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "dst_num_blocks must be positive");
   if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs must be >= 0");
@@ -232,7 +240,7 @@ int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, voi
   if (int st = device_view(src_v, "src_v", &sv)) return st;
   if (int st = device_view(dst_k, "dst_k", &dk)) return st;
   if (int st = device_view(dst_v, "dst_v", &dv)) return st;
-  const int64_t block_bytes = (int64_t)num_kv_heads * kBlockSize * head_dim * 2;
+  const int64_t block_bytes = (int64_t)num_kv_heads * kBlockSize * head_dim * elem_bytes(dtype);
   for (int first = 0; first < num_pairs; first += kMaxCopyPairsPerLaunch) {
     const int n = std::min(kMaxCopyPairsPerLaunch, num_pairs - first);
     CopyPairs cp;
@@ -281,14 +289,19 @@ int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order) {
   return PA_OK;
 }
 
-int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, int max_blocks_per_seq,
-                    const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
-                    int max_context_len,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int num_blocks, float scale, int partition_tokens, void* workspace,
-                    size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
-  clear_error();
+}  // extern "C"
+
+namespace {
+
+// pa_paged_decode over a cache of type cache_dtype (dtype itself, or E4M3 with
+// key and value scales).
+int paged_decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                      int max_context_len, int num_q_heads, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, float scale, float k_scale, float v_scale,
+                      int partition_tokens, void* workspace, size_t workspace_bytes,
+                      int* dev_error, int dtype, int cache_dtype, void* stream) {
   if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "num_seqs must be >= 0");
   if (num_seqs > 65535)
@@ -339,15 +352,83 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
   a.num_blocks = num_blocks;
   a.part_blocks = lay.part_blocks;
   a.max_parts = lay.max_parts;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  const cudaError_t e =
-      launch_paged_decode(a, head_dim, group, dtype, static_cast<cudaStream_t>(stream));
+  a.scale_log2 = scale * 1.4426950408889634f * k_scale;
+  a.out_scale = v_scale;
+  const cudaError_t e = launch_paged_decode(a, head_dim, group, dtype, cache_dtype,
+                                            static_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidConfiguration)
     return fail(PA_ERR_UNSUPPORTED,
                 "%d partitions per sequence need more shared memory than the kernel allows; "
                 "use a larger partition_tokens",
                 lay.max_parts);
   return cuda_status(e, "paged_decode launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                    int max_context_len,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, float scale, int partition_tokens, void* workspace,
+                    size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
+  clear_error();
+  return paged_decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           context_lens, seq_order, num_seqs, max_context_len, num_q_heads,
+                           num_kv_heads, head_dim, block_size, num_blocks, scale, 1.f, 1.f,
+                           partition_tokens, workspace, workspace_bytes, dev_error, dtype, dtype,
+                           stream);
+}
+
+int pa_paged_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, int max_blocks_per_seq,
+                        const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
+                        int max_context_len, int num_q_heads, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, float scale, float k_scale,
+                        float v_scale, int partition_tokens, void* workspace,
+                        size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
+  clear_error();
+  if (!positive_finite(k_scale) || !positive_finite(v_scale))
+    return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
+  return paged_decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                           context_lens, seq_order, num_seqs, max_context_len, num_q_heads,
+                           num_kv_heads, head_dim, block_size, num_blocks, scale, k_scale, v_scale,
+                           partition_tokens, workspace, workspace_bytes, dev_error, dtype,
+                           PA_FP8_E4M3, stream);
+}
+
+int pa_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_token_stride,
+                             int64_t value_token_stride, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                             int head_dim, int block_size, int num_blocks, int src_dtype,
+                             float k_scale, float v_scale, int* dev_error, void* stream) {
+  clear_error();
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, src_dtype))
+    return st;
+  if (!positive_finite(k_scale) || !positive_finite(v_scale))
+    return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0");
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  const int64_t row = (int64_t)num_kv_heads * head_dim;
+  if (key_token_stride < row || value_token_stride < row || key_token_stride % 8 ||
+      value_token_stride % 8)
+    return fail(PA_ERR_INVALID_ARG,
+                "token strides (%lld, %lld) must be >= num_kv_heads*head_dim (%lld) and a "
+                "multiple of 8",
+                (long long)key_token_stride, (long long)value_token_stride, (long long)row);
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "key, value and cache pointers must be 16-byte aligned");
+  return cuda_status(
+      launch_reshape_and_cache_fp8(key, value, key_token_stride, value_token_stride, k_cache,
+                                   v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                   num_blocks, src_dtype, k_scale, v_scale, dev_error,
+                                   static_cast<cudaStream_t>(stream)),
+      "reshape_and_cache_fp8 launch");
 }
 
 }  // extern "C"

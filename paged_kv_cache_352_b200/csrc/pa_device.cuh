@@ -8,7 +8,9 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "pa_internal.h"
 
@@ -122,6 +124,75 @@ struct Storage<__nv_bfloat16> {
     return __float2bfloat16_rn(x);
   }
 };
+
+// Tag type of an 8-bit E4M3 cache (OCP FP8, no infinities; saturating stores).
+struct E4M3 {};
+
+// Element of a K/V cache: C is the query/output type T for 16-bit caches or E4M3.
+// Raw is the load unit holding 8 elements; to_f32 widens them exactly.
+template <typename C>
+struct CacheElem {
+  static constexpr int kBytes = 2;
+  using Raw = uint4;
+  static __device__ __forceinline__ void to_f32(const Raw& u, float (&f)[8]) {
+    Storage<C>::to_f32(u, f);
+  }
+};
+
+// Two E4M3 codes (low byte first) to two halves; exact (every code is a half).
+__device__ __forceinline__ uint32_t e4m3x2_to_half2_bits(uint32_t pair16) {
+  const __half2_raw h =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair16 & 0xffffu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h) {
+  __half2 v;
+  memcpy(&v, &h, sizeof(v));
+  return __half22float2(v);
+}
+
+template <>
+struct CacheElem<E4M3> {
+  static constexpr int kBytes = 1;
+  using Raw = uint2;
+  static __device__ __forceinline__ void to_f32(const Raw& u, float (&f)[8]) {
+    const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float2 x = half2_bits_to_float2(e4m3x2_to_half2_bits(w[i] >> (16 * k)));
+        f[4 * i + 2 * k] = x.x;
+        f[4 * i + 2 * k + 1] = x.y;
+      }
+    }
+  }
+};
+
+// Two E4M3 codes to the 16-bit pair of type T (exact for both half and bfloat16).
+template <typename T>
+__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t pair16);
+
+template <>
+__device__ __forceinline__ uint32_t e4m3x2_to<__half>(uint32_t pair16) {
+  return e4m3x2_to_half2_bits(pair16);
+}
+
+template <>
+__device__ __forceinline__ uint32_t e4m3x2_to<__nv_bfloat16>(uint32_t pair16) {
+  const float2 x = half2_bits_to_float2(e4m3x2_to_half2_bits(pair16));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(x.x, x.y);
+  uint32_t r;
+  memcpy(&r, &b, sizeof(r));
+  return r;
+}
+
+// Two floats to two E4M3 codes (`lo` in the low byte), nearest even, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
 
 // gpu-scope fetch-and-add with acquire + release semantics.
 __device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {

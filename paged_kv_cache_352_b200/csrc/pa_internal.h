@@ -46,7 +46,8 @@ struct DecodeArgs {
   int num_blocks;
   int part_blocks;   // blocks per split-KV partition
   int max_parts;     // partitions per sequence the grid covers
-  float scale_log2;  // softmax scale * log2(e)
+  float scale_log2;  // softmax scale * log2(e) (* the key scale of an E4M3 cache)
+  float out_scale;   // 1, or the value scale of an E4M3 cache
 };
 
 struct DecodeLayout {
@@ -59,8 +60,9 @@ struct DecodeLayout {
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                   int max_context_len, int partition_tokens, bool ordered, DecodeLayout* lay);
 
+// dtype: query/output type (PA_F16 or PA_BF16); cache_dtype: dtype or PA_FP8_E4M3.
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
-                                cudaStream_t stream);
+                                int cache_dtype, cudaStream_t stream);
 
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, int64_t key_stride,
@@ -68,6 +70,14 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, int64_t
                                      const int64_t* slot_mapping, int num_tokens,
                                      int num_kv_heads, int head_dim, int num_blocks,
                                      int* dev_error, cudaStream_t stream);
+
+// Quantizing write of 16-bit keys/values into E4M3 caches: code = E4M3(x / scale).
+cudaError_t launch_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_stride,
+                                         int64_t value_stride, void* k_cache, void* v_cache,
+                                         const int64_t* slot_mapping, int num_tokens,
+                                         int num_kv_heads, int head_dim, int num_blocks,
+                                         int src_dtype, float k_scale, float v_scale,
+                                         int* dev_error, cudaStream_t stream);
 
 struct CopyPairs {
   int32_t src[kMaxCopyPairsPerLaunch];

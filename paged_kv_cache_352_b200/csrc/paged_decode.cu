@@ -27,8 +27,13 @@
 //   all in logical order. Results depend only on logical token positions: not on
 //   physical placement, sharing or timing.
 //
+// E4M3 caches (8-bit codes with a key and a value scale) run the same kernel:
+// the key scale folds into the softmax scale, the value scale multiplies the
+// normalised output, and tiles are widened from codes on the chip.
+//
 // The kernel template lives in paged_decode_impl.cuh and is instantiated once
-// per (storage type, head_dim) in paged_decode_<type>_d<dim>.cu.
+// per (storage type, head_dim) in paged_decode_<type>_d<dim>.cu and once per
+// (query type, head_dim) over E4M3 caches in paged_decode_<type>_d<dim>_e4m3.cu.
 #include <cuda_runtime.h>
 
 #include "pa_internal.h"
@@ -39,15 +44,25 @@ cudaError_t launch_decode_f16_d64(const DecodeArgs& a, int group, cudaStream_t s
 cudaError_t launch_decode_f16_d128(const DecodeArgs& a, int group, cudaStream_t stream);
 cudaError_t launch_decode_bf16_d64(const DecodeArgs& a, int group, cudaStream_t stream);
 cudaError_t launch_decode_bf16_d128(const DecodeArgs& a, int group, cudaStream_t stream);
+cudaError_t launch_decode_f16_d64_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
+cudaError_t launch_decode_f16_d128_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
+cudaError_t launch_decode_bf16_d64_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
+cudaError_t launch_decode_bf16_d128_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
-                                cudaStream_t stream) {
+                                int cache_dtype, cudaStream_t stream) {
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (!fp8 && cache_dtype != dtype) return cudaErrorInvalidValue;
   if (dtype == PA_F16) {
-    if (head_dim == 64) return launch_decode_f16_d64(a, group, stream);
-    if (head_dim == 128) return launch_decode_f16_d128(a, group, stream);
+    if (head_dim == 64) return fp8 ? launch_decode_f16_d64_e4m3(a, group, stream)
+                                   : launch_decode_f16_d64(a, group, stream);
+    if (head_dim == 128) return fp8 ? launch_decode_f16_d128_e4m3(a, group, stream)
+                                    : launch_decode_f16_d128(a, group, stream);
   } else {
-    if (head_dim == 64) return launch_decode_bf16_d64(a, group, stream);
-    if (head_dim == 128) return launch_decode_bf16_d128(a, group, stream);
+    if (head_dim == 64) return fp8 ? launch_decode_bf16_d64_e4m3(a, group, stream)
+                                   : launch_decode_bf16_d64(a, group, stream);
+    if (head_dim == 128) return fp8 ? launch_decode_bf16_d128_e4m3(a, group, stream)
+                                    : launch_decode_bf16_d128(a, group, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -1,5 +1,6 @@
 // Paged-decode kernel template and its launcher, instantiated once per
-// (storage type, head_dim) in paged_decode_<type>_d<dim>.cu.
+// (storage type, head_dim) in paged_decode_<type>_d<dim>.cu, and per
+// (query type, head_dim) over E4M3 caches in paged_decode_<type>_d<dim>_e4m3.cu.
 #pragma once
 
 #include <cuda.h>
@@ -82,8 +83,9 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
   uint64_t* wbars = reinterpret_cast<uint64_t*>(smem + kRing) + warp * STAGES;
   int* wvalid = reinterpret_cast<int*>(smem + kRing + WARPS * STAGES * sizeof(uint64_t)) +
                 warp * STAGES;
-  float* wp = reinterpret_cast<float*>(smem + kRing + WARPS * STAGES * (sizeof(uint64_t) + 4)) +
-              warp * P::kPbufFloats;
+  constexpr size_t kHead = kRing + size_t(WARPS) * STAGES * (sizeof(uint64_t) + sizeof(int));
+  unsigned char* scratch =
+      smem + ((kHead + 127) & ~size_t(127)) + (size_t)warp * P::kScratchBytes;
   if (lane == 0) {
 #pragma unroll
     for (int st = 0; st < STAGES; ++st) mbar_init(&wbars[st], 1);
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
       break;
     }
     const int b = b_begin + warp + j * WARPS;
-    if (wvalid[st]) pol.block(wring + (size_t)st * P::kStageBytes, ctx - b * kBS, wp);
+    if (wvalid[st]) pol.block(wring + (size_t)st * P::kStageBytes, ctx - b * kBS, scratch);
     __syncwarp();
     if (j + STAGES < my_n) {
       if (lane == 0) fence_proxy_async_smem();  // this stage's reads precede its next copy
@@ -165,8 +167,8 @@ size_t smem_bytes(int max_parts) {
   const size_t wts = (size_t)max_parts * G * sizeof(float);
   size_t reuse = red > wts ? red : wts;
   if (reuse < ring) reuse = ring;
-  return P::kAlign + reuse + size_t(WARPS) * STAGES * (sizeof(uint64_t) + sizeof(int)) +
-         size_t(WARPS) * P::kPbufFloats * sizeof(float);
+  return P::kAlign + reuse + size_t(WARPS) * STAGES * (sizeof(uint64_t) + sizeof(int)) + 128 +
+         size_t(WARPS) * P::kScratchBytes;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -219,7 +221,7 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   CUtensorMap tk, tv;
   memset(&tk, 0, sizeof(tk));
   memset(&tv, 0, sizeof(tv));
-  if (!std::is_same<P, CudaCorePolicy<T, D, G>>::value) {
+  if (P::kTma2D) {
     const long long rows = (long long)a.num_blocks * a.num_kv_heads * kBS;
     if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA row coordinates are int32
     e = make_cache_map(&tk, a.k_cache, rows, D, dtype);
@@ -273,30 +275,32 @@ bool use_tensor_path(int group) {
   return group >= 4;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, typename C>
 cudaError_t launch_g(const DecodeArgs& a, int dtype, cudaStream_t stream) {
-  if (use_tensor_path(G)) return launch_tiles<TensorPolicy<T, D, G>, T, D, G>(a, dtype, stream);
-  return launch_tiles<CudaCorePolicy<T, D, G>, T, D, G>(a, dtype, stream);
+  if (use_tensor_path(G))
+    return launch_tiles<TensorPolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
+  return launch_tiles<CudaCorePolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
 }
 
-template <typename T, int D>
+template <typename T, int D, typename C>
 cudaError_t launch_group(const DecodeArgs& a, int group, int dtype, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_tiles<CudaCorePolicy<T, D, 1>, T, D, 1>(a, dtype, stream);
-    case 2: return launch_g<T, D, 2>(a, dtype, stream);
-    case 4: return launch_g<T, D, 4>(a, dtype, stream);
-    case 8: return launch_g<T, D, 8>(a, dtype, stream);
+    case 1: return launch_tiles<CudaCorePolicy<T, D, 1, C>, T, D, 1>(a, dtype, stream);
+    case 2: return launch_g<T, D, 2, C>(a, dtype, stream);
+    case 4: return launch_g<T, D, 4, C>(a, dtype, stream);
+    case 8: return launch_g<T, D, 8, C>(a, dtype, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-// Launches the persistent decode kernel for one storage type and head_dim.
-template <typename T, int D>
+// Launches the decode kernel for one query/output type T, head_dim and cache
+// element type C (T itself, or E4M3).
+template <typename T, int D, typename C = T>
 cudaError_t launch_decode_typed(const DecodeArgs& a, int group, int dtype,
                                 cudaStream_t stream) {
-  return launch_group<T, D>(a, group, dtype, stream);
+  return launch_group<T, D, C>(a, group, dtype, stream);
 }
 
 }  // namespace pa
