@@ -504,7 +504,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     err = torch.zeros(1, dtype=torch.int32, device=device)
     scale = 1.0 / math.sqrt(d)
     tot = {"steps": 0, "tokens": 0, "prefill_tokens": 0, "preempt": 0, "swap_blocks": 0,
-           "cow": 0, "kv_bytes": 0}
+           "cow": 0, "context": 0}
     util, contiguous = [], []
     row_bytes = hkv * d * 2
     torch.cuda.synchronize(device)
@@ -521,6 +521,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
         tot["preempt"] += c.num_preempted
         tot["swap_blocks"] += c.num_swap_out + c.num_swap_in
         tot["cow"] += c.num_copies
+        tot["context"] += c.total_context
         if tot["steps"] % 16 == 0 and c.num_seqs:
             filled, alloc = sched.kv_usage()
             util.append(filled / alloc)
@@ -537,6 +538,10 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
         "ms_per_step": round(ms / tot["steps"], 4),
         "host_ms_per_step": round(1e3 * host_s / tot["steps"], 4),
         "mean_batch": round(tot["tokens"] / tot["steps"], 1),
+        "mean_context": round(tot["context"] / max(tot["tokens"], 1), 1),
+        # K/V bytes the steps' decodes read, over the whole loop's time: how close
+        # the loop (host planning, copies, writes and decode together) runs to HBM
+        "decode_kv_gbs": round(tot["context"] * row_bytes * 2 / (ms / 1e3) / 1e9, 1),
         "generated_tokens": tot["tokens"], "prefill_tokens": tot["prefill_tokens"],
         "preemptions": tot["preempt"], "swapped_blocks": tot["swap_blocks"],
         "cow_copies": tot["cow"],
@@ -605,7 +610,7 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
             "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": round(achieved, 2),
             "frac_of_hbm_peak": round(achieved / peak, 4),
             "decode_tokens_per_s": round(wl.num_seqs / t, 1),
-            "speedup_vs_16bit_decode": round(dec16_s / t, 3),
+            "speedup_vs_16bit_decode": round(dec16_s / t, 3) if dec16_s == dec16_s else None,
             "what": "same batch as the 16-bit decode over E4M3 caches (random valid codes, "
                     "k_scale 0.05, v_scale 0.02), CUDA events per launch"}
 
@@ -691,6 +696,12 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     if r.error_bits():
         raise RuntimeError(f"device error bits {r.error_bits()} during warm-up")
+    if args.only == "fp8":
+        # profiling only: the 8-bit decode of this batch, nothing else
+        line = measure_fp8_decode(wl, r, device, l2_flush, float("nan"), _peaks()[0],
+                                  iters=args.steps)
+        print(json.dumps({"only": "fp8", "workload": wl.name, **line}), flush=True)
+        return 0
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -734,11 +745,12 @@ def run_ours(args):
     _barrier(world)
     e2e_s = _max_over_ranks(e_start.elapsed_time(e_end) / 1e3 / E, world, device)
 
-    swap = measure_swap(wl, r, device) if world == 1 else None
-    prefix_cache = measure_prefix_cache(wl, device) if world == 1 else None
-    batching = measure_continuous_batching(wl, device) if world == 1 else None
+    extras = world == 1 and args.only == "all"
+    swap = measure_swap(wl, r, device) if extras else None
+    prefix_cache = measure_prefix_cache(wl, device) if extras else None
+    batching = measure_continuous_batching(wl, device) if extras else None
     peak, peak_kind = _peaks()
-    fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) if world == 1 else None
+    fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) if extras else None
 
     sb = step_bytes(wl, r)
     db = decode_bytes(wl)
@@ -816,6 +828,10 @@ def main(argv=None):
                     help="profiling only: keep the first N sequences of the batch")
     ap.add_argument("--num-blocks", type=int, default=0,
                     help="profiling only: pool size for the truncated batch")
+    ap.add_argument("--only", choices=["all", "decode", "fp8"], default="all",
+                    help="profiling only: 'decode' times the step without the extra "
+                         "measurements (swap, prefix cache, batching loop, 8-bit decode); "
+                         "'fp8' times only the 8-bit decode of the batch (--steps launches)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     args = ap.parse_args(argv)

@@ -453,6 +453,7 @@ typedef struct {
   int num_seqs;            /* decode batch */
   int max_blocks_per_seq;  /* widest block table in the batch (>= 1) */
   int max_context_len;
+  int64_t total_context;   /* sum of the batch's context lengths (tokens decode reads) */
 } pa_sched_plan;
 
 /* num_blocks / block_size / initial_free_order as pa_bm_create. max_num_seqs

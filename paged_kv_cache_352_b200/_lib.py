@@ -561,7 +561,7 @@ class SchedPlanCounts(ctypes.Structure):
                 ("num_swap_in", ctypes.c_int), ("num_copies", ctypes.c_int),
                 ("num_prefill", ctypes.c_int), ("num_writes", ctypes.c_int),
                 ("num_seqs", ctypes.c_int), ("max_blocks_per_seq", ctypes.c_int),
-                ("max_context_len", ctypes.c_int)]
+                ("max_context_len", ctypes.c_int), ("total_context", ctypes.c_int64)]
 
 
 def _p(a):

@@ -89,6 +89,11 @@ struct CudaCorePolicy {
   static constexpr int kScratchBytes = G * kBS * 4;  // per warp: p values of one block
   static constexpr bool kTensorCores = false;
   static constexpr bool kTma2D = false;
+  static constexpr bool kFp8Cache = std::is_same<C, E4M3>::value;
+  // Three CTAs fit an SM's shared memory with the default 4 x 2 tiles (at most
+  // 170 registers a thread); the 4 and 8 query-head variants need more and are
+  // left to the compiler (they are not the default path).
+  static constexpr int kMinCtasPerSm = G > 2 ? 1 : 3;
   static_assert(LPT * TPW == 32 && TPL * TPW == kBS, "unsupported head_dim");
 
   int c, grp, own;
@@ -318,19 +323,17 @@ __device__ __forceinline__ uint32_t swz(int t, int chunk) {
   return (uint32_t)((chunk >> 3) * kHalfBytes + t * 128 + (((chunk & 7) ^ (t & 7)) << 4));
 }
 
-template <typename T, int D, int G, typename C = T>
+template <typename T, int D, int G>
 struct TensorPolicy {
-  // An E4M3 cache arrives raw by 1-D bulk copies and is widened into a per-warp
-  // scratch tile pair in the same swizzled 16-bit layout the TMA path produces.
-  static constexpr bool kFp8 = std::is_same<C, E4M3>::value;
   static constexpr int HALVES = D / 64;
-  static constexpr int kTileBytes = HALVES * kHalfBytes;  // a 16-bit tile
-  static constexpr int kRawTileBytes = kFp8 ? kBS * D : kTileBytes;
-  static constexpr int kStageBytes = 2 * kRawTileBytes;
-  static constexpr int kAlign = kFp8 ? 128 : 1024;  // 128-byte swizzled TMA destinations
-  static constexpr int kScratchBytes = kFp8 ? 2 * kTileBytes : 0;
+  static constexpr int kTileBytes = HALVES * kHalfBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kAlign = 1024;  // 128-byte swizzled TMA destinations
+  static constexpr int kScratchBytes = 0;
   static constexpr bool kTensorCores = true;
-  static constexpr bool kTma2D = !kFp8;
+  static constexpr bool kTma2D = true;
+  static constexpr bool kFp8Cache = false;
+  static constexpr int kMinCtasPerSm = 3;
   static constexpr int KSTEPS = D / 16;
   static constexpr int NTO = D / 8;  // output n-tiles of 8 columns
 
@@ -368,61 +371,18 @@ struct TensorPolicy {
   static __device__ __forceinline__ void issue(const DecodeArgs& a, const CUtensorMap* tm_k,
                                                const CUtensorMap* tm_v, unsigned char* dst,
                                                uint64_t* bar, int phys, int kvh) {
+    const int y = (phys * a.num_kv_heads + kvh) * kBS;
     mbar_arrive_expect_tx(bar, kStageBytes);
-    if constexpr (kFp8) {
-      const size_t off = ((size_t)phys * a.num_kv_heads + kvh) * kRawTileBytes;
-      bulk_copy_g2s(dst, static_cast<const unsigned char*>(a.k_cache) + off, kRawTileBytes, bar);
-      bulk_copy_g2s(dst + kRawTileBytes, static_cast<const unsigned char*>(a.v_cache) + off,
-                    kRawTileBytes, bar);
-    } else {
-      const int y = (phys * a.num_kv_heads + kvh) * kBS;
 #pragma unroll
-      for (int h = 0; h < HALVES; ++h) {
-        tma_load_2d(dst + h * kHalfBytes, tm_k, h * 64, y, bar);
-        tma_load_2d(dst + kTileBytes + h * kHalfBytes, tm_v, h * 64, y, bar);
-      }
+    for (int h = 0; h < HALVES; ++h) {
+      tma_load_2d(dst + h * kHalfBytes, tm_k, h * 64, y, bar);
+      tma_load_2d(dst + kTileBytes + h * kHalfBytes, tm_v, h * 64, y, bar);
     }
   }
 
-  // E4M3 tiles [16][D] bytes at `raw` -> 16-bit swizzled tiles at `dst`. Value
-  // rows past the context become zeros (their slots may hold NaN codes).
-  static __device__ __forceinline__ void widen(const unsigned char* raw, unsigned char* dst,
-                                               int valid) {
-    constexpr int CPR = D / 16;  // 16-byte chunks of codes per token row
-    constexpr int CHUNKS = 2 * kBS * CPR;
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int it = 0; it < CHUNKS / 32; ++it) {
-      const int idx = it * 32 + lane;
-      const int which = idx / (kBS * CPR);  // 0: K, 1: V (uniform across the warp)
-      const int rem = idx - which * kBS * CPR;
-      const int t = rem / CPR;
-      const int cc = rem - t * CPR;
-      uint4 w = *reinterpret_cast<const uint4*>(raw + which * kRawTileBytes + t * D + cc * 16);
-      if (which == 1 && t >= valid) w = make_uint4(0u, 0u, 0u, 0u);
-      uint4 lo, hi;
-      lo.x = e4m3x2_to<T>(w.x);
-      lo.y = e4m3x2_to<T>(w.x >> 16);
-      lo.z = e4m3x2_to<T>(w.y);
-      lo.w = e4m3x2_to<T>(w.y >> 16);
-      hi.x = e4m3x2_to<T>(w.z);
-      hi.y = e4m3x2_to<T>(w.z >> 16);
-      hi.z = e4m3x2_to<T>(w.w);
-      hi.w = e4m3x2_to<T>(w.w >> 16);
-      unsigned char* tile = dst + which * kTileBytes;
-      *reinterpret_cast<uint4*>(tile + swz(t, 2 * cc)) = lo;
-      *reinterpret_cast<uint4*>(tile + swz(t, 2 * cc + 1)) = hi;
-    }
-    __syncwarp();
-  }
-
-  __device__ __forceinline__ void block(unsigned char* stage, int valid, unsigned char* scratch) {
-    if constexpr (kFp8) {
-      widen(stage, scratch, valid);
-      stage = scratch;
-    }
+  __device__ __forceinline__ void block(unsigned char* stage, int valid, unsigned char*) {
     unsigned char* Vs = stage + kTileBytes;
-    if (!kFp8 && valid < kBS) {
+    if (valid < kBS) {
       // slots past the context may hold anything (even NaN patterns): zero them in V
       for (int idx = (threadIdx.x & 31); idx < (kBS - valid) * (D / 8); idx += 32) {
         const int t = valid + idx / (D / 8);

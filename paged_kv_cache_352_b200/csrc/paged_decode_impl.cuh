@@ -15,19 +15,18 @@
 
 #include "decode_common.cuh"
 #include "decode_policies.cuh"
+#include "decode_policy_fp8.cuh"
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
 namespace pa {
 namespace {
 
-// Register budget hint: with the default 4 x 2 tiles three CTAs fit an SM's
-// shared memory, so the kernels are compiled for three resident CTAs (at most
-// 170 registers a thread). The CUDA-core kernels for 4 and 8 query heads per KV
-// head need more and are left to the compiler (they are not the default path).
+// Register budget hint: each policy names the resident CTAs per SM its kernels
+// are compiled for (launch bounds), hence the registers a thread may use.
 template <class P, int G>
 constexpr int min_ctas_hint() {
-  return !P::kTensorCores && G > 2 ? 1 : 3;
+  return P::kMinCtasPerSm;
 }
 
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
@@ -202,6 +201,23 @@ cudaError_t make_cache_map(CUtensorMap* map, const void* base, long long rows, i
   return res == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// An E4M3 cache viewed as rows of head_dim (= 128) bytes, read in 16-row boxes
+// of whole rows with 128-byte swizzling.
+cudaError_t make_fp8_cache_map(CUtensorMap* map, const void* base, long long rows,
+                               int head_dim) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim};
+  cuuint32_t box[2] = {(cuuint32_t)head_dim, (cuuint32_t)kBS};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
 cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   const size_t smem = smem_bytes<P, WARPS, STAGES, G, D>(a.max_parts);
@@ -224,9 +240,15 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   if (P::kTma2D) {
     const long long rows = (long long)a.num_blocks * a.num_kv_heads * kBS;
     if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA row coordinates are int32
-    e = make_cache_map(&tk, a.k_cache, rows, D, dtype);
-    if (e != cudaSuccess) return e;
-    e = make_cache_map(&tv, a.v_cache, rows, D, dtype);
+    if constexpr (P::kFp8Cache) {
+      e = make_fp8_cache_map(&tk, a.k_cache, rows, D);
+      if (e != cudaSuccess) return e;
+      e = make_fp8_cache_map(&tv, a.v_cache, rows, D);
+    } else {
+      e = make_cache_map(&tk, a.k_cache, rows, D, dtype);
+      if (e != cudaSuccess) return e;
+      e = make_cache_map(&tv, a.v_cache, rows, D, dtype);
+    }
     if (e != cudaSuccess) return e;
   }
   dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
@@ -275,17 +297,38 @@ bool use_tensor_path(int group) {
   return group >= 4;
 }
 
+// Over E4M3 caches the CUDA-core path pays ~12 conversion instructions per 8
+// elements on top of its FMAs, while the tensor path converts each code pair
+// once, straight into its mma fragment; PA_DECODE_PATH overrides the choice here
+// too (for any group).
+bool use_tensor_path_e4m3(int group) {
+  static const int forced = [] {
+    const char* e = getenv("PA_DECODE_PATH");
+    if (e && !strcmp(e, "cuda_cores")) return 0;
+    if (e && !strcmp(e, "tensor")) return 1;
+    return -1;
+  }();
+  if (forced >= 0) return forced == 1;
+  return group >= 4;
+}
+
 template <typename T, int D, int G, typename C>
 cudaError_t launch_g(const DecodeArgs& a, int dtype, cudaStream_t stream) {
-  if (use_tensor_path(G))
-    return launch_tiles<TensorPolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
+  if constexpr (std::is_same<C, E4M3>::value) {
+    if (use_tensor_path_e4m3(G))
+      return launch_tiles<Fp8TensorPolicy<T, D, G>, T, D, G>(a, dtype, stream);
+  } else {
+    if (use_tensor_path(G)) return launch_tiles<TensorPolicy<T, D, G>, T, D, G>(a, dtype, stream);
+  }
   return launch_tiles<CudaCorePolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
 }
 
 template <typename T, int D, typename C>
 cudaError_t launch_group(const DecodeArgs& a, int group, int dtype, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_tiles<CudaCorePolicy<T, D, 1, C>, T, D, 1>(a, dtype, stream);
+    case 1:
+      if constexpr (std::is_same<C, E4M3>::value) return launch_g<T, D, 1, C>(a, dtype, stream);
+      return launch_tiles<CudaCorePolicy<T, D, 1, C>, T, D, 1>(a, dtype, stream);
     case 2: return launch_g<T, D, 2, C>(a, dtype, stream);
     case 4: return launch_g<T, D, 4, C>(a, dtype, stream);
     case 8: return launch_g<T, D, 8, C>(a, dtype, stream);

@@ -430,6 +430,9 @@ int pa_sched_step(pa_sched* s, pa_sched_plan* plan) {
   plan->num_seqs = (int)p.batch_request.size();
   plan->max_blocks_per_seq = p.max_blocks;
   plan->max_context_len = p.max_ctx;
+  int64_t total = 0;
+  for (int32_t c : p.batch_ctx) total += c;
+  plan->total_context = total;
   return PA_OK;
 }
 

@@ -39,6 +39,7 @@ def _compare_run(c, o, trace):
             ids = o.batch_seq_ids(op)
             want_t = o.bm.block_tables(ids, cp["tables"].shape[1])
             assert np.array_equal(cp["tables"], want_t), op.step
+        assert c.counts.total_context == sum(ctx for _, _, ctx in op.batch)
         assert c.kv_usage() == o.kv_usage()
         assert c.bm.free_list() == o.bm.free_list()
         stats["preempt"] += len(op.preempted)
