@@ -476,14 +476,15 @@ def continuous_batching_trace(num_requests: int = 1000, seed: int = 352, rate: f
 
 def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks: int = 8192,
                                 max_num_seqs: int = 256, host_blocks: int = 4096,
-                                max_model_len: int = 2048):
+                                max_model_len: int = 2048, fp8_scales=None):
     """The iteration-level batching loop end to end on one GPU: the library's
     scheduler plans each step and its executor runs swap-out/in, prefill writes,
     copy-on-write, new-token writes and decode (7B-like heads of ``wl``). Keys,
     values and queries are rows of a random device bank (no model). Reports
     generated tokens per second over the whole trace (CUDA events around the
     loop; host planning included), and KV occupancy sampled every 16 steps next
-    to what a contiguous ``max_model_len`` reservation per sequence would give."""
+    to what a contiguous ``max_model_len`` reservation per sequence would give.
+    ``fp8_scales = (k_scale, v_scale)`` runs the same trace over E4M3 caches."""
     import torch
     from paged_kv_cache_352_b200 import _lib as L
     trace = continuous_batching_trace(num_requests)
@@ -493,10 +494,11 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
                         max_num_seqs=max_num_seqs, num_host_blocks=host_blocks)
     for t in trace:
         sched.submit(*t)
-    sched.attach(hq, hkv, d, dt, max_model_len)
-    kc = torch.zeros(num_blocks, hkv, 16, d, dtype=dt, device=device)
+    sched.attach(hq, hkv, d, dt, max_model_len, fp8_scales=fp8_scales)
+    cdt = torch.uint8 if fp8_scales else dt
+    kc = torch.zeros(num_blocks, hkv, 16, d, dtype=cdt, device=device)
     vc = torch.zeros_like(kc)
-    hk = torch.zeros(host_blocks, hkv, 16, d, dtype=dt).pin_memory()
+    hk = torch.zeros(host_blocks, hkv, 16, d, dtype=cdt).pin_memory()
     hv = torch.zeros_like(hk).pin_memory()
     bank = torch.randn(num_blocks * 16, hkv, d, device=device).to(dt)
     qbank = torch.randn(max_num_seqs, hq, d, device=device).to(dt)
@@ -506,7 +508,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     tot = {"steps": 0, "tokens": 0, "prefill_tokens": 0, "preempt": 0, "swap_blocks": 0,
            "cow": 0, "context": 0}
     util, contiguous = [], []
-    row_bytes = hkv * d * 2
+    row_bytes = hkv * d * (1 if fp8_scales else 2)   # cached bytes of one (token, K or V) row
     torch.cuda.synchronize(device)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
@@ -548,6 +550,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
         "kv_utilization": round(float(np.mean(util)), 4) if util else None,
         "contiguous_reservation_utilization": (round(float(np.mean(contiguous)), 4)
                                                if contiguous else None),
+        "cache": "e4m3" if fp8_scales else wl.dtype,
         "what": f"{num_requests} requests (Poisson 1.0/step, lognormal prompts/outputs, "
                 f"1/2/4 samples), pool {num_blocks} blocks, batch cap {max_num_seqs}, "
                 f"host pool {host_blocks} blocks; utilization vs a {max_model_len}-token "
@@ -749,6 +752,8 @@ def run_ours(args):
     swap = measure_swap(wl, r, device) if extras else None
     prefix_cache = measure_prefix_cache(wl, device) if extras else None
     batching = measure_continuous_batching(wl, device) if extras else None
+    batching_fp8 = measure_continuous_batching(wl, device, fp8_scales=(0.05, 0.02)) \
+        if extras else None
     peak, peak_kind = _peaks()
     fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) if extras else None
 
@@ -799,6 +804,7 @@ def run_ours(args):
         "swap": swap,
         "prefix_cache": prefix_cache,
         "continuous_batching": batching,
+        "continuous_batching_fp8": batching_fp8,
         "fp8_kv": fp8,
         "clocks": csum,
     }

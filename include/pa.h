@@ -514,6 +514,13 @@ const pa_bm* pa_sched_block_manager(const pa_sched* s);
 int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim, int dtype,
                     int max_context_len);
 
+/* pa_sched_attach over 8-bit caches: the executor writes tokens with
+ * pa_reshape_and_cache_fp8 (key/value inputs of type dtype, scales k_scale /
+ * v_scale), decodes with pa_paged_decode_fp8 and copies and swaps one-byte
+ * pools (PA_FP8_E4M3; the pinned host pool holds codes too). */
+int pa_sched_attach_fp8(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim, int dtype,
+                        int max_context_len, float k_scale, float v_scale);
+
 /* Runs the last planned step on `stream` in device order: pa_swap_blocks for
  * the swap pairs (device pool k_cache/v_cache <-> pinned host pool
  * host_k/host_v, [num_host_blocks][Hkv][16][d]; may be NULL when the plan has

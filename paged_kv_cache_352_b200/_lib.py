@@ -105,6 +105,8 @@ _SIGS = {
     "pa_sched_kv_usage": (_c_int, [_vp, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64)]),
     "pa_sched_block_manager": (_vp, [_vp]),
     "pa_sched_attach": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "pa_sched_attach_fp8": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
+                                     ctypes.c_float]),
     "pa_sched_execute": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                   ctypes.c_float, _vp, _vp]),
 }
@@ -666,11 +668,20 @@ class Scheduler:
         }
 
     def attach(self, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype,
-               max_context_len: int) -> None:
+               max_context_len: int, fp8_scales=None) -> None:
+        """Allocate the executor for queries/inputs of ``dtype``; with
+        ``fp8_scales=(k_scale, v_scale)`` the pools are 8-bit E4M3 caches."""
         code = dtype if isinstance(dtype, int) else (
             PA_F16 if dtype == _torch().float16 else PA_BF16)
-        _check(self._lib.pa_sched_attach(self._h, num_q_heads, num_kv_heads, head_dim, code,
-                                         max_context_len))
+        if fp8_scales is None:
+            _check(self._lib.pa_sched_attach(self._h, num_q_heads, num_kv_heads, head_dim, code,
+                                             max_context_len))
+        else:
+            _check(self._lib.pa_sched_attach_fp8(self._h, num_q_heads, num_kv_heads, head_dim,
+                                                 code, max_context_len, float(fp8_scales[0]),
+                                                 float(fp8_scales[1])))
+        self.io_dtype = code
+        self.fp8 = fp8_scales is not None
 
     def execute(self, k_cache, v_cache, host_k, host_v, prefill_key, prefill_value, key, value,
                 q, out, scale: float, dev_error=None, stream=None) -> None:
@@ -678,10 +689,13 @@ class Scheduler:
         whose leading dimension covers the plan's counts; host_k/host_v are the
         pinned host pool (or None)."""
         torch = _torch()
-        dt = k_cache.dtype
+        if (dtype_code(k_cache) == PA_FP8_E4M3) != getattr(self, "fp8", False):
+            raise PAError(PA_ERR_INVALID_ARG, "cache element type differs from the attached one")
+        cdt = k_cache.dtype
+        dt = q.dtype
         host = lambda t, n: None if t is None else _pool_ptr(t, n)
         _check(self._lib.pa_sched_execute(
-            self._h, _dev_ptr(k_cache, "k_cache", dt), _dev_ptr(v_cache, "v_cache", dt),
+            self._h, _dev_ptr(k_cache, "k_cache", cdt), _dev_ptr(v_cache, "v_cache", cdt),
             host(host_k, "host_k"), host(host_v, "host_v"),
             _dev_ptr(prefill_key, "prefill_key", dt), _dev_ptr(prefill_value, "prefill_value", dt),
             _dev_ptr(key, "key", dt), _dev_ptr(value, "value", dt), _dev_ptr(q, "q", dt),

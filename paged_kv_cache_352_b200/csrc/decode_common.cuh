@@ -3,6 +3,7 @@
 #pragma once
 
 #include <math.h>
+#include <string.h>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -100,19 +101,60 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
     wts[idx] = headL[g] > 0.f ? exp2f(__ldcg(ml + idx * 2) - headM[g]) / headL[g] : 0.f;
   }
   __syncthreads();
-  const float* accp = a.ws_acc + unit * a.max_parts * G * D;
-  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
-    const int g = item / D;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+  // Each thread merges four adjacent output columns (one float4 of every
+  // partition's state), keeping kMergeInFlight partitions' loads in flight: the
+  // merge is bound by load latency, not bandwidth. Accumulator u takes the
+  // partitions p = u (mod kMergeInFlight) in increasing order and the
+  // accumulators are added in a fixed tree, so the result depends only on the
+  // partition count.
+  constexpr int kMergeInFlight = 8;
+  constexpr int kItems4 = G * D / 4;
+  const float4* accp = reinterpret_cast<const float4*>(a.ws_acc + unit * a.max_parts * G * D);
+  for (int it = threadIdx.x; it < kItems4; it += blockDim.x) {
+    const int g = (it * 4) / D;
+    float4 acc[kMergeInFlight];
+#pragma unroll
+    for (int u = 0; u < kMergeInFlight; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
     int p = 0;
-    for (; p + 4 <= nparts; p += 4) {
-      o0 = fmaf(wts[(p + 0) * G + g], __ldcg(accp + (size_t)(p + 0) * G * D + item), o0);
-      o1 = fmaf(wts[(p + 1) * G + g], __ldcg(accp + (size_t)(p + 1) * G * D + item), o1);
-      o2 = fmaf(wts[(p + 2) * G + g], __ldcg(accp + (size_t)(p + 2) * G * D + item), o2);
-      o3 = fmaf(wts[(p + 3) * G + g], __ldcg(accp + (size_t)(p + 3) * G * D + item), o3);
+    for (; p + kMergeInFlight <= nparts; p += kMergeInFlight) {
+#pragma unroll
+      for (int u = 0; u < kMergeInFlight; ++u) {
+        const float w = wts[(p + u) * G + g];
+        const float4 v = __ldcg(accp + (size_t)(p + u) * kItems4 + it);
+        acc[u].x = fmaf(w, v.x, acc[u].x);
+        acc[u].y = fmaf(w, v.y, acc[u].y);
+        acc[u].z = fmaf(w, v.z, acc[u].z);
+        acc[u].w = fmaf(w, v.w, acc[u].w);
+      }
     }
-    for (; p < nparts; ++p) o0 = fmaf(wts[p * G + g], __ldcg(accp + (size_t)p * G * D + item), o0);
-    out_rows[item] = Storage<T>::from_f32(((o0 + o1) + (o2 + o3)) * a.out_scale);
+#pragma unroll
+    for (int u = 0; u < kMergeInFlight; ++u) {
+      if (p + u < nparts) {
+        const float w = wts[(p + u) * G + g];
+        const float4 v = __ldcg(accp + (size_t)(p + u) * kItems4 + it);
+        acc[u].x = fmaf(w, v.x, acc[u].x);
+        acc[u].y = fmaf(w, v.y, acc[u].y);
+        acc[u].z = fmaf(w, v.z, acc[u].z);
+        acc[u].w = fmaf(w, v.w, acc[u].w);
+      }
+    }
+#pragma unroll
+    for (int step = 1; step < kMergeInFlight; step *= 2) {
+#pragma unroll
+      for (int u = 0; u < kMergeInFlight; u += 2 * step) {
+        acc[u].x += acc[u + step].x;
+        acc[u].y += acc[u + step].y;
+        acc[u].z += acc[u + step].z;
+        acc[u].w += acc[u + step].w;
+      }
+    }
+    T r[4] = {Storage<T>::from_f32(acc[0].x * a.out_scale),
+              Storage<T>::from_f32(acc[0].y * a.out_scale),
+              Storage<T>::from_f32(acc[0].z * a.out_scale),
+              Storage<T>::from_f32(acc[0].w * a.out_scale)};
+    uint2 packed;
+    memcpy(&packed, r, sizeof(packed));
+    *reinterpret_cast<uint2*>(out_rows + 4 * it) = packed;
   }
   if (threadIdx.x == 0) a.ws_count[unit] = 0;
   __syncthreads();

@@ -101,6 +101,8 @@ struct pa_sched {
   // executor
   bool attached = false;
   int hq = 0, hkv = 0, head_dim = 0, dtype = 0, max_ctx_cap = 0, max_blocks_cap = 0;
+  int cache_dtype = 0;              // dtype, or PA_FP8_E4M3
+  float k_scale = 1.f, v_scale = 1.f;
   size_t cap_prefill = 0, cap_tokens = 0, meta_bytes = 0;
   void* dev_meta = nullptr;
   void* host_meta[kRing] = {};
@@ -569,7 +571,22 @@ int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim
     return fail(PA_ERR_CUDA, "executor allocation failed: %s", cudaGetErrorString(e));
   }
   s->workspace_bytes = ws;
+  s->cache_dtype = dtype;
   s->attached = true;
+  return PA_OK;
+}
+
+int pa_sched_attach_fp8(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim, int dtype,
+                        int max_context_len, float k_scale, float v_scale) {
+  pa::clear_error();
+  if (!(k_scale > 0.f && k_scale <= 3.4028234663852886e38f && v_scale > 0.f &&
+        v_scale <= 3.4028234663852886e38f))
+    return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
+  if (int st = pa_sched_attach(s, num_q_heads, num_kv_heads, head_dim, dtype, max_context_len))
+    return st;
+  s->cache_dtype = PA_FP8_E4M3;
+  s->k_scale = k_scale;
+  s->v_scale = v_scale;
   return PA_OK;
 }
 
@@ -632,39 +649,46 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
   s->executed = true;
 
   const int nh = s->bm->num_host_blocks;
+  const int cdt = s->cache_dtype;
+  const bool fp8 = cdt == PA_FP8_E4M3;
   if (!p.swap_out.empty())
     if (int r = pa_swap_blocks(k_cache, v_cache, nb, host_k, host_v, nh, p.swap_out.data(),
-                               (int)p.swap_out.size() / 2, hkv, d, bs, s->dtype, stream))
+                               (int)p.swap_out.size() / 2, hkv, d, bs, cdt, stream))
       return r;
   if (!p.swap_in.empty())
     if (int r = pa_swap_blocks(host_k, host_v, nh, k_cache, v_cache, nb, p.swap_in.data(),
-                               (int)p.swap_in.size() / 2, hkv, d, bs, s->dtype, stream))
+                               (int)p.swap_in.size() / 2, hkv, d, bs, cdt, stream))
       return r;
   const int64_t row = (int64_t)hkv * d;
+  // the cache writes of one token list (prefill or new tokens) in the cache's type
+  auto write = [&](const void* kk, const void* vv, size_t off_slots, int n) {
+    const int64_t* slots = reinterpret_cast<const int64_t*>(dm + off_slots);
+    return fp8 ? pa_reshape_and_cache_fp8(kk, vv, row, row, k_cache, v_cache, slots, n, hkv, d, bs,
+                                          nb, s->dtype, s->k_scale, s->v_scale, dev_error, stream)
+               : pa_reshape_and_cache(kk, vv, row, row, k_cache, v_cache, slots, n, hkv, d, bs, nb,
+                                      s->dtype, dev_error, stream);
+  };
   if (!p.prefill.empty())
-    if (int r = pa_reshape_and_cache(prefill_key, prefill_value, row, row, k_cache, v_cache,
-                                     reinterpret_cast<const int64_t*>(dm + off_prefill),
-                                     (int)p.prefill.size(), hkv, d, bs, nb, s->dtype, dev_error,
-                                     stream))
-      return r;
+    if (int r = write(prefill_key, prefill_value, off_prefill, (int)p.prefill.size())) return r;
   if (!p.copies.empty())
     if (int r = pa_copy_blocks(k_cache, v_cache, p.copies.data(), (int)p.copies.size() / 2, hkv, d,
-                               bs, nb, s->dtype, stream))
+                               bs, nb, cdt, stream))
       return r;
   if (!p.writes.empty())
-    if (int r = pa_reshape_and_cache(key, value, row, row, k_cache, v_cache,
-                                     reinterpret_cast<const int64_t*>(dm + off_tok),
-                                     (int)p.writes.size(), hkv, d, bs, nb, s->dtype, dev_error,
-                                     stream))
-      return r;
-  if (nseq)
-    if (int r = pa_paged_decode(out, q, k_cache, v_cache,
-                                reinterpret_cast<const int32_t*>(dm + off_tables), p.max_blocks,
-                                reinterpret_cast<const int32_t*>(dm + off_ctx),
-                                reinterpret_cast<const int32_t*>(dm + off_order), nseq, p.max_ctx,
-                                s->hq, hkv, d, bs, nb, scale, 0, s->workspace, s->workspace_bytes,
-                                dev_error, s->dtype, stream))
-      return r;
+    if (int r = write(key, value, off_tok, (int)p.writes.size())) return r;
+  if (nseq) {
+    const int32_t* tables = reinterpret_cast<const int32_t*>(dm + off_tables);
+    const int32_t* ctx = reinterpret_cast<const int32_t*>(dm + off_ctx);
+    const int32_t* order = reinterpret_cast<const int32_t*>(dm + off_order);
+    const int r =
+        fp8 ? pa_paged_decode_fp8(out, q, k_cache, v_cache, tables, p.max_blocks, ctx, order, nseq,
+                                  p.max_ctx, s->hq, hkv, d, bs, nb, scale, s->k_scale, s->v_scale,
+                                  0, s->workspace, s->workspace_bytes, dev_error, s->dtype, stream)
+            : pa_paged_decode(out, q, k_cache, v_cache, tables, p.max_blocks, ctx, order, nseq,
+                              p.max_ctx, s->hq, hkv, d, bs, nb, scale, 0, s->workspace,
+                              s->workspace_bytes, dev_error, s->dtype, stream);
+    if (r) return r;
+  }
   return PA_OK;
 }
 

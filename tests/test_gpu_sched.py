@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import paged_kv_cache_352_b200 as pa
+from oracle import fp8 as F
 from oracle import scheduler as SCH
 from oracle.attention import softmax_attention
 from oracle.fpbits import bits_to_f64
@@ -20,8 +21,11 @@ from workloads import gen
 pytestmark = pytest.mark.gpu
 
 
-def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed):
+def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
+    """fp8 = (k_scale, v_scale) runs the loop over E4M3 caches; the oracle then
+    attends to the quantized-then-dequantized rows."""
     tdt = torch.float16 if dt == "f16" else torch.bfloat16
+    cdt = torch.uint8 if fp8 else tdt
     order = np.random.default_rng(seed).permutation(nb)
     c = pa.Scheduler(nb, 16, order, max_num_seqs=cap, num_host_blocks=host, preempt_mode=mode)
     o = SCH.Scheduler(nb, 16, order, max_num_seqs=cap, num_host_blocks=host, preempt_mode=mode)
@@ -29,10 +33,10 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed):
         c.submit(*t)
         o.submit(*t)
     max_ctx = max(p + n for _, p, n, _, _ in trace)
-    c.attach(hq, hkv, d, tdt, max_ctx)
-    kc = torch.zeros(nb, hkv, 16, d, dtype=tdt, device="cuda")
+    c.attach(hq, hkv, d, tdt, max_ctx, fp8_scales=fp8)
+    kc = torch.zeros(nb, hkv, 16, d, dtype=cdt, device="cuda")
     vc = torch.zeros_like(kc)
-    hk = torch.zeros(max(host, 1), hkv, 16, d, dtype=tdt).pin_memory() if host else None
+    hk = torch.zeros(max(host, 1), hkv, 16, d, dtype=cdt).pin_memory() if host else None
     hv = torch.zeros_like(hk).pin_memory() if host else None
     toks = gen.RequestTokens(seed, {r: p for r, p, *_ in trace}, hkv, d, dt)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -65,9 +69,13 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed):
         got = out_to_f64(out, dt)
         for i, (r, s, ctx) in enumerate(op.batch):
             K, V = toks.rows(r, s, range(ctx))
-            ref = np.stack([softmax_attention(bits_to_f64(q_bits[i, h], dt),
-                                              bits_to_f64(K[:, h // G], dt),
-                                              bits_to_f64(V[:, h // G], dt), scale)
+            if fp8:
+                Kf = F.dequantize(F.quantize(K, dt, fp8[0]), fp8[0])
+                Vf = F.dequantize(F.quantize(V, dt, fp8[1]), fp8[1])
+            else:
+                Kf, Vf = bits_to_f64(K, dt), bits_to_f64(V, dt)
+            ref = np.stack([softmax_attention(bits_to_f64(q_bits[i, h], dt), Kf[:, h // G],
+                                              Vf[:, h // G], scale)
                             for h in range(hq)])
             assert_close(got[i], ref, f"step {op.step} request {r} sample {s}")
         stats["steps"] += 1
@@ -107,3 +115,17 @@ def test_long_prompts_split_kv():
     st = _run_trace(trace, nb=600, cap=8, host=0, mode=pa.PA_PREEMPT_SWAP,
                     hq=16, hkv=2, d=128, dt="bf16", seed=43)
     assert st["steps"] > 0
+
+
+def test_swap_mode_trace_over_fp8_cache():
+    """The loop over E4M3 caches: quantizing writes, copy-on-write and swaps of
+    one-byte blocks, decode over the codes (tensor-core path, G = 4)."""
+    st = _run_trace(_trace(11, 24, 3), nb=26, cap=12, host=400, mode=pa.PA_PREEMPT_SWAP,
+                    hq=8, hkv=2, d=128, dt="bf16", seed=41, fp8=(0.02, 0.015))
+    assert st["preempt"] > 0 and st["swap"] > 0 and st["cow"] > 0, st
+
+
+def test_recompute_mode_trace_over_fp8_cache_mha():
+    st = _run_trace(_trace(12, 24, 1), nb=24, cap=10, host=0, mode=pa.PA_PREEMPT_RECOMPUTE,
+                    hq=4, hkv=4, d=64, dt="f16", seed=42, fp8=(0.01, 0.01))
+    assert st["preempt"] > 0, st
