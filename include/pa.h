@@ -240,6 +240,16 @@ int pa_paged_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_hea
                                    int head_dim, int max_context_len, int block_size,
                                    int partition_tokens, size_t* bytes);
 
+/* The split-KV plan pa_paged_decode (or pa_paged_decode_fp8) would use for these
+ * arguments (ordered != 0: a seq_order is passed): blocks per partition, the
+ * partitions per sequence the grid covers, and the kernel launches the call
+ * makes (1; 2 when short partitions run one warp per partition followed by a
+ * merge launch; 0 for an empty batch). The split mode itself is not observable
+ * in the results beyond floating-point rounding order. */
+int pa_paged_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                         int max_context_len, int block_size, int partition_tokens, int ordered,
+                         int* part_blocks, int* max_parts, int* launches);
+
 /* Host helper: order[0..n) = sequence indices by decreasing context_lens (ties
  * by index), the recommended seq_order. Both arrays are host memory. */
 int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order);

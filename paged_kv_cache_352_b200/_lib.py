@@ -63,6 +63,9 @@ _SIGS = {
                                          _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                          ctypes.c_float, _c_int, _vp, _c_int, _vp]),
     "pa_longest_first_order": (_c_int, [_vp, _c_int, _vp]),
+    "pa_paged_decode_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                      _c_int, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int),
+                                      ctypes.POINTER(_c_int)]),
     "pa_reshape_and_cache_fp8": (_c_int, [_vp, _vp, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int,
                                           _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
                                           ctypes.c_float, _vp, _vp]),
@@ -252,6 +255,16 @@ def pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim
                                                 max_context_len, block_size, partition_tokens,
                                                 ctypes.byref(out)))
     return out.value
+
+
+def pa_paged_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                         partition_tokens=0, ordered=False, block_size=BLOCK_SIZE):
+    """(blocks per partition, partitions per sequence, kernel launches) of a decode."""
+    pb, mp, nl = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().pa_paged_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                      max_context_len, block_size, partition_tokens, int(ordered),
+                                      ctypes.byref(pb), ctypes.byref(mp), ctypes.byref(nl)))
+    return pb.value, mp.value, nl.value
 
 
 def decode_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,

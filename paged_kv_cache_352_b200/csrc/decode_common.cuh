@@ -52,8 +52,8 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
       const size_t row = (unit * a.max_parts + part) * G + g;
       a.ws_acc[row * D + (item % D)] = A;
       if (item % D == 0) {
-        a.ws_ml[row * 2] = M;
-        a.ws_ml[row * 2 + 1] = L;
+        a.ws_m[row] = M;
+        a.ws_l[row] = L;
       }
     }
   }
@@ -78,16 +78,17 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
 
   // per-(partition, head) weights exp2(m_p - M) / L, staged in shared memory [nparts][G]
   __shared__ float headM[G], headL[G];
-  const float* ml = a.ws_ml + unit * a.max_parts * G * 2;
+  const float* pm = a.ws_m + unit * a.max_parts * G;
+  const float* pl = a.ws_l + unit * a.max_parts * G;
   for (int g = warp; g < G; g += WARPS) {
     float M = -INFINITY;
-    for (int p = lane; p < nparts; p += 32) M = fmaxf(M, __ldcg(ml + (p * G + g) * 2));
+    for (int p = lane; p < nparts; p += 32) M = fmaxf(M, __ldcg(pm + p * G + g));
 #pragma unroll
     for (int mask = 16; mask > 0; mask >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, mask));
     if (M == -INFINITY) M = 0.f;
     float L = 0.f;
     for (int p = lane; p < nparts; p += 32)
-      L += exp2f(__ldcg(ml + (p * G + g) * 2) - M) * __ldcg(ml + (p * G + g) * 2 + 1);
+      L += exp2f(__ldcg(pm + p * G + g) - M) * __ldcg(pl + p * G + g);
 #pragma unroll
     for (int mask = 16; mask > 0; mask >>= 1) L += __shfl_xor_sync(0xffffffffu, L, mask);
     if (lane == 0) {
@@ -98,7 +99,7 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
   __syncthreads();
   for (int idx = threadIdx.x; idx < nparts * G; idx += blockDim.x) {
     const int g = idx % G;
-    wts[idx] = headL[g] > 0.f ? exp2f(__ldcg(ml + idx * 2) - headM[g]) / headL[g] : 0.f;
+    wts[idx] = headL[g] > 0.f ? exp2f(__ldcg(pm + idx) - headM[g]) / headL[g] : 0.f;
   }
   __syncthreads();
   // Each thread merges four adjacent output columns (one float4 of every

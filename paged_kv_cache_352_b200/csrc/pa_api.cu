@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <algorithm>
 #include <string>
@@ -97,6 +99,23 @@ int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks, boo
   const int cap = ordered ? kMaxPartitionBlocksOrdered : kMaxPartitionBlocks;
   if (pb > cap) pb = cap;
   return (int)(pb < max_blocks ? pb : max_blocks);
+}
+
+// One warp per partition (plus a merge launch) pays off only for short partitions
+// and only while its grid, WARPS = 4 times smaller, still fills the GPU: the
+// library's own short partitions arise for small batches, which keep one CTA
+// per partition.
+bool use_warp_parts(int num_seqs, int num_kv_heads, int part_blocks, int max_parts) {
+  static const int forced = [] {
+    const char* e = getenv("PA_DECODE_SPLIT");
+    if (e && !strcmp(e, "cta")) return 0;
+    if (e && !strcmp(e, "warp")) return 1;
+    return -1;
+  }();
+  if (max_parts <= 1) return false;
+  if (forced >= 0) return forced == 1;
+  const long long ctas = (long long)num_kv_heads * num_seqs * ((max_parts + 3) / 4);
+  return part_blocks <= kWarpPartMaxBlocks && ctas >= kSplitTargetUnits;
 }
 
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -277,6 +296,28 @@ int pa_paged_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_hea
   return PA_OK;
 }
 
+int pa_paged_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                         int max_context_len, int block_size, int partition_tokens, int ordered,
+                         int* part_blocks, int* max_parts, int* launches) {
+  clear_error();
+  if (!part_blocks || !max_parts || !launches)
+    return fail(PA_ERR_INVALID_ARG, "null output pointer");
+  if (block_size != kBlockSize)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d: only %d is supported", block_size,
+                kBlockSize);
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "bad sequence or head counts");
+  DecodeLayout lay;
+  if (int st = decode_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                             partition_tokens, ordered != 0, &lay))
+    return st;
+  *part_blocks = lay.part_blocks;
+  *max_parts = lay.max_parts;
+  *launches = num_seqs == 0 ? 0
+              : use_warp_parts(num_seqs, num_kv_heads, lay.part_blocks, lay.max_parts) ? 2 : 1;
+  return PA_OK;
+}
+
 int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order) {
   clear_error();
   if (n < 0) return fail(PA_ERR_INVALID_ARG, "n must be >= 0");
@@ -341,7 +382,8 @@ int paged_decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.seq_order = seq_order;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   a.ws_count = lay.bytes ? reinterpret_cast<int*>(ws + lay.count_off) : nullptr;
-  a.ws_ml = lay.bytes ? reinterpret_cast<float*>(ws + lay.ml_off) : nullptr;
+  a.ws_m = lay.bytes ? reinterpret_cast<float*>(ws + lay.ml_off) : nullptr;
+  a.ws_l = lay.bytes ? a.ws_m + (size_t)num_seqs * num_kv_heads * lay.max_parts * group : nullptr;
   a.ws_acc = lay.bytes ? reinterpret_cast<float*>(ws + lay.acc_off) : nullptr;
   a.dev_error = dev_error;
   a.max_blocks_per_seq = max_blocks_per_seq;
@@ -354,6 +396,7 @@ int paged_decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.max_parts = lay.max_parts;
   a.scale_log2 = scale * 1.4426950408889634f * k_scale;
   a.out_scale = v_scale;
+  a.warp_parts = use_warp_parts(num_seqs, num_kv_heads, lay.part_blocks, lay.max_parts);
   const cudaError_t e = launch_paged_decode(a, head_dim, group, dtype, cache_dtype,
                                             static_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidConfiguration)

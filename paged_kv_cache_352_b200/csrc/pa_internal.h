@@ -34,7 +34,8 @@ struct DecodeArgs {
   const int32_t* block_tables;
   const int32_t* context_lens;
   const int32_t* seq_order;  // nullable: CTA z serves sequence seq_order[z]
-  float* ws_ml;      // [B][Hkv][max_parts][G][2]  (m, l) per partition
+  float* ws_m;       // [B][Hkv][max_parts][G]  running maximum (base 2) per partition
+  float* ws_l;       // [B][Hkv][max_parts][G]  sum of exponentials per partition
   float* ws_acc;     // [B][Hkv][max_parts][G][D]  unnormalised partition outputs
   int* ws_count;     // [B][Hkv]  partitions finished (returned to 0 by the merging CTA)
   int* dev_error;
@@ -48,7 +49,13 @@ struct DecodeArgs {
   int max_parts;     // partitions per sequence the grid covers
   float scale_log2;  // softmax scale * log2(e) (* the key scale of an E4M3 cache)
   float out_scale;   // 1, or the value scale of an E4M3 cache
+  int warp_parts;    // split mode: one warp per partition + a merge launch (else one CTA)
 };
+
+// Split partitions of at most this many blocks run one warp per partition when
+// that grid still has kSplitTargetUnits CTAs (PA_DECODE_SPLIT=cta|warp forces a mode).
+constexpr int kWarpPartMaxBlocks = 64;
+bool use_warp_parts(int num_seqs, int num_kv_heads, int part_blocks, int max_parts);
 
 struct DecodeLayout {
   int part_blocks;

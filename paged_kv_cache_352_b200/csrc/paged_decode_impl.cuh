@@ -154,6 +154,212 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
                                    out_rows);
 }
 
+// Split-KV with one warp per partition, for short partitions (at most
+// kWarpPartMaxBlocks blocks): warp w of CTA (kvh, y, z) streams partition
+// y * WARPS + w of sequence seq_order[z] through its own ring and leaves that
+// partition's state (m, l, unnormalised rows) in the workspace; no warp waits
+// for another. merge_partitions_kernel then writes every output. Compared with
+// one CTA per partition, each pipeline ramp and state write is amortised over
+// WARPS times more blocks, and no CTA-wide merge runs per partition.
+template <class P, typename T, int D, int G, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
+    paged_decode_warp_parts_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                                   const __grid_constant__ CUtensorMap tm_v) {
+  constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + P::kAlign - 1) & ~(uintptr_t)(P::kAlign - 1));
+  const int kvh = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int part = blockIdx.y * WARPS + warp;
+  const int s = a.seq_order ? __ldg(a.seq_order + blockIdx.z) : (int)blockIdx.z;
+  if ((unsigned)s >= (unsigned)a.num_seqs) {
+    if (blockIdx.y == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
+    return;
+  }
+  const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+  const int b_begin = part * a.part_blocks;
+  int ctx = __ldg(a.context_lens + s);
+  int win = -1;  // lane i holds the table entry of the warp's block win_base + i
+  {
+    const int idx = b_begin + lane;
+    if (lane < a.part_blocks && idx < a.max_blocks_per_seq) win = __ldg(table + idx);
+  }
+  P pol;
+  pol.init(lane);
+  pol.prefetch_q(a, s, kvh);
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * kBS || ctx > a.max_context_len) {
+    if (part == 0 && kvh == 0 && lane == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
+    ctx = 0;
+  }
+  const int nblk = (ctx + kBS - 1) / kBS;
+  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  if (part >= nparts) return;  // the whole warp: no barrier spans warps here
+  const int my_n = min(nblk, b_begin + a.part_blocks) - b_begin;
+
+  unsigned char* wring = smem + (size_t)warp * STAGES * P::kStageBytes;
+  uint64_t* wbars = reinterpret_cast<uint64_t*>(smem + kRing) + warp * STAGES;
+  int* wvalid = reinterpret_cast<int*>(smem + kRing + WARPS * STAGES * sizeof(uint64_t)) +
+                warp * STAGES;
+  constexpr size_t kHead = kRing + size_t(WARPS) * STAGES * (sizeof(uint64_t) + sizeof(int));
+  unsigned char* scratch =
+      smem + ((kHead + 127) & ~size_t(127)) + (size_t)warp * P::kScratchBytes;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&wbars[st], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  int win_base = 0;
+  auto issue = [&](int j) {
+    if (j >= win_base + 32) {
+      win_base = j & ~31;
+      win = win_base + lane < my_n ? __ldg(table + b_begin + win_base + lane) : -1;
+    }
+    const int phys = __shfl_sync(0xffffffffu, win, j - win_base);
+    if (lane == 0) {
+      const int st = j % STAGES;
+      uint64_t* bar = &wbars[st];
+      const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
+      wvalid[st] = ok;
+      if (!ok) {
+        report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
+        mbar_arrive(bar);
+      } else {
+        P::issue(a, &tm_k, &tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
+      }
+    }
+  };
+  for (int j = 0; j < STAGES && j < my_n; ++j) issue(j);
+  int issued = my_n < STAGES ? my_n : STAGES;
+  pol.begin(a.scale_log2);
+
+  bool aborted = false;
+  int j = 0;
+  for (; j < my_n; ++j) {
+    const int st = j % STAGES;
+    if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
+      if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+      aborted = true;
+      break;
+    }
+    if (wvalid[st]) pol.block(wring + (size_t)st * P::kStageBytes, ctx - (b_begin + j) * kBS, scratch);
+    __syncwarp();
+    if (j + STAGES < my_n) {
+      if (lane == 0) fence_proxy_async_smem();
+      issue(j + STAGES);
+      issued = j + STAGES + 1;
+    }
+  }
+  if (aborted) {
+    for (int k = j; k < issued; ++k)
+      mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
+  }
+  // the partition's state straight from registers: rows [G] of m, l and [G][D] of acc
+  const size_t row = (((size_t)s * a.num_kv_heads + kvh) * a.max_parts + part) * G;
+  pol.to_red(a.ws_m + row, a.ws_l + row, a.ws_acc + row * D, 0, lane);
+}
+
+// Second pass of the warp-per-partition split: one CTA per (sequence, query
+// head) merges that row's partition states in logical order,
+//   out = sum_p exp2(m_p - M) acc_p / sum_p exp2(m_p - M) l_p,  M = max_p m_p,
+// each thread owning a float4 of columns for the partitions p = set (mod kSets);
+// the sets are added in a fixed order.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(128) merge_partitions_kernel(const DecodeArgs a) {
+  constexpr int kCols = D / 4;
+  constexpr int kSets = 128 / kCols;
+  __shared__ float red[128];
+  __shared__ float4 part_sum[kSets][kCols];
+  const int kvh = blockIdx.x / G;
+  const int g = blockIdx.x - kvh * G;
+  const int s = blockIdx.y;
+  const int tid = threadIdx.x;
+  int ctx = __ldg(a.context_lens + s);
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * kBS || ctx > a.max_context_len) ctx = 0;
+  const int nblk = (ctx + kBS - 1) / kBS;
+  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  T* out = reinterpret_cast<T*>(a.out) + ((size_t)s * a.num_q_heads + (size_t)kvh * G + g) * D;
+  if (nparts == 0) {
+    for (int i = tid; i < D; i += blockDim.x) out[i] = Storage<T>::from_f32(0.f);
+    return;
+  }
+  const size_t base = ((size_t)s * a.num_kv_heads + kvh) * a.max_parts * G + g;
+  // M, then L, by fixed-order block reductions
+  float m = -INFINITY;
+  for (int p = tid; p < nparts; p += blockDim.x) m = fmaxf(m, __ldcg(a.ws_m + base + (size_t)p * G));
+  red[tid] = m;
+  __syncthreads();
+  for (int w = 64; w > 0; w >>= 1) {
+    if (tid < w) red[tid] = fmaxf(red[tid], red[tid + w]);
+    __syncthreads();
+  }
+  const float M = red[0] == -INFINITY ? 0.f : red[0];
+  __syncthreads();
+  float l = 0.f;
+  for (int p = tid; p < nparts; p += blockDim.x)
+    l += exp2f(__ldcg(a.ws_m + base + (size_t)p * G) - M) * __ldcg(a.ws_l + base + (size_t)p * G);
+  red[tid] = l;
+  __syncthreads();
+  for (int w = 64; w > 0; w >>= 1) {
+    if (tid < w) red[tid] += red[tid + w];
+    __syncthreads();
+  }
+  const float L = red[0];
+  const int col = tid % kCols;
+  const int set = tid / kCols;
+  const float4* acc = reinterpret_cast<const float4*>(a.ws_acc) + base * kCols;
+  float4 sum[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  int p = set;
+  for (; p + 3 * kSets < nparts; p += 4 * kSets) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = p + u * kSets;
+      const float w = exp2f(__ldcg(a.ws_m + base + (size_t)q * G) - M);
+      const float4 v = __ldcg(acc + (size_t)q * G * kCols + col);
+      sum[u].x = fmaf(w, v.x, sum[u].x);
+      sum[u].y = fmaf(w, v.y, sum[u].y);
+      sum[u].z = fmaf(w, v.z, sum[u].z);
+      sum[u].w = fmaf(w, v.w, sum[u].w);
+    }
+  }
+  for (int u = 0; p < nparts; p += kSets, ++u) {
+    const float w = exp2f(__ldcg(a.ws_m + base + (size_t)p * G) - M);
+    const float4 v = __ldcg(acc + (size_t)p * G * kCols + col);
+    sum[u].x = fmaf(w, v.x, sum[u].x);
+    sum[u].y = fmaf(w, v.y, sum[u].y);
+    sum[u].z = fmaf(w, v.z, sum[u].z);
+    sum[u].w = fmaf(w, v.w, sum[u].w);
+  }
+  float4 t;
+  t.x = (sum[0].x + sum[1].x) + (sum[2].x + sum[3].x);
+  t.y = (sum[0].y + sum[1].y) + (sum[2].y + sum[3].y);
+  t.z = (sum[0].z + sum[1].z) + (sum[2].z + sum[3].z);
+  t.w = (sum[0].w + sum[1].w) + (sum[2].w + sum[3].w);
+  part_sum[set][col] = t;
+  __syncthreads();
+  if (set == 0) {
+    float4 r = part_sum[0][col];
+#pragma unroll
+    for (int k = 1; k < kSets; ++k) {
+      r.x += part_sum[k][col].x;
+      r.y += part_sum[k][col].y;
+      r.z += part_sum[k][col].z;
+      r.w += part_sum[k][col].w;
+    }
+    const float f = L > 0.f ? a.out_scale / L : 0.f;
+    T o[4] = {Storage<T>::from_f32(r.x * f), Storage<T>::from_f32(r.y * f),
+              Storage<T>::from_f32(r.z * f), Storage<T>::from_f32(r.w * f)};
+    uint2 packed;
+    memcpy(&packed, o, sizeof(packed));
+    *reinterpret_cast<uint2*>(out + 4 * col) = packed;
+  }
+}
+
 constexpr size_t kSmemLimit = 200 * 1024;
 constexpr int kMaxDevices = 64;
 
@@ -250,6 +456,23 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
       e = make_cache_map(&tv, a.v_cache, rows, D, dtype);
     }
     if (e != cudaSuccess) return e;
+  }
+  if (a.warp_parts) {
+    auto wkern = paged_decode_warp_parts_kernel<P, T, D, G, WARPS, STAGES>;
+    static std::atomic<bool> wready[kMaxDevices];
+    if (!wready[dev].load(std::memory_order_acquire)) {
+      e = cudaFuncSetAttribute(wkern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmemLimit);
+      if (e != cudaSuccess) return e;
+      wready[dev].store(true, std::memory_order_release);
+    }
+    dim3 wgrid(a.num_kv_heads, (a.max_parts + WARPS - 1) / WARPS, a.num_seqs);
+    wkern<<<wgrid, WARPS * 32, smem, stream>>>(a, tk, tv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dim3 mgrid(a.num_kv_heads * G, a.num_seqs);
+    merge_partitions_kernel<T, D, G><<<mgrid, 128, 0, stream>>>(a);
+    return cudaGetLastError();
   }
   dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
   kern<<<grid, WARPS * 32, smem, stream>>>(a, tk, tv);

@@ -180,8 +180,12 @@ class DecodeRunner:
         return self.decode()
 
     def launches_per_step(self) -> int:
+        wl = self.wl
+        _, _, decode = L.pa_paged_decode_plan(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                              wl.head_dim, wl.max_context_len,
+                                              self.partition_tokens or 0, ordered=True)
         return int(len(self.cow_pairs) > 0) * -(-len(self.cow_pairs) // 1024) + \
-            int(len(self.step_slots_host) > 0) + 1
+            int(len(self.step_slots_host) > 0) + decode
 
     def error_bits(self) -> int:
         return int(self.dev_error.item())

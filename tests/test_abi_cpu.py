@@ -318,3 +318,23 @@ def test_block_manager_seventy_tokens(golden):
     t = bm.table(0)
     assert len(t) == g["blocks"]
     assert sum(1 for s in slots if s // 16 == t[-1]) == g["last_block_used"]
+
+
+def test_decode_plan_split_modes():
+    """Short caller-chosen partitions over a large grid run one warp per partition
+    plus a merge launch; small batches and unsplit calls keep one launch."""
+    if os.environ.get("PA_DECODE_SPLIT"):
+        pytest.skip("split mode forced by the environment")
+    # the long-context configuration: 8 sequences up to 128k tokens, 512-token partitions
+    assert L.pa_paged_decode_plan(8, 64, 8, 128, 131072, 512, ordered=True) == (32, 256, 2)
+    # one long sequence: too few CTAs for one warp per partition
+    assert L.pa_paged_decode_plan(1, 64, 8, 128, 32768, 512, ordered=True) == (32, 64, 1)
+    # long partitions stay one CTA per partition
+    assert L.pa_paged_decode_plan(8, 64, 8, 128, 131072, 2048, ordered=True)[2] == 1
+    # no split at all, and an empty batch
+    assert L.pa_paged_decode_plan(64, 32, 32, 128, 2048, 0, ordered=True) == (128, 1, 1)
+    assert L.pa_paged_decode_plan(0, 32, 32, 128, 2048, 0)[2] == 0
+    with pytest.raises(L.PAError):
+        L.pa_paged_decode_plan(4, 30, 8, 128, 100, 0)          # heads not a multiple
+    with pytest.raises(L.PAError):
+        L.pa_paged_decode_plan(4, 32, 8, 128, 100, 24)         # partition not whole blocks
