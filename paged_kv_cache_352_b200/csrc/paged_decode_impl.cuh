@@ -267,11 +267,13 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
 //   out = sum_p exp2(m_p - M) acc_p / sum_p exp2(m_p - M) l_p,  M = max_p m_p,
 // each thread owning a float4 of columns for the partitions p = set (mod kSets);
 // the sets are added in a fixed order.
+constexpr int kMergeThreads = 512;
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(128) merge_partitions_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) merge_partitions_kernel(const DecodeArgs a) {
   constexpr int kCols = D / 4;
-  constexpr int kSets = 128 / kCols;
-  __shared__ float red[128];
+  constexpr int kSets = kMergeThreads / kCols;
+  __shared__ float red[kMergeThreads];
   __shared__ float4 part_sum[kSets][kCols];
   const int kvh = blockIdx.x / G;
   const int g = blockIdx.x - kvh * G;
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(128) merge_partitions_kernel(const DecodeArgs 
   for (int p = tid; p < nparts; p += blockDim.x) m = fmaxf(m, __ldcg(a.ws_m + base + (size_t)p * G));
   red[tid] = m;
   __syncthreads();
-  for (int w = 64; w > 0; w >>= 1) {
+  for (int w = kMergeThreads / 2; w > 0; w >>= 1) {
     if (tid < w) red[tid] = fmaxf(red[tid], red[tid + w]);
     __syncthreads();
   }
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(128) merge_partitions_kernel(const DecodeArgs 
     l += exp2f(__ldcg(a.ws_m + base + (size_t)p * G) - M) * __ldcg(a.ws_l + base + (size_t)p * G);
   red[tid] = l;
   __syncthreads();
-  for (int w = 64; w > 0; w >>= 1) {
+  for (int w = kMergeThreads / 2; w > 0; w >>= 1) {
     if (tid < w) red[tid] += red[tid + w];
     __syncthreads();
   }
@@ -327,13 +329,17 @@ __global__ void __launch_bounds__(128) merge_partitions_kernel(const DecodeArgs 
       sum[u].w = fmaf(w, v.w, sum[u].w);
     }
   }
-  for (int u = 0; p < nparts; p += kSets, ++u) {
-    const float w = exp2f(__ldcg(a.ws_m + base + (size_t)p * G) - M);
-    const float4 v = __ldcg(acc + (size_t)p * G * kCols + col);
-    sum[u].x = fmaf(w, v.x, sum[u].x);
-    sum[u].y = fmaf(w, v.y, sum[u].y);
-    sum[u].z = fmaf(w, v.z, sum[u].z);
-    sum[u].w = fmaf(w, v.w, sum[u].w);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {  // at most three partitions of this set are left
+    const int q = p + u * kSets;
+    if (q < nparts) {
+      const float w = exp2f(__ldcg(a.ws_m + base + (size_t)q * G) - M);
+      const float4 v = __ldcg(acc + (size_t)q * G * kCols + col);
+      sum[u].x = fmaf(w, v.x, sum[u].x);
+      sum[u].y = fmaf(w, v.y, sum[u].y);
+      sum[u].z = fmaf(w, v.z, sum[u].z);
+      sum[u].w = fmaf(w, v.w, sum[u].w);
+    }
   }
   float4 t;
   t.x = (sum[0].x + sum[1].x) + (sum[2].x + sum[3].x);
@@ -471,7 +477,7 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 mgrid(a.num_kv_heads * G, a.num_seqs);
-    merge_partitions_kernel<T, D, G><<<mgrid, 128, 0, stream>>>(a);
+    merge_partitions_kernel<T, D, G><<<mgrid, kMergeThreads, 0, stream>>>(a);
     return cudaGetLastError();
   }
   dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
