@@ -474,9 +474,29 @@ def continuous_batching_trace(num_requests: int = 1000, seed: int = 352, rate: f
             for i in range(num_requests)]
 
 
+def shared_prompt_trace(num_requests: int = 1000, seed: int = 353, systems: int = 8,
+                        system_len: int = 512, rate: float = 1.0):
+    """Seeded trace whose prompts are one of ``systems`` shared ``system_len``-token
+    system prompts followed by a lognormal number (median 128, clipped to
+    8..1024) of the request's own tokens, with token ids; outputs and samples as
+    ``continuous_batching_trace``."""
+    rng = np.random.default_rng(seed)
+    sys_prompts = [rng.integers(0, 32000, system_len).tolist() for _ in range(systems)]
+    arrival = np.floor(np.cumsum(rng.exponential(1 / rate, num_requests))).astype(np.int64)
+    own = np.clip(np.rint(rng.lognormal(np.log(128), 0.8, num_requests)), 8, 1024).astype(int)
+    output = np.clip(np.rint(rng.lognormal(np.log(200), 0.8, num_requests)), 4, 512)
+    samples = rng.choice([1, 2, 4], num_requests, p=[0.85, 0.10, 0.05])
+    trace = []
+    for i in range(num_requests):
+        toks = sys_prompts[int(rng.integers(systems))] + rng.integers(0, 32000, own[i]).tolist()
+        trace.append((i, len(toks), int(output[i]), int(samples[i]), int(arrival[i]), toks))
+    return trace
+
+
 def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks: int = 8192,
                                 max_num_seqs: int = 256, host_blocks: int = 4096,
-                                max_model_len: int = 2048, fp8_scales=None):
+                                max_model_len: int = 2048, fp8_scales=None, trace=None,
+                                use_tokens: bool = False):
     """The iteration-level batching loop end to end on one GPU: the library's
     scheduler plans each step and its executor runs swap-out/in, prefill writes,
     copy-on-write, new-token writes and decode (7B-like heads of ``wl``). Keys,
@@ -484,16 +504,19 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     generated tokens per second over the whole trace (CUDA events around the
     loop; host planning included), and KV occupancy sampled every 16 steps next
     to what a contiguous ``max_model_len`` reservation per sequence would give.
-    ``fp8_scales = (k_scale, v_scale)`` runs the same trace over E4M3 caches."""
+    ``fp8_scales = (k_scale, v_scale)`` runs the same trace over E4M3 caches;
+    ``trace`` replaces the default trace, and ``use_tokens`` submits its token ids
+    so that admission goes through the prefix cache."""
     import torch
     from paged_kv_cache_352_b200 import _lib as L
-    trace = continuous_batching_trace(num_requests)
+    trace = continuous_batching_trace(num_requests) if trace is None else trace
+    num_requests = len(trace)
     dt = torch.float16 if wl.dtype == "f16" else torch.bfloat16
     hq, hkv, d = wl.num_q_heads, wl.num_kv_heads, wl.head_dim
     sched = L.Scheduler(num_blocks, 16, np.random.default_rng(7).permutation(num_blocks),
                         max_num_seqs=max_num_seqs, num_host_blocks=host_blocks)
     for t in trace:
-        sched.submit(*t)
+        sched.submit(*t[:5], tokens=t[5] if use_tokens else None)
     sched.attach(hq, hkv, d, dt, max_model_len, fp8_scales=fp8_scales)
     cdt = torch.uint8 if fp8_scales else dt
     kc = torch.zeros(num_blocks, hkv, 16, d, dtype=cdt, device=device)
@@ -506,7 +529,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     err = torch.zeros(1, dtype=torch.int32, device=device)
     scale = 1.0 / math.sqrt(d)
     tot = {"steps": 0, "tokens": 0, "prefill_tokens": 0, "preempt": 0, "swap_blocks": 0,
-           "cow": 0, "context": 0}
+           "cow": 0, "context": 0, "cached": 0}
     util, contiguous = [], []
     row_bytes = hkv * d * (1 if fp8_scales else 2)   # cached bytes of one (token, K or V) row
     torch.cuda.synchronize(device)
@@ -524,6 +547,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
         tot["swap_blocks"] += c.num_swap_out + c.num_swap_in
         tot["cow"] += c.num_copies
         tot["context"] += c.total_context
+        tot["cached"] += c.num_cached_tokens
         if tot["steps"] % 16 == 0 and c.num_seqs:
             filled, alloc = sched.kv_usage()
             util.append(filled / alloc)
@@ -545,6 +569,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
         # the loop (host planning, copies, writes and decode together) runs to HBM
         "decode_kv_gbs": round(tot["context"] * row_bytes * 2 / (ms / 1e3) / 1e9, 1),
         "generated_tokens": tot["tokens"], "prefill_tokens": tot["prefill_tokens"],
+        "cached_prompt_tokens": tot["cached"],
         "preemptions": tot["preempt"], "swapped_blocks": tot["swap_blocks"],
         "cow_copies": tot["cow"],
         "kv_utilization": round(float(np.mean(util)), 4) if util else None,
@@ -754,6 +779,13 @@ def run_ours(args):
     batching = measure_continuous_batching(wl, device) if extras else None
     batching_fp8 = measure_continuous_batching(wl, device, fp8_scales=(0.05, 0.02)) \
         if extras else None
+    batching_prefix = None
+    if extras:
+        spt = shared_prompt_trace()
+        batching_prefix = {
+            "with_cache": measure_continuous_batching(wl, device, trace=spt, use_tokens=True),
+            "without_cache": measure_continuous_batching(wl, device, trace=spt),
+        }
     peak, peak_kind = _peaks()
     fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) if extras else None
 
@@ -805,6 +837,7 @@ def run_ours(args):
         "prefix_cache": prefix_cache,
         "continuous_batching": batching,
         "continuous_batching_fp8": batching_fp8,
+        "continuous_batching_shared_prompts": batching_prefix,
         "fp8_kv": fp8,
         "clocks": csum,
     }

@@ -382,6 +382,12 @@ int pa_bm_host_free_list(const pa_bm* bm, int32_t* out, int capacity);
  * All-or-nothing like the other calls. */
 int pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* token_ids, int num_tokens,
                          int64_t* slots_out, int* num_cached_tokens);
+/* Read-only look-up for admission decisions: *hit_blocks = the leading full
+ * blocks of these prompt tokens found in the cache (what pa_bm_add_seq_cached
+ * would share), *revived_blocks = how many of those are held by no sequence
+ * (counted in pa_bm_num_free, so sharing them uses up free blocks). */
+int pa_bm_cached_prefix(const pa_bm* bm, const int32_t* token_ids, int num_tokens,
+                        int* hit_blocks, int* revived_blocks);
 int pa_bm_num_cached(const pa_bm* bm);
 /* Evictable cached blocks, oldest first, into out[capacity]; returns the count or -1. */
 int pa_bm_evictable_list(const pa_bm* bm, int32_t* out, int capacity);
@@ -464,6 +470,7 @@ typedef struct {
   int max_blocks_per_seq;  /* widest block table in the batch (>= 1) */
   int max_context_len;
   int64_t total_context;   /* sum of the batch's context lengths (tokens decode reads) */
+  int64_t num_cached_tokens;  /* prompt tokens of admitted requests found in the prefix cache */
 } pa_sched_plan;
 
 /* num_blocks / block_size / initial_free_order as pa_bm_create. max_num_seqs
@@ -480,6 +487,18 @@ void pa_sched_destroy(pa_sched* s);
  * output_len) / block_size) > num_blocks). */
 int pa_sched_submit(pa_sched* s, int64_t request_id, int prompt_len, int output_len,
                     int num_samples, int64_t arrival_step);
+
+/* pa_sched_submit with the prompt's token ids (prompt_tokens[prompt_len], copied):
+ * the request is admitted through the block manager's prefix cache
+ * (pa_bm_add_seq_cached). Leading full prompt blocks already cached (by earlier
+ * requests, or by this one before it was dropped for recomputation) are shared
+ * and not written again; the admission check counts the blocks found, less
+ * those no sequence holds. A recomputed request re-registers its prompt this
+ * way and appends its generated tokens after it ("PagedAttention: The vLLM
+ * Paper", "Impact and Follow-Ups", item 1, prefix caching). */
+int pa_sched_submit_tokens(pa_sched* s, int64_t request_id, const int32_t* prompt_tokens,
+                           int prompt_len, int output_len, int num_samples,
+                           int64_t arrival_step);
 
 /* Plans the next step and writes its counts to *plan. PA_ERR_NO_FREE_BLOCKS if
  * a many-sample request could not be preempted (host pool full); the scheduler

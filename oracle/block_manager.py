@@ -253,6 +253,22 @@ class BlockManager:
         self._lens[seq_id] = num_tokens
         return [self._slot(table, p) for p in range(num_tokens)]
 
+    def cached_prefix(self, token_ids):
+        """(leading full blocks of these prompt tokens found in the cache, how many
+        of them are evictable, i.e. held by no sequence); changes nothing."""
+        tokens = [int(t) for t in token_ids]
+        bs = self.block_size
+        hits = revived = 0
+        parent = -1
+        for i in range(len(tokens) // bs):
+            b = self._cache.get((parent, tuple(tokens[i * bs:(i + 1) * bs])))
+            if b is None:
+                break
+            hits += 1
+            revived += self._ref[b] == 0
+            parent = b
+        return hits, revived
+
     def add_seq_cached(self, seq_id: int, token_ids):
         """Register a sequence from its prompt's token ids, sharing the leading
         full blocks already cached. Returns ``(slots, num_cached_tokens)``; the

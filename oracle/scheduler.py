@@ -47,6 +47,12 @@ rules so that plans can be compared bit for bit):
     cannot be swapped is an error. In recompute mode there is no host pool
     and every request must have one sample.
   * Arrival order is (arrival step, submission order).
+  * A request submitted with its prompt's token ids is admitted through the
+    block manager's prefix cache (``add_seq_cached``): the leading full prompt
+    blocks found cached are shared and only the rest of the prompt is written.
+    Its admission need subtracts the blocks found and adds back those of them
+    that no sequence holds (they are counted as free). A recomputed request
+    re-registers its prompt the same way and then appends its generated tokens.
   * The device executes a step in this order: swap-out pairs, swap-in pairs,
     prefill writes (the prompts, and recomputed tokens, of admitted requests),
     copy-on-write pairs, new-token writes, then decode. Prefill comes before
@@ -85,6 +91,7 @@ class Request:
     order: int
     generated: int = 0
     state: str = "pending"      # pending, waiting, running, swapped, finished
+    tokens: tuple = None        # prompt token ids (admission through the prefix cache)
 
 
 @dataclass
@@ -100,6 +107,7 @@ class Plan:
     copies: list = field(default_factory=list)          # (src block, dst block)
     writes: list = field(default_factory=list)          # (request, sample, position, slot)
     batch: list = field(default_factory=list)           # (request, sample, context_len)
+    cached: int = 0                                     # prompt tokens found in the prefix cache
 
 
 class Scheduler:
@@ -127,7 +135,7 @@ class Scheduler:
 
     # -- requests ---------------------------------------------------------
     def submit(self, rid: int, prompt_len: int, output_len: int, num_samples: int = 1,
-               arrival: int = 0) -> None:
+               arrival: int = 0, tokens=None) -> None:
         if rid in self.requests or rid < 0:
             raise BlockManagerError(ERR_INVALID_ARG, "bad or duplicate request id")
         if prompt_len < 1 or output_len < 1 or not 1 <= num_samples <= MAX_SAMPLES:
@@ -137,7 +145,10 @@ class Scheduler:
         worst = num_samples * _ceil_div(prompt_len + output_len, self.block_size)
         if num_samples > self.max_num_seqs or worst > self.bm.num_blocks:
             raise BlockManagerError(ERR_NO_FREE_BLOCKS, "request can never fit")
-        r = Request(rid, prompt_len, output_len, num_samples, arrival, self._submitted)
+        if tokens is not None and len(tokens) != prompt_len:
+            raise BlockManagerError(ERR_INVALID_ARG, "one token id per prompt position")
+        r = Request(rid, prompt_len, output_len, num_samples, arrival, self._submitted,
+                    tokens=None if tokens is None else tuple(int(t) for t in tokens))
         self._submitted += 1
         self.requests[rid] = r
         self.pending.append(r)
@@ -181,7 +192,10 @@ class Scheduler:
     def _admit_need(self, r: Request) -> int:
         length = r.prompt_len + r.generated
         extra = r.num_samples if length % self.block_size == 0 else r.num_samples - 1
-        return _ceil_div(length, self.block_size) + extra
+        hits = revived = 0
+        if r.tokens is not None:
+            hits, revived = self.bm.cached_prefix(r.tokens)
+        return _ceil_div(length, self.block_size) - hits + revived + extra
 
     # -- one iteration ----------------------------------------------------
     def _append(self, r: Request, plan: Plan) -> None:
@@ -263,8 +277,18 @@ class Scheduler:
                     break
                 self.waiting.pop(0)
                 length = r.prompt_len + r.generated
-                slots = self.bm.add_seq(seq_id(r.rid, 0), length)
-                plan.prefill.extend((r.rid, 0, p, slots[p]) for p in range(length))
+                if r.tokens is None:
+                    slots = self.bm.add_seq(seq_id(r.rid, 0), length)
+                    plan.prefill.extend((r.rid, 0, p, slots[p]) for p in range(length))
+                else:
+                    slots, cached = self.bm.add_seq_cached(seq_id(r.rid, 0), r.tokens)
+                    plan.cached += cached
+                    plan.prefill.extend((r.rid, 0, p, slots[p])
+                                        for p in range(cached, r.prompt_len))
+                    if r.generated:
+                        gslots, _ = self.bm.append_slots(seq_id(r.rid, 0), r.generated)
+                        plan.prefill.extend((r.rid, 0, r.prompt_len + i, gslots[i])
+                                            for i in range(r.generated))
                 for s in range(1, r.num_samples):
                     self.bm.fork(seq_id(r.rid, 0), seq_id(r.rid, s))
                 r.state = "running"

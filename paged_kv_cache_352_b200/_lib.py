@@ -95,10 +95,13 @@ _SIGS = {
     "pa_bm_host_free_list": (_c_int, [_vp, _vp, _c_int]),
     "pa_bm_add_seq_cached": (_c_int, [_vp, _c_i64, _vp, _c_int, _vp, ctypes.POINTER(_c_int)]),
     "pa_bm_num_cached": (_c_int, [_vp]),
+    "pa_bm_cached_prefix": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(_c_int),
+                                     ctypes.POINTER(_c_int)]),
     "pa_bm_evictable_list": (_c_int, [_vp, _vp, _c_int]),
     "pa_sched_create": (_c_int, [_c_int, _c_int, _vp, _c_int, _c_int, _c_int, ctypes.POINTER(_vp)]),
     "pa_sched_destroy": (None, [_vp]),
     "pa_sched_submit": (_c_int, [_vp, _c_i64, _c_int, _c_int, _c_int, _c_i64]),
+    "pa_sched_submit_tokens": (_c_int, [_vp, _c_i64, _vp, _c_int, _c_int, _c_int, _c_i64]),
     "pa_sched_step": (_c_int, [_vp, _vp]),
     "pa_sched_idle": (_c_int, [_vp]),
     "pa_sched_plan_requests": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
@@ -519,6 +522,14 @@ class BlockManager:
     def num_cached(self) -> int:
         return self._lib.pa_bm_num_cached(self._h)
 
+    def cached_prefix(self, token_ids):
+        """(leading full blocks found in the cache, how many of them are evictable)."""
+        toks = np.ascontiguousarray(np.asarray(list(token_ids), dtype=np.int32))
+        hits, revived = ctypes.c_int(0), ctypes.c_int(0)
+        _check(self._lib.pa_bm_cached_prefix(self._h, toks.ctypes.data if len(toks) else None,
+                                             len(toks), ctypes.byref(hits), ctypes.byref(revived)))
+        return hits.value, revived.value
+
     def evictable_list(self) -> list:
         out = np.empty(max(self.num_blocks, 1), np.int32)
         n = self._lib.pa_bm_evictable_list(self._h, out.ctypes.data, self.num_blocks)
@@ -576,7 +587,8 @@ class SchedPlanCounts(ctypes.Structure):
                 ("num_swap_in", ctypes.c_int), ("num_copies", ctypes.c_int),
                 ("num_prefill", ctypes.c_int), ("num_writes", ctypes.c_int),
                 ("num_seqs", ctypes.c_int), ("max_blocks_per_seq", ctypes.c_int),
-                ("max_context_len", ctypes.c_int), ("total_context", ctypes.c_int64)]
+                ("max_context_len", ctypes.c_int), ("total_context", ctypes.c_int64),
+                ("num_cached_tokens", ctypes.c_int64)]
 
 
 def _p(a):
@@ -622,9 +634,19 @@ class Scheduler:
             pass
 
     def submit(self, request_id: int, prompt_len: int, output_len: int, num_samples: int = 1,
-               arrival: int = 0) -> None:
-        _check(self._lib.pa_sched_submit(self._h, request_id, prompt_len, output_len,
-                                         num_samples, arrival))
+               arrival: int = 0, tokens=None) -> None:
+        """Queue a request; with ``tokens`` (the prompt's token ids) it is admitted
+        through the prefix cache."""
+        if tokens is None:
+            _check(self._lib.pa_sched_submit(self._h, request_id, prompt_len, output_len,
+                                             num_samples, arrival))
+            return
+        toks = np.ascontiguousarray(np.asarray(list(tokens), dtype=np.int32))
+        if len(toks) != prompt_len:
+            raise PAError(PA_ERR_INVALID_ARG, "one token id per prompt position")
+        _check(self._lib.pa_sched_submit_tokens(self._h, request_id,
+                                                toks.ctypes.data if len(toks) else None,
+                                                prompt_len, output_len, num_samples, arrival))
 
     def step(self) -> SchedPlanCounts:
         c = SchedPlanCounts()
@@ -677,6 +699,7 @@ class Scheduler:
             "swap_out": pairs(so), "swap_in": pairs(si), "copies": pairs(cp),
             "prefill": writes[0], "writes": writes[1],
             "batch": list(zip(br.tolist(), bsm.tolist(), ctx.tolist())),
+            "cached": int(c.num_cached_tokens),
             "tables": tables,
         }
 

@@ -38,6 +38,24 @@ namespace {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Physical blocks of the leading full blocks of a prompt found in the cache.
+std::vector<int32_t> cached_prefix_blocks(const pa_bm* bm, const int32_t* token_ids,
+                                          int num_tokens) {
+  const int bs = bm->block_size;
+  std::vector<int32_t> hits;
+  std::vector<int32_t> key(bs + 1);
+  int32_t parent = -1;
+  for (int i = 0; i < num_tokens / bs; ++i) {
+    key[0] = parent;
+    for (int t = 0; t < bs; ++t) key[1 + t] = token_ids[i * bs + t];
+    auto c = bm->cache.find(key);
+    if (c == bm->cache.end()) break;
+    hits.push_back(c->second);
+    parent = c->second;
+  }
+  return hits;
+}
+
 int swapped_error(int64_t seq_id) {
   return fail(PA_ERR_SEQ_SWAPPED, "sequence %lld is swapped out", (long long)seq_id);
 }
@@ -204,17 +222,9 @@ int pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* token_ids, in
     return fail(PA_ERR_SEQ_EXISTS, "sequence %lld exists", (long long)seq_id);
   const int bs = bm->block_size;
   const int full = num_tokens / bs;
-  std::vector<int32_t> hits;
+  std::vector<int32_t> hits = cached_prefix_blocks(bm, token_ids, num_tokens);
   std::vector<int32_t> key(bs + 1);
-  int32_t parent = -1;
-  for (int i = 0; i < full; ++i) {
-    key[0] = parent;
-    for (int t = 0; t < bs; ++t) key[1 + t] = token_ids[i * bs + t];
-    auto c = bm->cache.find(key);
-    if (c == bm->cache.end()) break;
-    hits.push_back(c->second);
-    parent = c->second;
-  }
+  int32_t parent = hits.empty() ? -1 : hits.back();
   const int64_t need = ceil_div(num_tokens, bs) - (int64_t)hits.size();
   int64_t revived = 0;
   for (int32_t b : hits) revived += bm->ref[b] == 0;
@@ -248,6 +258,20 @@ int pa_bm_add_seq_cached(pa_bm* bm, int64_t seq_id, const int32_t* token_ids, in
   for (int64_t p = 0; p < num_tokens; ++p) slots_out[p] = bm->slot(s, p);
   bm->seqs.emplace(seq_id, std::move(s));
   *num_cached_tokens = (int)hits.size() * bs;
+  return PA_OK;
+}
+
+int pa_bm_cached_prefix(const pa_bm* bm, const int32_t* token_ids, int num_tokens,
+                        int* hit_blocks, int* revived_blocks) {
+  pa::clear_error();
+  if (!bm || !hit_blocks || !revived_blocks) return fail(PA_ERR_INVALID_ARG, "null argument");
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0");
+  if (num_tokens > 0 && !token_ids) return fail(PA_ERR_INVALID_ARG, "null token_ids");
+  const std::vector<int32_t> hits = cached_prefix_blocks(bm, token_ids, num_tokens);
+  int revived = 0;
+  for (int32_t b : hits) revived += bm->ref[b] == 0;
+  *hit_blocks = (int)hits.size();
+  *revived_blocks = revived;
   return PA_OK;
 }
 

@@ -36,6 +36,7 @@ struct Request {
   int64_t arrival = 0;
   int64_t order = 0;  // submission index
   int generated = 0;
+  std::vector<int32_t> tokens;  // prompt token ids (admission through the prefix cache)
 };
 
 struct Write {
@@ -55,6 +56,7 @@ struct Plan {
   std::vector<int32_t> batch_sample, batch_ctx, tables;
   int max_blocks = 1;
   int max_ctx = 0;
+  int64_t cached = 0;  // prompt tokens found in the prefix cache
 
   void clear() {
     finished.clear();
@@ -73,6 +75,7 @@ struct Plan {
     tables.clear();
     max_blocks = 1;
     max_ctx = 0;
+    cached = 0;
   }
 };
 
@@ -167,7 +170,10 @@ struct pa_sched {
   int64_t admit_need(const Request& r) const {
     const int64_t len = (int64_t)r.prompt_len + r.generated;
     const int64_t extra = len % block_size == 0 ? r.num_samples : r.num_samples - 1;
-    return ceil_div(len, block_size) + extra;
+    int hits = 0, revived = 0;
+    if (!r.tokens.empty())
+      pa_bm_cached_prefix(bm, r.tokens.data(), r.prompt_len, &hits, &revived);
+    return ceil_div(len, block_size) - hits + revived + extra;
   }
 
   int append(const Request& r) {
@@ -281,8 +287,26 @@ struct pa_sched {
         waiting.erase(waiting.begin());
         const int len = r.prompt_len + r.generated;
         std::vector<int64_t> slots(len);
-        if (int st = pa_bm_add_seq(bm, seq_of(r.id, 0), len, slots.data())) return st;
-        for (int p = 0; p < len; ++p) plan.prefill.push_back({r.id, 0, p, slots[p]});
+        if (r.tokens.empty()) {
+          if (int st = pa_bm_add_seq(bm, seq_of(r.id, 0), len, slots.data())) return st;
+          for (int p = 0; p < len; ++p) plan.prefill.push_back({r.id, 0, p, slots[p]});
+        } else {
+          int cached = 0;
+          if (int st = pa_bm_add_seq_cached(bm, seq_of(r.id, 0), r.tokens.data(), r.prompt_len,
+                                            slots.data(), &cached))
+            return st;
+          plan.cached += cached;
+          for (int p = cached; p < r.prompt_len; ++p) plan.prefill.push_back({r.id, 0, p, slots[p]});
+          if (r.generated) {
+            int64_t cow[2];
+            int n_cow = 0;
+            if (int st = pa_bm_append_slots(bm, seq_of(r.id, 0), r.generated,
+                                            slots.data() + r.prompt_len, cow, &n_cow))
+              return st;
+            for (int i = 0; i < r.generated; ++i)
+              plan.prefill.push_back({r.id, 0, r.prompt_len + i, slots[r.prompt_len + i]});
+          }
+        }
         for (int s = 1; s < r.num_samples; ++s)
           if (int st = pa_bm_fork(bm, seq_of(r.id, 0), seq_of(r.id, s))) return st;
         running.push_back(r.id);
@@ -410,6 +434,19 @@ int pa_sched_submit(pa_sched* s, int64_t request_id, int prompt_len, int output_
   return PA_OK;
 }
 
+int pa_sched_submit_tokens(pa_sched* s, int64_t request_id, const int32_t* prompt_tokens,
+                           int prompt_len, int output_len, int num_samples,
+                           int64_t arrival_step) {
+  if (prompt_len > 0 && !prompt_tokens) {
+    pa::clear_error();
+    return fail(PA_ERR_INVALID_ARG, "null prompt_tokens");
+  }
+  if (int st = pa_sched_submit(s, request_id, prompt_len, output_len, num_samples, arrival_step))
+    return st;
+  s->requests.at(request_id).tokens.assign(prompt_tokens, prompt_tokens + prompt_len);
+  return PA_OK;
+}
+
 int pa_sched_step(pa_sched* s, pa_sched_plan* plan) {
   pa::clear_error();
   if (!s || !plan) return fail(PA_ERR_INVALID_ARG, "null argument");
@@ -435,6 +472,7 @@ int pa_sched_step(pa_sched* s, pa_sched_plan* plan) {
   int64_t total = 0;
   for (int32_t c : p.batch_ctx) total += c;
   plan->total_context = total;
+  plan->num_cached_tokens = p.cached;
   return PA_OK;
 }
 

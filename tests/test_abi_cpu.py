@@ -209,6 +209,7 @@ def test_block_manager_matches_oracle(seed):
             keep = int(rng.integers(0, 65))
             toks = base[:keep] + rng.integers(0, 50, int(rng.integers(0, 40))).tolist()
             args = ("add_seq_cached", nid, toks)
+            assert cbm.cached_prefix(toks) == obm.cached_prefix(toks)
         elif op == 0 or not live:
             n = int(rng.integers(0, 70))
             args = ("add_seq", nid, n)

@@ -30,19 +30,21 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
     c = pa.Scheduler(nb, 16, order, max_num_seqs=cap, num_host_blocks=host, preempt_mode=mode)
     o = SCH.Scheduler(nb, 16, order, max_num_seqs=cap, num_host_blocks=host, preempt_mode=mode)
     for t in trace:
-        c.submit(*t)
-        o.submit(*t)
-    max_ctx = max(p + n for _, p, n, _, _ in trace)
+        toks = t[5] if len(t) > 5 else None
+        c.submit(*t[:5], tokens=toks)
+        o.submit(*t[:5], tokens=toks)
+    max_ctx = max(t[1] + t[2] for t in trace)
     c.attach(hq, hkv, d, tdt, max_ctx, fp8_scales=fp8)
     kc = torch.zeros(nb, hkv, 16, d, dtype=cdt, device="cuda")
     vc = torch.zeros_like(kc)
     hk = torch.zeros(max(host, 1), hkv, 16, d, dtype=cdt).pin_memory() if host else None
     hv = torch.zeros_like(hk).pin_memory() if host else None
-    toks = gen.RequestTokens(seed, {r: p for r, p, *_ in trace}, hkv, d, dt)
+    toks = gen.RequestTokens(seed, {t[0]: t[1] for t in trace}, hkv, d, dt,
+                             prompt_tokens={t[0]: (t[5] if len(t) > 5 else None) for t in trace})
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     scale = 1 / math.sqrt(d)
     G = hq // hkv
-    stats = {"steps": 0, "preempt": 0, "swap": 0, "cow": 0, "seqs": 0}
+    stats = {"steps": 0, "preempt": 0, "swap": 0, "cow": 0, "seqs": 0, "cached": 0}
     while not o.idle():
         c.step()
         op = o.step()
@@ -83,6 +85,7 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
         stats["swap"] += len(op.swap_out) + len(op.swap_in)
         stats["cow"] += len(op.copies)
         stats["seqs"] += len(op.batch)
+        stats["cached"] += op.cached
     assert int(err.item()) == 0
     return stats
 
@@ -129,3 +132,21 @@ def test_recompute_mode_trace_over_fp8_cache_mha():
     st = _run_trace(_trace(12, 24, 1), nb=24, cap=10, host=0, mode=pa.PA_PREEMPT_RECOMPUTE,
                     hq=4, hkv=4, d=64, dt="f16", seed=42, fp8=(0.01, 0.01))
     assert st["preempt"] > 0, st
+
+
+def test_prefix_cached_requests_share_prompt_blocks():
+    """Requests submitted with token ids and sharing system prompts: cached prompt
+    blocks are read, never rewritten, and every step decodes to the oracle's
+    attention over each request's prompt-determined keys and values."""
+    from tests.test_oracle_scheduler import _prompt_trace
+    st = _run_trace(_prompt_trace(23, 24, 3), nb=30, cap=12, host=400, mode=pa.PA_PREEMPT_SWAP,
+                    hq=8, hkv=2, d=128, dt="bf16", seed=44)
+    assert st["cached"] > 0 and st["cow"] > 0, st
+
+
+def test_prefix_cached_recompute_over_fp8_cache():
+    from tests.test_oracle_scheduler import _prompt_trace
+    st = _run_trace(_prompt_trace(24, 24, 1), nb=18, cap=10, host=0,
+                    mode=pa.PA_PREEMPT_RECOMPUTE, hq=4, hkv=4, d=64, dt="f16", seed=45,
+                    fp8=(0.02, 0.02))
+    assert st["cached"] > 0 and st["preempt"] > 0, st

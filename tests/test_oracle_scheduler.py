@@ -91,13 +91,24 @@ def _replay(sched_factory, trace, check_fcfs=True):
     admission, newest-first preemption and internal fragmentation."""
     s = sched_factory()
     bs = s.block_size
-    for rid, p, o, n, a in trace:
-        s.submit(rid, p, o, n, a)
+    prompts = {}
+    for entry in trace:
+        rid, p, o, n, a = entry[:5]
+        toks = entry[5] if len(entry) > 5 else None
+        s.submit(rid, p, o, n, a, tokens=toks)
+        prompts[rid] = toks
+
+    def tag(r, smp, pos):
+        # a prompt token's keys/values depend on its whole prefix: requests that
+        # share a prompt prefix share these tags; everything else is per request
+        if pos < info[r][0] and prompts[r] is not None:
+            return ("prefix", hash(tuple(prompts[r][:pos + 1])))
+        return (r, -1 if pos < info[r][0] else smp, pos)
     dev = {}
     host = {}
-    produced = {rid: 0 for rid, *_ in trace}
-    info = {rid: (p, o, n, a) for rid, p, o, n, a in trace}
-    order = {rid: k for k, (rid, *_) in enumerate(trace)}
+    produced = {e[0]: 0 for e in trace}
+    info = {e[0]: tuple(e[1:5]) for e in trace}
+    order = {e[0]: k for k, e in enumerate(trace)}
     steps = 0
     while not s.idle():
         running_before = [r.rid for r in s.running]
@@ -127,20 +138,19 @@ def _replay(sched_factory, trace, check_fcfs=True):
             for o_ in range(bs):
                 dev[d * bs + o_] = host.get(h * bs + o_)
         for r, smp, pos, slot in pl.prefill:
-            dev[slot] = (r, -1 if pos < info[r][0] else smp, pos)
+            dev[slot] = tag(r, smp, pos)
         for src, dst in pl.copies:
             for o_ in range(bs):
                 dev[dst * bs + o_] = dev.get(src * bs + o_)
         for r, smp, pos, slot in pl.writes:
-            branch = -1 if pos < info[r][0] else smp
-            dev[slot] = (r, branch, pos)
+            dev[slot] = tag(r, smp, pos)
         assert sum(1 for _ in pl.batch) <= s.max_num_seqs
         ids = [SCH.seq_id(r, smp) for r, smp, _ in pl.batch]
         maxb = max([-(-c // bs) for _, _, c in pl.batch], default=1)
         tables = s.bm.block_tables(ids, maxb) if ids else np.zeros((0, 1), np.int32)
         for (r, smp, ctx), row in zip(pl.batch, tables):
             for pos in range(ctx):
-                want = (r, -1 if pos < info[r][0] else smp, pos)
+                want = tag(r, smp, pos)
                 got = dev.get(int(row[pos // bs]) * bs + pos % bs)
                 assert got == want, (pl.step, r, smp, pos, got, want)
         for r, smp, ctx in pl.batch:
@@ -155,7 +165,7 @@ def _replay(sched_factory, trace, check_fcfs=True):
         assert 0 <= alloc - filled < bs * max(nseq, 1)
     for rid, (p, o, n, a) in info.items():
         assert produced[rid] == o, (rid, produced[rid], o)
-    assert s.bm.num_free() == s.bm.num_blocks
+    assert s.bm.num_free() == s.bm.num_blocks   # cached blocks left behind count as free
     return steps
 
 
@@ -183,8 +193,74 @@ def pin_replay_swap_falls_back_to_recompute():
     _replay(lambda: SCH.Scheduler(20, 16, None, max_num_seqs=8, num_host_blocks=6), tr)
 
 
+def _prompt_trace(seed, n_req, max_samples, systems=3, sys_len=(20, 70), own=(0, 30),
+                  out=(1, 30), arrive=40):
+    """Requests whose prompts are one of a few shared system prompts plus tokens of
+    their own, with their token ids."""
+    rng = np.random.default_rng(seed)
+    sys_prompts = [rng.integers(0, 1000, int(rng.integers(*sys_len))).tolist()
+                   for _ in range(systems)]
+    trace = []
+    for i in range(n_req):
+        toks = sys_prompts[int(rng.integers(systems))] + \
+            rng.integers(1000, 2000, int(rng.integers(*own))).tolist()
+        trace.append((i, len(toks), int(rng.integers(*out)), int(rng.integers(1, max_samples + 1)),
+                      int(rng.integers(0, arrive)), toks))
+    return trace
+
+
+def pin_prefix_cache_closed_form():
+    """A second request with the same 100-token prompt shares its 6 full blocks:
+    96 tokens found cached, 4 written; a third with a different third block
+    shares only the first 2 blocks."""
+    prompt = list(range(500, 600))
+    other = prompt[:32] + [7] * 16 + prompt[48:]
+    s = SCH.Scheduler(64, 16, max_num_seqs=8)
+    s.submit(0, 100, 5, 1, 0, tokens=prompt)
+    s.submit(1, 100, 5, 1, 2, tokens=prompt)
+    s.submit(2, 100, 5, 1, 3, tokens=other)
+    plans = _run(s)
+    adm = {r: pl for pl in plans for r in pl.admitted}
+    assert adm[0].cached == 0 and len(adm[0].prefill) == 100
+    assert adm[1].cached == 96 and [p for _, _, p, _ in adm[1].prefill] == [96, 97, 98, 99]
+    assert adm[2].cached == 32 and len(adm[2].prefill) == 68
+    t0 = SCH.seq_id(0, 0)
+    assert t0 not in s.bm._tables          # finished and freed, blocks left cached
+    assert s.bm.num_cached() > 0 and s.bm.num_free() == 64
+
+
+def pin_prefix_cache_recompute_hits_own_blocks():
+    """A request dropped for recomputation finds its own prompt blocks still cached
+    when it is admitted again: only the partial block and its generated tokens
+    are written again."""
+    prompt = list(range(40))                       # 2 full blocks + 8 tokens
+    s = SCH.Scheduler(6, 16, max_num_seqs=4, preempt_mode=SCH.PREEMPT_RECOMPUTE)
+    s.submit(0, 40, 40, 1, 0, tokens=prompt)       # grows to 80 tokens: 5 blocks
+    s.submit(1, 30, 30, 1, 0)                      # uncached; preempted when short
+    plans = _run(s)
+    rec = [(pl.step, r) for pl in plans for r, m in pl.preempted if m == SCH.PREEMPT_RECOMPUTE]
+    assert rec, "the trace must preempt"
+    readmits = [pl for pl in plans for r in pl.admitted if r == 0 and pl.step > 0]
+    for pl in readmits:
+        assert pl.cached == 32 and min(p for r, _, p, _ in pl.prefill if r == 0) == 32
+
+
+def pin_replay_prefix_cache_swap_mode():
+    _replay(lambda: SCH.Scheduler(30, 16, np.random.default_rng(3).permutation(30),
+                                  max_num_seqs=12, num_host_blocks=400),
+            _prompt_trace(21, 30, 3), check_fcfs=True)
+
+
+def pin_replay_prefix_cache_recompute_mode():
+    _replay(lambda: SCH.Scheduler(18, 16, np.random.default_rng(4).permutation(18),
+                                  max_num_seqs=10, preempt_mode=SCH.PREEMPT_RECOMPUTE),
+            _prompt_trace(22, 30, 1), check_fcfs=True)
+
+
 PINS = [pin_pages_example, pin_unconstrained_closed_form, pin_batch_cap_waves,
-        pin_replay_swap_mode, pin_replay_recompute_mode, pin_replay_swap_falls_back_to_recompute]
+        pin_replay_swap_mode, pin_replay_recompute_mode, pin_replay_swap_falls_back_to_recompute,
+        pin_prefix_cache_closed_form, pin_prefix_cache_recompute_hits_own_blocks,
+        pin_replay_prefix_cache_swap_mode, pin_replay_prefix_cache_recompute_mode]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -254,6 +330,14 @@ def _mutant(method: str, old: str, new: str):
 # the batch cap on resume (nothing is admitted while a request is swapped out,
 # so resumed requests fit the cap they fitted before).
 MISTAKES = {
+    "prefix_cache_ignored": (
+        "step", "if r.tokens is None:\n                slots = self.bm.add_seq",
+        "if True:\n                slots = self.bm.add_seq", False),
+    "admit_need_ignores_revived": (
+        "_admit_need", "- hits + revived + extra", "- hits + extra", False),
+    "recompute_rewrites_whole_prompt": (
+        "step", "for p in range(cached, r.prompt_len))",
+        "for p in range(0, r.prompt_len))", False),
     "admission_newest_first": (
         "_insert_by_arrival", "queue.insert(i, r)", "queue.insert(0, r)", True),
     "admit_need_ignores_samples": (

@@ -20,8 +20,9 @@ def _pair(nb, order, cap, host, mode):
 
 def _compare_run(c, o, trace):
     for t in trace:
-        c.submit(*t)
-        o.submit(*t)
+        toks = t[5] if len(t) > 5 else None
+        c.submit(*t[:5], tokens=toks)
+        o.submit(*t[:5], tokens=toks)
     steps = 0
     stats = {"preempt": 0, "swap_in": 0, "cow": 0, "prefill": 0}
     while not o.idle():
@@ -30,6 +31,7 @@ def _compare_run(c, o, trace):
         op = o.step()
         cp = c.plan()
         assert cp["step"] == op.step
+        assert cp["cached"] == op.cached
         for f in ("finished", "preempted", "resumed", "admitted", "swap_out", "swap_in",
                   "copies", "prefill", "writes", "batch"):
             got = [tuple(x) if isinstance(x, (tuple, list)) else x for x in cp[f]]
@@ -147,3 +149,22 @@ def test_execute_requires_attach_and_a_plan():
     st = c._lib.pa_sched_execute(c._h, None, None, None, None, None, None, None, None, None,
                                  None, 1.0, None, None)
     assert st == pa._lib.PA_ERR_INVALID_ARG and "no executor attached" in pa.last_error()
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefix_cached_requests_match_oracle(seed):
+    from tests.test_oracle_scheduler import _prompt_trace
+    mode = pa.PA_PREEMPT_SWAP if seed % 2 == 0 else pa.PA_PREEMPT_RECOMPUTE
+    host = 400 if mode == pa.PA_PREEMPT_SWAP else 0
+    samples = 3 if mode == pa.PA_PREEMPT_SWAP else 1
+    nb = 26 + 4 * seed
+    c, o = _pair(nb, np.random.default_rng(seed).permutation(nb), 10, host, mode)
+    trace = _prompt_trace(400 + seed, 30, samples)
+    _compare_run(c, o, trace)
+    assert c.bm.num_cached() == o.bm.num_cached() > 0
+
+
+def test_submit_tokens_checks_length():
+    c = pa.Scheduler(8, 16)
+    with pytest.raises(pa.PAError):
+        c.submit(0, 5, 3, tokens=[1, 2, 3])

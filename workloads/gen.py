@@ -14,6 +14,7 @@ on sampled outputs.
 from __future__ import annotations
 
 from concurrent.futures import ThreadPoolExecutor
+import hashlib
 import os
 
 import numpy as np
@@ -25,6 +26,7 @@ STREAM_OWN_KV = 3      # per-sample tokens appended after a fork (shared-prefix 
 STREAM_META = 4        # context lengths and block placement
 STREAM_REQUEST_KV = 5  # request traces: one key/value row per (request, branch, position)
 STREAM_STEP_QUERY = 6  # request traces: one query per (request, sample, step)
+STREAM_PREFIX_KV = 7   # request traces with token ids: one key/value row per prompt prefix
 
 _DTYPES = ("f16", "bf16")
 
@@ -118,17 +120,40 @@ def step_query_bits(seed: int, request: int, sample: int, step: int, num_q_heads
                        (num_q_heads, head_dim), dtype)
 
 
+def prefix_keys(tokens) -> list:
+    """A 64-bit key per prompt position identifying the whole prefix up to it (a
+    chained BLAKE2b): two prompts share a position's key exactly when they share
+    every token up to it, as a model's keys and values would."""
+    keys, h = [], b""
+    for t in tokens:
+        h = hashlib.blake2b(h + int(t).to_bytes(4, "little", signed=True), digest_size=8).digest()
+        keys.append(int.from_bytes(h, "little"))
+    return keys
+
+
 class RequestTokens:
     """Memoised token rows of a request trace: position ``p`` of sample ``s`` of
-    request ``r`` is a prompt row when ``p < prompt_len[r]``, else sample ``s``'s own."""
+    request ``r`` is a prompt row when ``p < prompt_len[r]``, else sample ``s``'s own.
+    A request given its prompt token ids (``prompt_tokens[r]``) draws its prompt
+    rows by prefix key, so requests sharing a prompt prefix share those rows."""
 
     def __init__(self, seed: int, prompt_len: dict, num_kv_heads: int, head_dim: int,
-                 dtype: str):
+                 dtype: str, prompt_tokens: dict = None):
         self.seed, self.prompt_len = seed, prompt_len
         self.hkv, self.d, self.dtype = num_kv_heads, head_dim, dtype
         self._rows = {}
+        self._keys = {r: prefix_keys(t) for r, t in (prompt_tokens or {}).items()
+                      if t is not None}
 
     def row(self, request: int, sample: int, position: int):
+        if position < self.prompt_len[request] and request in self._keys:
+            k = self._keys[request][position]
+            key = ("prefix", k)
+            if key not in self._rows:
+                b = normal_bits([self.seed, STREAM_PREFIX_KV, k >> 32, k & 0xffffffff, position],
+                                (2, self.hkv, self.d), self.dtype)
+                self._rows[key] = (b[0], b[1])
+            return self._rows[key]
         branch = 0 if position < self.prompt_len[request] else 1 + sample
         key = (request, branch, position)
         if key not in self._rows:
