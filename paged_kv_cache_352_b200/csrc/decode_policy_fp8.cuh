@@ -211,13 +211,15 @@ struct Fp8TensorPolicy {
         vr[mm][1] = v.y;
       }
     }
-    // rows past the context may hold any codes (NaN included): clear their bytes
-    uint32_t keep = 0xffffffffu;
+    // rows past the context may hold any codes (NaN included): clear them. Only a
+    // sequence's last block is partly filled, and the test is uniform across the warp.
     if (valid < kBS) {
-      keep = 0u;
 #pragma unroll
       for (int mm = 0; mm < 4; ++mm)
-        if (j + 4 * mm < valid) keep |= 0xffu << (8 * mm);
+        if (j + 4 * mm >= valid) {
+#pragma unroll
+          for (int w = 0; w < VW; ++w) vr[mm][w] = 0u;
+        }
     }
 #pragma unroll
     for (int w = 0; w < VW; ++w) {
@@ -226,8 +228,8 @@ struct Fp8TensorPolicy {
       const uint32_t t1 = __byte_perm(vr[0][w], vr[1][w], 0x7362);
       const uint32_t t2 = __byte_perm(vr[2][w], vr[3][w], 0x5140);
       const uint32_t t3 = __byte_perm(vr[2][w], vr[3][w], 0x7362);
-      const uint32_t y[4] = {__byte_perm(t0, t2, 0x5410) & keep, __byte_perm(t0, t2, 0x7632) & keep,
-                             __byte_perm(t1, t3, 0x5410) & keep, __byte_perm(t1, t3, 0x7632) & keep};
+      const uint32_t y[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
+                             __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632)};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int nt = 4 * w + i;
