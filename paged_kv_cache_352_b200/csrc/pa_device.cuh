@@ -170,24 +170,6 @@ struct CacheElem<E4M3> {
   }
 };
 
-// Two E4M3 codes to the 16-bit pair of type T (exact for both half and bfloat16).
-template <typename T>
-__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t pair16);
-
-template <>
-__device__ __forceinline__ uint32_t e4m3x2_to<__half>(uint32_t pair16) {
-  return e4m3x2_to_half2_bits(pair16);
-}
-
-template <>
-__device__ __forceinline__ uint32_t e4m3x2_to<__nv_bfloat16>(uint32_t pair16) {
-  const float2 x = half2_bits_to_float2(e4m3x2_to_half2_bits(pair16));
-  const __nv_bfloat162 b = __floats2bfloat162_rn(x.x, x.y);
-  uint32_t r;
-  memcpy(&r, &b, sizeof(r));
-  return r;
-}
-
 // Two floats to two E4M3 codes (`lo` in the low byte), nearest even, saturating.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return static_cast<uint32_t>(
