@@ -102,9 +102,14 @@ int default_partition_blocks(int num_seqs, int num_kv_heads, int max_blocks, boo
 }
 
 // One warp per partition (plus a merge launch) pays off only for short partitions
-// and only while its grid, WARPS = 4 times smaller, still fills the GPU: the
-// library's own short partitions arise for small batches, which keep one CTA
-// per partition.
+// of long sequences, and only while its grid, WARPS = 4 times smaller, still
+// fills the GPU. A CTA takes four consecutive partitions of one sequence, so a
+// sequence with fewer partitions leaves warps idle: measured on 256 lognormal
+// contexts (median ~660 tokens) at 1024-token partitions, warp mode took 2.2x
+// the time of one CTA per partition. The library's own short partitions arise
+// for small batches, which keep one CTA per partition.
+constexpr int kWarpPartMinParts = 16;
+
 bool use_warp_parts(int num_seqs, int num_kv_heads, int part_blocks, int max_parts) {
   static const int forced = [] {
     const char* e = getenv("PA_DECODE_SPLIT");
@@ -115,7 +120,8 @@ bool use_warp_parts(int num_seqs, int num_kv_heads, int part_blocks, int max_par
   if (max_parts <= 1) return false;
   if (forced >= 0) return forced == 1;
   const long long ctas = (long long)num_kv_heads * num_seqs * ((max_parts + 3) / 4);
-  return part_blocks <= kWarpPartMaxBlocks && ctas >= kSplitTargetUnits;
+  return part_blocks <= kWarpPartMaxBlocks && max_parts >= kWarpPartMinParts &&
+         ctas >= kSplitTargetUnits;
 }
 
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,

@@ -52,8 +52,9 @@ struct DecodeArgs {
   int warp_parts;    // split mode: one warp per partition + a merge launch (else one CTA)
 };
 
-// Split partitions of at most this many blocks run one warp per partition when
-// that grid still has kSplitTargetUnits CTAs (PA_DECODE_SPLIT=cta|warp forces a mode).
+// Split partitions of at most this many blocks, for batches whose longest
+// context spans at least 16 of them, run one warp per partition when that grid
+// still has kSplitTargetUnits CTAs (PA_DECODE_SPLIT=cta|warp forces a mode).
 constexpr int kWarpPartMaxBlocks = 64;
 bool use_warp_parts(int num_seqs, int num_kv_heads, int part_blocks, int max_parts);
 

@@ -332,6 +332,8 @@ def test_decode_plan_split_modes():
     assert L.pa_paged_decode_plan(1, 64, 8, 128, 32768, 512, ordered=True) == (32, 64, 1)
     # long partitions stay one CTA per partition
     assert L.pa_paged_decode_plan(8, 64, 8, 128, 131072, 2048, ordered=True)[2] == 1
+    # short partitions of short sequences (few partitions each) too
+    assert L.pa_paged_decode_plan(256, 32, 8, 128, 4096, 1024, ordered=True) == (64, 4, 1)
     # no split at all, and an empty batch
     assert L.pa_paged_decode_plan(64, 32, 32, 128, 2048, 0, ordered=True) == (128, 1, 1)
     assert L.pa_paged_decode_plan(0, 32, 32, 128, 2048, 0)[2] == 0
