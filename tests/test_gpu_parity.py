@@ -14,7 +14,6 @@ import pytest
 import torch
 
 from oracle import step as OS
-from oracle.fpbits import bits_to_f64
 import paged_kv_cache_352_b200 as pa
 from paged_kv_cache_352_b200.runner import DecodeRunner
 from tests.parity import assert_close, out_to_f64, tensor_bits
