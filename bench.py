@@ -12,7 +12,9 @@ step; % of measured HBM peak alongside) and decode tokens/s.
 
 Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events
 on the launching stream; a barrier + synchronize on both sides of the timed
-region; max over ranks. Workloads whose inputs exceed 4x the 126 MB L2 run
+region; max over ranks. Every 32 steps a GPU spin (outside the events) keeps
+the stream busy while the host enqueues them, so the steps run back to back
+and the events measure device time rather than host issue gaps. Workloads whose inputs exceed 4x the 126 MB L2 run
 without a flush (a cyclic scan larger than the cache reuses nothing); smaller
 ones flush L2 between steps, outside the events, by reading a 256 MiB buffer
 (a write flush would leave dirty lines whose write-back the next kernel pays).
@@ -583,6 +585,19 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     }
 
 
+HOLD_EVERY = 32           # timed launches queued behind one hold
+HOLD_PER_STEP_S = 150e-6  # generous host time to enqueue one timed step
+
+
+def gpu_hold(seconds: float) -> None:
+    """Keep the current stream busy (a spin of about ``seconds`` at <= 2 GHz) while
+    the host enqueues the next timed launches, so that they run back to back and
+    CUDA events measure device time, not gaps while the host issues the next
+    launch. Placed outside every pair of timing events."""
+    import torch
+    torch.cuda._sleep(int(seconds * 2.0e9))
+
+
 def fp8_decode_bytes(wl) -> int:
     """Algorithmic bytes of one decode over an E4M3 cache: one byte per cached K
     and V element, 16-bit q and out, the used block-table entries and lengths."""
@@ -623,7 +638,9 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
     torch.cuda.synchronize(device)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(iters)]
-    for a, b in ev:
+    for i, (a, b) in enumerate(ev):
+        if i % HOLD_EVERY == 0:
+            gpu_hold(HOLD_EVERY * HOLD_PER_STEP_S)
         l2_flush()
         a.record(stream)
         launch()
@@ -737,6 +754,8 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     with ClockSampler(device) as clocks:
         for k in range(K):
+            if k % HOLD_EVERY == 0:
+                gpu_hold(HOLD_EVERY * HOLD_PER_STEP_S)
             l2_flush()
             ev[k][0].record(stream)
             r.copy_blocks()
@@ -752,6 +771,27 @@ def run_ours(args):
     dec_s = _max_over_ranks(float(t_dec.mean()), world, device)
     if r.error_bits():
         raise RuntimeError(f"device error bits {r.error_bits()} during timing")
+    decode_ms = {"mean": round(1e3 * float(t_dec.mean()), 4),
+                 "median": round(1e3 * float(np.median(t_dec)), 4),
+                 "min": round(1e3 * float(t_dec.min()), 4)}
+    # the step's cache writes (copy-on-write copies + new tokens) before the decode
+    cache_write_ms = round(1e3 * float((t_step - t_dec).mean()), 4)
+    copy_blocks = None
+    if len(r.cow_pairs) > 0 and world == 1:
+        # copy-on-write copies alone (idempotent: each pair copies the same source)
+        ca, cb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gpu_hold(20 * HOLD_PER_STEP_S)
+        ca.record(stream)
+        for _ in range(20):
+            r.copy_blocks()
+        cb.record(stream)
+        torch.cuda.synchronize(device)
+        tc = ca.elapsed_time(cb) / 20 / 1e3
+        nbytes = len(r.cow_pairs) * 2 * 2 * wl.num_kv_heads * 16 * wl.head_dim * wl.elem_bytes
+        copy_blocks = {"pairs": len(r.cow_pairs), "ms": round(tc * 1e3, 4),
+                       "bytes": nbytes, "gbs": round(nbytes / tc / 1e9, 1),
+                       "what": "pa_copy_blocks of the step's copy-on-write pairs (K and V, "
+                               "read + write), CUDA events around 20 back-to-back launches"}
 
     # e2e: the same step fed from pinned host buffers, result read back to the
     # host, with the next step's input copy overlapping this step's kernels
@@ -821,6 +861,7 @@ def run_ours(args):
         "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
         "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
         "read_stream_ref_gbs": round(read_ref, 1) if read_ref else None,
+        "decode_ms": decode_ms, "cache_write_ms": cache_write_ms, "copy_blocks": copy_blocks,
         "decode_tokens_per_s": round(world * wl.num_seqs / step_s, 1),
         "decode_only_tokens_per_s": round(world * wl.num_seqs / dec_s, 1),
         "bytes_per_step": sb,

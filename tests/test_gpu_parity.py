@@ -344,3 +344,27 @@ def test_host_pipeline_returns_each_steps_output():
     for o in outs[-2:]:
         assert torch.equal(o.view(torch.int16), ref.cpu().view(torch.int16))
     assert hp.h2d_bytes >= (r.q.numel() + r.step_k.numel() + r.step_v.numel()) * 2
+
+
+@pytest.mark.parametrize("name", ["mha_7b_fp16", "gqa_32_8_bf16", "long_ctx_split_kv"])
+@pytest.mark.parametrize("factor", [8.0, 32.0])
+def test_peaked_softmax(name, factor):
+    """N(0,1) queries and keys give nearly flat weights, which an absolute
+    tolerance passes too easily. Queries scaled by 8 and 32 (exact in 16-bit
+    floats) make the weights peaked: one or a few tokens dominate, and every
+    rescale of the online softmax and every split-KV merge shows up in the
+    output. Unsplit and split (64-token partitions) decodes against the oracle."""
+    from oracle.attention import paged_decode
+    wl = workloads.workload(name, small=True)
+    r = DecodeRunner(wl)
+    r.step()
+    _sync()
+    r.q = (r.q.float() * factor).to(r.q.dtype)
+    ref = paged_decode(tensor_bits(r.q), tensor_bits(r.k_cache), tensor_bits(r.v_cache),
+                       r.block_tables_host, r.context_lens_host, wl.scale, wl.dtype)
+    for pt in (0, 64):
+        out = torch.empty_like(r.out)
+        r.decode(out, partition_tokens=pt)
+        _sync()
+        assert_close(out_to_f64(out, wl.dtype), ref, f"{name} q x{factor} partition {pt}")
+    assert r.error_bits() == 0
