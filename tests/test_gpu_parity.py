@@ -368,3 +368,34 @@ def test_peaked_softmax(name, factor):
         _sync()
         assert_close(out_to_f64(out, wl.dtype), ref, f"{name} q x{factor} partition {pt}")
     assert r.error_bits() == 0
+
+
+@pytest.mark.parametrize("name", ["mha_7b_fp16", "gqa_32_8_bf16", "long_ctx_split_kv"])
+def test_planted_key(name):
+    """One key per (sequence, KV head) replaced by 4 x the group's first query
+    head: that token's logit is about 4 |q|^2 / sqrt(d) ~ 45 above the rest, so
+    its weight is ~1 and the output is ~its value row, wherever in the context
+    (first token, a block boundary, the last token, a random position) it sits.
+    A kernel that loses a token, a block or a partition misses it by O(1)."""
+    from oracle.attention import paged_decode
+    wl = workloads.workload(name, small=True)
+    r = DecodeRunner(wl)
+    r.step()
+    _sync()
+    g = wl.num_q_heads // wl.num_kv_heads
+    rng = np.random.default_rng(wl.seed + 77)
+    tables = r.block_tables_host
+    for s, c in enumerate(r.context_lens_host.tolist()):
+        t = int([0, min(16, c - 1), c - 1, rng.integers(0, c)][s % 4])
+        blk, off = int(tables[s][t // 16]), t % 16
+        for h in range(wl.num_kv_heads):
+            r.k_cache[blk, h, off] = (r.q[s, h * g].float() * 4.0).to(r.k_cache.dtype)
+    _sync()
+    ref = paged_decode(tensor_bits(r.q), tensor_bits(r.k_cache), tensor_bits(r.v_cache),
+                       tables, r.context_lens_host, wl.scale, wl.dtype)
+    for pt in (0, 64):
+        out = torch.empty_like(r.out)
+        r.decode(out, partition_tokens=pt)
+        _sync()
+        assert_close(out_to_f64(out, wl.dtype), ref, f"{name} planted key, partition {pt}")
+    assert r.error_bits() == 0
