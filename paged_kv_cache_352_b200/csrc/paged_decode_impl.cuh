@@ -24,14 +24,15 @@ namespace pa {
 namespace {
 
 // Register budget hint: each policy names the resident CTAs per SM its kernels
-// are compiled for (launch bounds), hence the registers a thread may use.
-template <class P, int G>
+// are compiled for (launch bounds) with 4-warp CTAs, hence the registers a
+// thread may use; other CTA sizes keep the same resident threads per SM.
+template <class P, int WARPS>
 constexpr int min_ctas_hint() {
-  return P::kMinCtasPerSm;
+  return P::kMinCtasPerSm * 4 / WARPS > 0 ? P::kMinCtasPerSm * 4 / WARPS : 1;
 }
 
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
+__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
     paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v) {
   constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
 // one CTA per partition, each pipeline ramp and state write is amortised over
 // WARPS times more blocks, and no CTA-wide merge runs per partition.
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, G>()))
+__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
     paged_decode_warp_parts_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                                    const __grid_constant__ CUtensorMap tm_v) {
   constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
@@ -423,10 +424,10 @@ bool use_tensor_path(int group) {
   return group >= 4;
 }
 
-// Over E4M3 caches the CUDA-core path pays ~12 conversion instructions per 8
-// elements on top of its FMAs, while the tensor path converts each code pair
-// once, straight into its mma fragment; PA_DECODE_PATH overrides the choice here
-// too (for any group).
+// Over E4M3 caches 4 and 8 query heads per KV head run on tensor cores, which
+// take each converted code pair straight into an mma fragment; 1 and 2 run on
+// CUDA cores (Fp8CudaCorePolicy). PA_DECODE_PATH overrides the choice here too
+// (for any group).
 bool use_tensor_path_e4m3(int group) {
   static const int forced = [] {
     const char* e = getenv("PA_DECODE_PATH");
@@ -443,10 +444,17 @@ cudaError_t launch_g(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   if constexpr (std::is_same<C, E4M3>::value) {
     if (use_tensor_path_e4m3(G))
       return launch_tiles<Fp8TensorPolicy<T, D, G>, T, D, G>(a, dtype, stream);
+    if constexpr (G <= 2) {
+      return launch_tiles<Fp8CudaCorePolicy<T, D, G>, T, D, G>(a, dtype, stream);
+    } else {
+      // 4 and 8 query heads reach the CUDA cores only when PA_DECODE_PATH
+      // forces them; the generic policy keeps their register use lower
+      return launch_tiles<CudaCorePolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
+    }
   } else {
     if (use_tensor_path(G)) return launch_tiles<TensorPolicy<T, D, G>, T, D, G>(a, dtype, stream);
+    return launch_tiles<CudaCorePolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
   }
-  return launch_tiles<CudaCorePolicy<T, D, G, C>, T, D, G>(a, dtype, stream);
 }
 
 template <typename T, int D, typename C>
