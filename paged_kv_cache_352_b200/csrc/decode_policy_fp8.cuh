@@ -67,10 +67,10 @@ struct Fp8TensorPolicy {
   static constexpr bool kTensorCores = true;
   static constexpr bool kTma2D = kSwizzled;
   static constexpr bool kFp8Cache = true;
-  // Four CTAs (16 warps) per SM: the code conversions make this path issue-
-  // rather than memory-latency-limited, and the extra warps hide their latency
-  // (measured 4 % faster at 8 query heads per KV head than three CTAs).
-  static constexpr int kMinCtasPerSm = 4;
+  // Three CTAs per SM (168 registers; the one-warp-per-partition kernels keep
+  // everything in registers). Four CTAs (128 registers) spilled 90-180 bytes a
+  // thread and measured 10 % slower at 4 query heads per KV head and 7 % at 8.
+  static constexpr int kMinCtasPerSm = 3;
   static_assert(D == 64 || D == 128, "unsupported head_dim");
 
   int g, j;

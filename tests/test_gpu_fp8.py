@@ -107,6 +107,37 @@ def test_decode_fp8_matches_oracle(hq, hkv, d, dt, partition_tokens):
         assert_close(got[s], want[s], f"seq {s} ctx {ctx[s]}")
 
 
+@pytest.mark.parametrize("hq,hkv", [(8, 4), (16, 4)])
+def test_decode_fp8_bf16_queries_beyond_half_range(hq, hkv):
+    """bf16 query rows whose largest magnitude is far above 2^15 (N(0,1) times
+    2^16, exact in bf16) with the softmax scale shrunk by 2^-16: both 8-bit paths
+    (2 query heads per KV head on CUDA cores, 4 on tensor cores) hold the query
+    in half precision and must bring such rows into range by a power of two. The
+    logits equal those of the unscaled queries, so the oracle's values are of
+    ordinary size."""
+    B, nb, d, dt = 5, 160, 128, "bf16"
+    ctx, tables, kc8, vc8, q = _case(917 + hq, B, hq, hkv, d, dt, 300, nb)
+    qf = torch.from_numpy(np.ascontiguousarray(q).view(np.int16)).view(torch.bfloat16).float()
+    big = (qf * 65536.0).to(torch.bfloat16)
+    assert float(big.float().abs().amax(dim=-1).min()) >= 32768.0
+    q_big = big.view(torch.int16).numpy().view(np.uint16)
+    ks, vs = 0.05, 0.02
+    scale = 1 / math.sqrt(d) / 65536.0
+    want = F.paged_decode_fp8(q_big, kc8, vc8, tables, ctx, scale, ks, vs, dt)
+    out = torch.empty(B, hq, d, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = pa.decode_workspace(B, hq, hkv, d, int(ctx.max()), 0)
+    pa.pa_paged_decode_fp8(out, big.cuda(), torch.from_numpy(kc8).cuda(),
+                           torch.from_numpy(vc8).cuda(), torch.from_numpy(tables).cuda(),
+                           torch.from_numpy(ctx).cuda(), int(ctx.max()), scale, ks, vs,
+                           workspace=ws, dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    got = out_to_f64(out, dt)
+    for s in range(B):
+        assert_close(got[s], want[s], f"seq {s} ctx {ctx[s]}")
+
+
 def test_quantize_then_decode_end_to_end():
     """Keys/values written by the fp8 cache write, then decoded, against the oracle's
     write and decode of the same 16-bit inputs; also the quantization error of the
