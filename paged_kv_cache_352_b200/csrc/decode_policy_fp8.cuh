@@ -337,7 +337,8 @@ struct Fp8CudaCorePolicy {
   static constexpr bool kTensorCores = false;
   static constexpr bool kTma2D = false;
   static constexpr bool kFp8Cache = true;
-  static constexpr int kMinCtasPerSm = G > 2 ? 1 : 4;
+  static constexpr int kMinCtasPerSm = 4;  // at most 128 registers a thread
+  static_assert(G <= 2, "4 and 8 query heads per KV head use another policy");
   static_assert(D == 64 || D == 128, "unsupported head_dim");
   static_assert(LPT * TPW == 32 && TPL * TPW == kBS, "unsupported head_dim");
 
