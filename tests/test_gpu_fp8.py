@@ -82,6 +82,8 @@ def _case(seed, B, hq, hkv, d, dt, max_ctx, nb, nan_fill=True):
 
 
 @pytest.mark.parametrize("hq,hkv,d,dt", [(4, 4, 64, "f16"), (8, 4, 128, "bf16"),
+                                          (6, 6, 128, "bf16"), (8, 4, 64, "bf16"),
+                                          (6, 3, 128, "f16"),
                                           (16, 4, 128, "bf16"), (16, 2, 64, "f16"),
                                           (32, 4, 128, "f16")])
 @pytest.mark.parametrize("partition_tokens", [0, 64])
