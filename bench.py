@@ -222,25 +222,28 @@ def _peaks():
 
 DECODE_SOURCES = ("paged_decode_impl.cuh", "decode_policies.cuh", "decode_common.cuh",
                   "pa_device.cuh")
+# a cascade figure (":cascade" entries) also depends on the cascade's own kernels
+CASCADE_SOURCES = DECODE_SOURCES + ("cascade.cu",)
 
 
-def decode_source_sha() -> str:
+def decode_source_sha(sources=DECODE_SOURCES) -> str:
     """Hash of the decode kernel's sources (ties a traffic figure to the code profiled)."""
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "paged_kv_cache_352_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def _traffic_for(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    """DRAM bytes per decode call from the committed ncu summary, if it was taken
     on the current kernel sources for this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(workload)
-        sha = decode_source_sha()
+        sha = decode_source_sha(CASCADE_SOURCES if workload.endswith(":cascade")
+                                else DECODE_SOURCES)
     except (OSError, ValueError, AttributeError):
         return None
     if not rec or rec.get("source_sha") != sha:
@@ -788,7 +791,7 @@ def run_ours(args):
             r.copy_blocks()
             r.reshape_and_cache()
             ev[k][1].record(stream)
-            r.decode()
+            r.decode_step()
             ev[k][2].record(stream)
         torch.cuda.synchronize(device)
     _barrier(world)
@@ -819,6 +822,23 @@ def run_ours(args):
                        "bytes": nbytes, "gbs": round(nbytes / tc / 1e9, 1),
                        "what": "pa_copy_blocks of the step's copy-on-write pairs (K and V, "
                                "read + write), CUDA events around 20 back-to-back launches"}
+
+    plain_decode = None
+    if r.groups is not None and world == 1:
+        # the same batch through pa_paged_decode, which reads shared blocks per sequence
+        pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(20)]
+        gpu_hold(20 * HOLD_PER_STEP_S)
+        for a_, b_ in pe:
+            l2_flush()
+            a_.record(stream)
+            r.decode()
+            b_.record(stream)
+        torch.cuda.synchronize(device)
+        tp = float(np.mean([a_.elapsed_time(b_) for a_, b_ in pe])) / 1e3
+        plain_decode = {"ms": round(tp * 1e3, 4), "cascade_speedup": round(tp / dec_s, 3),
+                        "what": "pa_paged_decode of the same batch (every sequence reads its "
+                                "shared blocks itself), CUDA events, mean of 20"}
 
     # e2e: the same step fed from pinned host buffers, result read back to the
     # host, with the next step's input copy overlapping this step's kernels
@@ -858,9 +878,22 @@ def run_ours(args):
 
     sb = step_bytes(wl, r)
     db = decode_bytes(wl)
+    effective = None
+    kernel = "paged_decode_kernel"
+    if r.groups is not None:
+        # Sequences share blocks: the bytes that must leave HBM are those of the
+        # distinct blocks read; the logical rate is reported beside them.
+        ub = unique_decode_bytes(wl, r)
+        effective = {"decode_gbs_logical": round(db / dec_s / 1e9, 2),
+                     "step_gbs_logical": round(world * sb / step_s / 1e9, 2),
+                     "logical_decode_bytes": db, "unique_decode_bytes": ub}
+        sb = sb - db + ub
+        db = ub
+        kernel = ("pa_paged_decode_cascade: cascade_prepare_kernel, paged_decode_kernel over "
+                  "the groups' shared blocks and over the own blocks, cascade_merge_kernel")
     value = world * sb / step_s / 1e9
     achieved = db / dec_s / 1e9
-    traffic = _traffic_for(wl.name)
+    traffic = _traffic_for(wl.name + (":cascade" if r.groups is not None else ""))
     read_ref = read_stream_gbs(device) if world == 1 else None
     csum = clocks.summary()
     launches_per_step = r.launches_per_step()
@@ -892,7 +925,8 @@ def run_ours(args):
         "decode_tokens_per_s": round(world * wl.num_seqs / step_s, 1),
         "decode_only_tokens_per_s": round(world * wl.num_seqs / dec_s, 1),
         "bytes_per_step": sb,
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel",
+        "shared_blocks": effective, "plain_decode": plain_decode,
+        "roofline": {"bound": "hbm", "kernel": kernel,
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": db,

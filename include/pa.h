@@ -70,6 +70,11 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 #define PA_DEVERR_CONTEXT_RANGE 4 /* context_lens[s] < 0, > max_blocks_per_seq*block_size,
                                      or > max_context_len: sequence skipped (zero output) */
 #define PA_DEVERR_WAIT_TIMEOUT 8  /* a bounded on-chip wait gave up: output invalid */
+#define PA_DEVERR_GROUP 16        /* a cascade group descriptor was rejected (a member that
+                                     does not hold the group's prefix blocks, an id out of
+                                     range, a member claimed twice): that group's members
+                                     were decoded without the shared prefix; outputs stay
+                                     correct */
 
 /* Message for the last failed call on this thread ("" if none). */
 const char* pa_last_error(void);
@@ -298,11 +303,77 @@ int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache, const
                             int dtype, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_paged_decode_cascade — paged decode that reads blocks shared by several
+ * sequences once.
+ *
+ * Forks of one prompt hold the same physical blocks for the prompt's full
+ * blocks ("PagedAttention and Continuous Batching", "Pages, from operating
+ * systems": copy-on-write sharing; "PagedAttention: The vLLM Paper",
+ * "Implementation Essentials": prefix sharing). pa_paged_decode reads such a
+ * block once per sequence; this call reads it once per group:
+ *   1. a prepare kernel checks each group, stacks its members' query heads as
+ *      one KV head's query group and writes the group's prefix table and every
+ *      sequence's table of the blocks after its prefix;
+ *   2. one decode over the groups' prefix blocks (group_size * G query heads
+ *      per KV head), leaving its partition states in the workspace;
+ *   3. one decode over every sequence's remaining blocks, likewise;
+ *   4. a merge of the two sets of softmax states per output row.
+ * The result is the decode of pa_paged_decode up to floating-point rounding
+ * (the same fp32 arithmetic summed in another order).
+ *
+ * Arguments as for pa_paged_decode (no seq_order, no partition_tokens: both
+ * decodes use the library's default split), plus the group descriptor, in
+ * device memory, as pa_bm_prefix_groups writes it:
+ *   group_members        int32 [num_groups][group_size], batch indices, -1 pads;
+ *                        slot 0 is the group's leader
+ *   group_prefix_blocks  int32 [num_groups]: blocks shared by every member
+ *   seq_group, seq_member int32 [num_seqs]: each sequence's group and slot, or -1
+ *   num_groups, group_size, max_prefix_blocks: host bounds (grid and workspace
+ *                        sizing); group_size * (num_q_heads / num_kv_heads) must
+ *                        be 1, 2, 4 or 8, max_prefix_blocks >= every prefix
+ *   workspace            device, 256-byte aligned, at least
+ *                        pa_paged_decode_cascade_workspace_size bytes; fully
+ *                        rewritten by each call (no clearing needed)
+ * A sequence belongs to a group only if group_members[seq_group[s]][seq_member[s]]
+ * names s. A group whose members do not all hold the leader's first prefix
+ * blocks as full blocks inside their contexts, or whose descriptor is otherwise
+ * inconsistent, is decoded without its prefix (every member over its whole
+ * context) and PA_DEVERR_GROUP is set: the outputs stay correct. Host-side
+ * errors as for pa_paged_decode. pa_paged_decode_cascade_fp8 decodes E4M3
+ * caches with key and value scales, as pa_paged_decode_fp8.
+ * ------------------------------------------------------------------------- */
+int pa_paged_decode_cascade_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                           int head_dim, int max_context_len,
+                                           int max_blocks_per_seq, int block_size, int num_groups,
+                                           int group_size, int max_prefix_blocks, size_t* bytes);
+
+int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int max_context_len,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float scale, const int32_t* group_members,
+                            const int32_t* group_prefix_blocks, const int32_t* seq_group,
+                            const int32_t* seq_member, int num_groups, int group_size,
+                            int max_prefix_blocks, void* workspace, size_t workspace_bytes,
+                            int* dev_error, int dtype, void* stream);
+
+int pa_paged_decode_cascade_fp8(void* out, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                int max_context_len, int num_q_heads, int num_kv_heads,
+                                int head_dim, int block_size, int num_blocks, float scale,
+                                float k_scale, float v_scale, const int32_t* group_members,
+                                const int32_t* group_prefix_blocks, const int32_t* seq_group,
+                                const int32_t* seq_member, int num_groups, int group_size,
+                                int max_prefix_blocks, void* workspace, size_t workspace_bytes,
+                                int* dev_error, int dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Host block manager.
  *
- * "A pre-allocated memory pool, block allocation/reclamation, and refcounts
- * enabling cross-sequence sharing" ("PagedAttention: The vLLM Paper",
- * "Implementation Essentials"); blocks are taken on demand and only the last
+ * The pool is allocated once; blocks are handed out and taken back, and a
+ * reference count per block lets sequences share it ("PagedAttention: The vLLM
+ * Paper", "Implementation Essentials"); blocks are taken on demand and only the last
  * block of a sequence may be partly filled ("The design yields three immediate
  * wins", item 1); parallel samples share the prompt's blocks (item 3 and
  * "Implementation Essentials", prefix sharing).
@@ -344,6 +415,21 @@ int pa_bm_free_seq(pa_bm* bm, int64_t seq_id);
  * PA_ERR_INVALID_ARG if a table is longer than max_blocks. */
 int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* out,
                        int max_blocks);
+
+/* Groups of the batch seq_ids[0..n) that hold the same leading blocks, for
+ * pa_paged_decode_cascade. Members are batch indices (rows of the block tables).
+ * Rule: sequences with at least one full block are bucketed by their first
+ * block id (buckets in order of first appearance, members in batch order); each
+ * bucket is cut into runs of group_size; a run of two or more becomes a group
+ * whose prefix is the longest run of leading block ids the members all share
+ * and all hold full (at most each member's length / block_size). Outputs:
+ * group_members[n][group_size] (-1 pads), group_prefix_blocks[n], seq_group[n]
+ * (group of each batch index or -1) and seq_member[n] (its slot, -1 if none);
+ * *num_groups and *max_prefix_blocks (0 when there is no group). Swapped or
+ * unknown sequences are refused and nothing is written. */
+int pa_bm_prefix_groups(const pa_bm* bm, const int64_t* seq_ids, int n, int group_size,
+                        int32_t* group_members, int32_t* group_prefix_blocks, int32_t* seq_group,
+                        int32_t* seq_member, int* num_groups, int* max_prefix_blocks);
 
 /* Swapping. pa_bm_set_host_pool sizes the host pool (host blocks 0..n-1, handed
  * out 0 first; refused while any sequence is swapped out). pa_bm_swap_out moves

@@ -370,3 +370,51 @@ class BlockManager:
                 raise BlockManagerError(ERR_INVALID_ARG, "table longer than max_blocks")
             out[i, :len(t)] = t
         return out
+
+    def prefix_groups(self, seq_ids, group_size: int):
+        """Groups of the batch ``seq_ids`` whose members hold the same leading
+        blocks, for decoding a shared prefix once (a reading of this build: the
+        pages share a prompt's blocks among forks, "Implementation Essentials",
+        prefix sharing, but name no grouping rule).
+
+        Sequences with at least one full block are bucketed by their first block
+        id; buckets keep the order in which their first member appears, members
+        keep batch order. Each bucket is cut into consecutive runs of
+        ``group_size``; a run of two or more is a group whose prefix is the
+        number of leading block ids shared by all its members, capped at every
+        member's count of full blocks; a run whose prefix is 0 is no group.
+
+        Returns ``(members, prefix_blocks, seq_group, seq_member)``: a list of
+        member lists (batch indices), a list of prefix lengths, and per batch
+        index its group and slot (-1 when it has none).
+        """
+        seq_ids = list(seq_ids)
+        for s in seq_ids:
+            self._need(s)
+            self._resident(s)
+        full = [self._lens[s] // self.block_size for s in seq_ids]
+        buckets: dict[int, list[int]] = {}
+        for i, s in enumerate(seq_ids):
+            if full[i] >= 1:
+                buckets.setdefault(self._tables[s][0], []).append(i)
+        members, prefix = [], []
+        seq_group = [-1] * len(seq_ids)
+        seq_member = [-1] * len(seq_ids)
+        for run_source in buckets.values():
+            for c in range(0, len(run_source), group_size):
+                run = run_source[c:c + group_size]
+                if len(run) < 2:
+                    continue
+                tables = [self._tables[seq_ids[i]] for i in run]
+                p = min(full[i] for i in run)
+                shared = 0
+                while shared < p and all(t[shared] == tables[0][shared] for t in tables):
+                    shared += 1
+                if shared == 0:
+                    continue
+                for slot, i in enumerate(run):
+                    seq_group[i] = len(members)
+                    seq_member[i] = slot
+                members.append(run)
+                prefix.append(shared)
+        return members, prefix, seq_group, seq_member

@@ -13,19 +13,24 @@ from ._lib import (  # noqa: F401
     PA_BF16,
     PA_DEVERR_BLOCK_RANGE,
     PA_DEVERR_CONTEXT_RANGE,
+    PA_DEVERR_GROUP,
     PA_DEVERR_SLOT_RANGE,
     PA_DEVERR_WAIT_TIMEOUT,
     PA_F16,
     PA_FP8_E4M3,
     PA_PREEMPT_RECOMPUTE,
     PA_PREEMPT_SWAP,
+    PrefixGroups,
     Scheduler,
+    cascade_workspace,
     decode_workspace,
     last_error,
     lib,
     pa_copy_blocks,
     pa_longest_first_order,
     pa_paged_decode,
+    pa_paged_decode_cascade,
+    pa_paged_decode_cascade_workspace_size,
     pa_paged_decode_fp8,
     pa_paged_decode_workspace_size,
     pa_reshape_and_cache,

@@ -34,6 +34,7 @@ PA_DEVERR_SLOT_RANGE = 1
 PA_DEVERR_BLOCK_RANGE = 2
 PA_DEVERR_CONTEXT_RANGE = 4
 PA_DEVERR_WAIT_TIMEOUT = 8
+PA_DEVERR_GROUP = 16
 
 BLOCK_SIZE = 16
 
@@ -73,6 +74,19 @@ _SIGS = {
                                      _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
                                      ctypes.c_float, ctypes.c_float, _c_int, _vp, ctypes.c_size_t,
                                      _vp, _c_int, _vp]),
+    "pa_paged_decode_cascade_workspace_size": (_c_int, [_c_int] * 10 +
+                                                [ctypes.POINTER(ctypes.c_size_t)]),
+    "pa_paged_decode_cascade": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
+                                         _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp,
+                                         ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_paged_decode_cascade_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int,
+                                             _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                             ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                             _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp,
+                                             ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_bm_prefix_groups": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp,
+                                     ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "pa_bm_create": (_c_int, [_c_int, _c_int, _vp, ctypes.POINTER(_vp)]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_c_int, [_vp, _c_i64, _c_int, _vp]),
@@ -367,6 +381,94 @@ def pa_paged_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, ma
         ws_bytes, _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(q), _stream(stream)))
 
 
+def pa_paged_decode_cascade_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                           max_context_len, max_blocks_per_seq, num_groups,
+                                           group_size, max_prefix_blocks) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().pa_paged_decode_cascade_workspace_size(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, int(max_context_len),
+        int(max_blocks_per_seq), BLOCK_SIZE, int(num_groups), int(group_size),
+        int(max_prefix_blocks), ctypes.byref(n)))
+    return n.value
+
+
+class PrefixGroups:
+    """Groups of a batch that share leading blocks (``BlockManager.prefix_groups``),
+    as host arrays and, after ``to(device)``, as the device tensors
+    ``pa_paged_decode_cascade`` reads."""
+
+    def __init__(self, members, prefix_blocks, seq_group, seq_member, group_size,
+                 max_prefix_blocks):
+        self.members = members                # int32 [num_groups, group_size], -1 pads
+        self.prefix_blocks = prefix_blocks    # int32 [num_groups]
+        self.seq_group = seq_group            # int32 [num_seqs]
+        self.seq_member = seq_member          # int32 [num_seqs]
+        self.group_size = group_size
+        self.max_prefix_blocks = max_prefix_blocks
+        self.dev = None
+
+    @property
+    def num_groups(self) -> int:
+        return len(self.prefix_blocks)
+
+    def to(self, device):
+        torch = _torch()
+        members = self.members if self.num_groups else np.full((1, self.group_size), -1, np.int32)
+        prefix = self.prefix_blocks if self.num_groups else np.zeros(1, np.int32)
+        self.dev = tuple(torch.from_numpy(np.ascontiguousarray(x)).to(device)
+                         for x in (members, prefix, self.seq_group, self.seq_member))
+        return self
+
+
+def cascade_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                      max_blocks_per_seq, groups: PrefixGroups, device=None):
+    """A workspace tensor for pa_paged_decode_cascade (each call rewrites it)."""
+    torch = _torch()
+    n = pa_paged_decode_cascade_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                               max_context_len, max_blocks_per_seq,
+                                               groups.num_groups, groups.group_size,
+                                               groups.max_prefix_blocks)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def pa_paged_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens,
+                            max_context_len, scale, groups: PrefixGroups, workspace,
+                            dev_error=None, stream=None, k_scale=None, v_scale=None):
+    """Decode attention that reads blocks shared by a group's members once; writes
+    ``out`` ``[B, Hq, d]``. ``groups`` comes from ``BlockManager.prefix_groups`` for
+    the same batch order, moved to the device (``groups.to(device)``). E4M3 caches
+    take ``k_scale`` and ``v_scale``."""
+    torch = _torch()
+    nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
+    B, hq, dq = q.shape
+    fp8 = dtype_code(k_cache) == PA_FP8_E4M3
+    if dq != d or out.shape != q.shape or out.dtype != q.dtype or \
+            (not fp8 and q.dtype != k_cache.dtype):
+        raise PAError(PA_ERR_INVALID_ARG, "q/out must be [B, num_q_heads, head_dim] in the "
+                                          "query dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
+    if groups.dev is None or groups.seq_group.shape != (B,):
+        raise PAError(PA_ERR_INVALID_ARG, "groups must describe this batch and be on the device")
+    members, prefix, sgroup, smember = groups.dev
+    i32 = torch.int32
+    head = [_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", i32),
+            block_tables.shape[1], _dev_ptr(context_lens, "context_lens", i32), B,
+            int(max_context_len), hq, hkv, d, bs, nb, float(scale)]
+    tail = [_dev_ptr(members, "group_members", i32), _dev_ptr(prefix, "group_prefix_blocks", i32),
+            _dev_ptr(sgroup, "seq_group", i32), _dev_ptr(smember, "seq_member", i32),
+            groups.num_groups, groups.group_size, groups.max_prefix_blocks,
+            _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            _dev_ptr(dev_error, "dev_error", i32), dtype_code(q), _stream(stream)]
+    if fp8:
+        if k_scale is None or v_scale is None:
+            raise PAError(PA_ERR_INVALID_ARG, "E4M3 caches need k_scale and v_scale")
+        _check(lib().pa_paged_decode_cascade_fp8(*head, float(k_scale), float(v_scale), *tail))
+    else:
+        _check(lib().pa_paged_decode_cascade(*head, *tail))
+
+
 NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 
@@ -479,6 +581,24 @@ class BlockManager:
         _check(self._lib.pa_bm_block_tables(self._h, _i64p(ids), len(ids),
                                             out.ctypes.data if out.size else None, max_blocks))
         return out
+
+    def prefix_groups(self, seq_ids, group_size: int) -> "PrefixGroups":
+        """Groups of the batch ``seq_ids`` that hold the same leading blocks
+        (``pa_bm_prefix_groups``); members are batch indices."""
+        ids = np.ascontiguousarray(np.asarray(list(seq_ids), dtype=np.int64))
+        n = len(ids)
+        members = np.empty((max(n, 1), group_size), np.int32)
+        prefix = np.empty(max(n, 1), np.int32)
+        sgroup = np.empty(max(n, 1), np.int32)
+        smember = np.empty(max(n, 1), np.int32)
+        ng, mp = _c_int(0), _c_int(0)
+        _check(self._lib.pa_bm_prefix_groups(self._h, _i64p(ids), n, group_size,
+                                             members.ctypes.data, prefix.ctypes.data,
+                                             sgroup.ctypes.data, smember.ctypes.data,
+                                             ctypes.byref(ng), ctypes.byref(mp)))
+        k = ng.value
+        return PrefixGroups(members[:k].copy(), prefix[:k].copy(), sgroup[:n].copy(),
+                            smember[:n].copy(), group_size, mp.value)
 
     def num_free(self) -> int:
         return self._lib.pa_bm_num_free(self._h)

@@ -25,6 +25,7 @@
 //
 // Every mutating call first works out how many free blocks it needs and fails
 // before touching any state when the pool cannot cover it.
+#include <algorithm>
 #include <stdint.h>
 
 #include <new>
@@ -206,6 +207,68 @@ int pa_bm_block_tables(const pa_bm* bm, const int64_t* seq_ids, int n, int32_t* 
     for (; k < t.size(); ++k) row[k] = t[k];
     for (; k < (size_t)max_blocks; ++k) row[k] = -1;
   }
+  return PA_OK;
+}
+
+int pa_bm_prefix_groups(const pa_bm* bm, const int64_t* seq_ids, int n, int group_size,
+                        int32_t* group_members, int32_t* group_prefix_blocks, int32_t* seq_group,
+                        int32_t* seq_member, int* num_groups, int* max_prefix_blocks) {
+  pa::clear_error();
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "null manager");
+  if (n < 0 || group_size < 1) return fail(PA_ERR_INVALID_ARG, "bad n or group_size");
+  if (!num_groups || !max_prefix_blocks) return fail(PA_ERR_INVALID_ARG, "null output pointer");
+  if (n > 0 && (!seq_ids || !group_members || !group_prefix_blocks || !seq_group || !seq_member))
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  std::vector<const pa_bm::Seq*> seqs(n);
+  for (int i = 0; i < n; ++i) {  // validate everything before writing anything
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end())
+      return fail(PA_ERR_UNKNOWN_SEQ, "unknown sequence %lld", (long long)seq_ids[i]);
+    if (it->second.swapped) return swapped_error(seq_ids[i]);
+    seqs[i] = &it->second;
+  }
+  auto full = [&](int i) { return (int)(seqs[i]->len / bm->block_size); };
+  std::vector<int32_t> first_keys;
+  std::unordered_map<int32_t, std::vector<int>> buckets;
+  for (int i = 0; i < n; ++i) {
+    seq_group[i] = -1;
+    seq_member[i] = -1;
+    if (full(i) < 1) continue;
+    const int32_t key = seqs[i]->table[0];
+    auto& b = buckets[key];
+    if (b.empty()) first_keys.push_back(key);
+    b.push_back(i);
+  }
+  int ng = 0, maxp = 0;
+  for (int32_t key : first_keys) {
+    const std::vector<int>& b = buckets[key];
+    for (size_t c = 0; c < b.size(); c += group_size) {
+      const size_t m = std::min(b.size() - c, (size_t)group_size);
+      if (m < 2) continue;
+      const std::vector<int32_t>& lead = seqs[b[c]]->table;
+      int P = full(b[c]);
+      for (size_t j = 1; j < m; ++j) {
+        const std::vector<int32_t>& t = seqs[b[c + j]]->table;
+        P = std::min(P, full(b[c + j]));
+        int k = 0;
+        while (k < P && t[k] == lead[k]) ++k;
+        P = k;
+      }
+      if (P < 1) continue;
+      int32_t* row = group_members + (size_t)ng * group_size;
+      for (int j = 0; j < group_size; ++j) row[j] = -1;
+      for (size_t j = 0; j < m; ++j) {
+        row[j] = b[c + j];
+        seq_group[b[c + j]] = ng;
+        seq_member[b[c + j]] = (int32_t)j;
+      }
+      group_prefix_blocks[ng] = P;
+      maxp = std::max(maxp, P);
+      ++ng;
+    }
+  }
+  *num_groups = ng;
+  *max_prefix_blocks = maxp;
   return PA_OK;
 }
 

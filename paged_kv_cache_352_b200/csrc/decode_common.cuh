@@ -18,7 +18,8 @@ namespace pa {
 // to the common maximum. A sequence with a single partition writes `out`
 // directly. Otherwise the CTA stores its partition state in the workspace, and
 // the CTA that completes the sequence's last partition merges all partitions
-// in logical order and returns the counter to zero.
+// in logical order and returns the counter to zero. With a.states_only every
+// partition stores its state and nothing is merged.
 // `wts` (>= nparts * G floats of shared memory) may alias red_*: it is written
 // only after they have been read. Every thread of the CTA must call this with
 // the same arguments; it ends with a barrier, so shared memory it used can be
@@ -30,7 +31,7 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
                                                  int nparts, T* out_rows) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool split = nparts > 1;
+  const bool split = nparts > 1 || a.states_only;
   const size_t unit = (size_t)s * a.num_kv_heads + kvh;
   for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
     const int g = item / D;
@@ -57,7 +58,7 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, float* wts
       }
     }
   }
-  if (!split) {
+  if (!split || a.states_only) {
     __syncthreads();
     return;
   }

@@ -403,6 +403,7 @@ int paged_decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.scale_log2 = scale * 1.4426950408889634f * k_scale;
   a.out_scale = v_scale;
   a.warp_parts = use_warp_parts(num_seqs, num_kv_heads, lay.part_blocks, lay.max_parts);
+  a.states_only = 0;
   const cudaError_t e = launch_paged_decode(a, head_dim, group, dtype, cache_dtype,
                                             static_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidConfiguration)
@@ -413,9 +414,305 @@ int paged_decode_impl(void* out, const void* q, const void* k_cache, const void*
   return cuda_status(e, "paged_decode launch");
 }
 
+// Workspace of a cascade decode: stacked queries, the groups' prefix tables and
+// lengths, the own-block tables and lengths, then the partition states of the
+// decode over the groups' prefixes and of the decode over the own blocks.
+struct CascadeLayout {
+  int g_part_blocks, g_parts, s_part_blocks, s_parts;
+  size_t gq_off, gt_off, gctx_off, st_off, sctx_off, spb_off, snp_off;
+  size_t gcount_off, gml_off, gacc_off, scount_off, sml_off, sacc_off, bytes;
+};
+
+int cascade_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                   int max_context_len, int max_blocks_per_seq, int num_groups, int group_size,
+                   int max_prefix_blocks, CascadeLayout* L) {
+  if (num_seqs < 0 || num_seqs > 65535)
+    return fail(PA_ERR_INVALID_ARG, "num_seqs %d: expected 0 .. 65535", num_seqs);
+  if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads %d must be a positive multiple of num_kv_heads %d",
+                num_q_heads, num_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", head_dim);
+  const int gh = num_q_heads / num_kv_heads;
+  if (gh != 1 && gh != 2 && gh != 4 && gh != 8)
+    return fail(PA_ERR_UNSUPPORTED, "query heads per KV head = %d: supported 1, 2, 4, 8", gh);
+  if (max_context_len < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len must be >= 0");
+  if (max_blocks_per_seq <= 0) return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq must be > 0");
+  if (num_groups < 0 || num_groups > 65535)
+    return fail(PA_ERR_INVALID_ARG, "num_groups %d: expected 0 .. 65535", num_groups);
+  const int gg = group_size * gh;
+  if (group_size < 1 || (gg != 1 && gg != 2 && gg != 4 && gg != 8))
+    return fail(PA_ERR_UNSUPPORTED,
+                "group_size %d x %d query heads per KV head must be 1, 2, 4 or 8", group_size, gh);
+  if (num_groups > 0 && (max_prefix_blocks < 1 || max_prefix_blocks > max_blocks_per_seq))
+    return fail(PA_ERR_INVALID_ARG, "max_prefix_blocks %d: expected 1 .. max_blocks_per_seq (%d)",
+                max_prefix_blocks, max_blocks_per_seq);
+  const int ng = num_groups > 0 ? num_groups : 0;
+  const int pmax = num_groups > 0 ? max_prefix_blocks : 1;
+  L->g_part_blocks = default_partition_blocks(ng > 0 ? ng : 1, num_kv_heads, pmax, false);
+  L->g_parts = (pmax + L->g_part_blocks - 1) / L->g_part_blocks;
+  const int own_blocks = std::max(1, (max_context_len + kBlockSize - 1) / kBlockSize);
+  L->s_part_blocks = default_partition_blocks(num_seqs > 0 ? num_seqs : 1, num_kv_heads,
+                                              own_blocks, false);
+  L->s_parts = (own_blocks + L->s_part_blocks - 1) / L->s_part_blocks;
+  if (L->g_parts > 65535 || L->s_parts > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "too many partitions per sequence");
+  // prefix-state rows are addressed with 32-bit indices
+  if ((long long)ng * num_kv_heads * L->g_parts * gg >= 0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED, "too many groups x KV heads x partitions");
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = up(o + bytes);
+    return at;
+  };
+  const size_t gu = (size_t)ng * num_kv_heads, su = (size_t)num_seqs * num_kv_heads;
+  L->gq_off = take((size_t)ng * num_kv_heads * gg * head_dim * 2);
+  L->gt_off = take((size_t)ng * max_blocks_per_seq * 4);
+  L->gctx_off = take((size_t)ng * 4);
+  L->st_off = take((size_t)num_seqs * max_blocks_per_seq * 4);
+  L->sctx_off = take((size_t)num_seqs * 4);
+  L->spb_off = take((size_t)num_seqs * 4);
+  L->snp_off = take((size_t)num_seqs * 4);
+  L->gcount_off = take(gu * sizeof(int));
+  L->gml_off = take(gu * L->g_parts * gg * 2 * sizeof(float));
+  L->gacc_off = take(gu * L->g_parts * gg * head_dim * sizeof(float));
+  L->scount_off = take(su * sizeof(int));
+  L->sml_off = take(su * L->s_parts * gh * 2 * sizeof(float));
+  L->sacc_off = take(su * L->s_parts * gh * head_dim * sizeof(float));
+  L->bytes = o;
+  return PA_OK;
+}
+
+// The decode over the groups' prefixes runs on a second stream beside the
+// own-block decode on the caller's stream (the two read disjoint blocks and
+// write disjoint states), forked after the prepare kernel and joined before the
+// merge by events. One stream and two events per device and host thread, made
+// on first use and kept for the life of the process; the fork and join are
+// legal inside stream capture.
+struct AuxStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+constexpr int kMaxAuxDevices = 64;
+
+int aux_stream(AuxStream** out) {
+  thread_local AuxStream aux[kMaxAuxDevices];
+  int dev = 0;
+  if (int st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice")) return st;
+  if (dev < 0 || dev >= kMaxAuxDevices) return fail(PA_ERR_UNSUPPORTED, "device %d", dev);
+  AuxStream& a = aux[dev];
+  if (!a.stream) {
+    if (int st = cuda_status(cudaStreamCreateWithFlags(&a.stream, cudaStreamNonBlocking),
+                             "auxiliary stream"))
+      return st;
+    if (int st = cuda_status(cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming),
+                             "fork event"))
+      return st;
+    if (int st = cuda_status(cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming),
+                             "join event"))
+      return st;
+  }
+  *out = &a;
+  return PA_OK;
+}
+
+int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, int max_blocks_per_seq,
+                              const int32_t* context_lens, int num_seqs, int max_context_len,
+                              int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                              int num_blocks, float scale, float k_scale, float v_scale,
+                              const int32_t* group_members, const int32_t* group_prefix_blocks,
+                              const int32_t* seq_group, const int32_t* seq_member,
+                              int num_groups, int group_size, int max_prefix_blocks,
+                              void* workspace, size_t workspace_bytes, int* dev_error,
+                              int dtype, int cache_dtype, void* stream) {
+  if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
+  CascadeLayout lay;
+  if (int st = cascade_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                              max_blocks_per_seq, num_groups, group_size, max_prefix_blocks, &lay))
+    return st;
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !seq_group ||
+      !seq_member || (num_groups > 0 && (!group_members || !group_prefix_blocks)))
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "out, q and cache pointers must be 16-byte aligned");
+  if (!workspace || workspace_bytes < lay.bytes)
+    return fail(PA_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", lay.bytes,
+                workspace ? workspace_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const int gh = num_q_heads / num_kv_heads;
+  const int gg = group_size * gh;
+  CascadeArgs c;
+  c.q = q;
+  c.block_tables = block_tables;
+  c.context_lens = context_lens;
+  c.group_members = group_members;
+  c.group_prefix_blocks = group_prefix_blocks;
+  c.seq_group = seq_group;
+  c.seq_member = seq_member;
+  c.gq = ws + lay.gq_off;
+  c.g_tables = reinterpret_cast<int32_t*>(ws + lay.gt_off);
+  c.g_ctx = reinterpret_cast<int32_t*>(ws + lay.gctx_off);
+  c.s_tables = reinterpret_cast<int32_t*>(ws + lay.st_off);
+  c.s_ctx = reinterpret_cast<int32_t*>(ws + lay.sctx_off);
+  c.s_pbase = reinterpret_cast<int32_t*>(ws + lay.spb_off);
+  c.s_np = reinterpret_cast<int32_t*>(ws + lay.snp_off);
+  const size_t gu = (size_t)num_groups * num_kv_heads, su = (size_t)num_seqs * num_kv_heads;
+  float* gm = reinterpret_cast<float*>(ws + lay.gml_off);
+  float* sm = reinterpret_cast<float*>(ws + lay.sml_off);
+  c.g_m = gm;
+  c.g_l = gm + gu * lay.g_parts * gg;
+  c.g_acc = reinterpret_cast<float*>(ws + lay.gacc_off);
+  c.s_m = sm;
+  c.s_l = sm + su * lay.s_parts * gh;
+  c.s_acc = reinterpret_cast<float*>(ws + lay.sacc_off);
+  c.out = out;
+  c.dev_error = dev_error;
+  c.num_seqs = num_seqs;
+  c.num_groups = num_groups;
+  c.group_size = group_size;
+  c.num_q_heads = num_q_heads;
+  c.num_kv_heads = num_kv_heads;
+  c.max_blocks_per_seq = max_blocks_per_seq;
+  c.max_prefix_blocks = num_groups > 0 ? max_prefix_blocks : 0;
+  c.max_context_len = max_context_len;
+  c.g_parts = lay.g_parts;
+  c.g_part_blocks = lay.g_part_blocks;
+  c.s_parts = lay.s_parts;
+  c.s_part_blocks = lay.s_part_blocks;
+  c.out_scale = v_scale;
+  if (int e = cuda_status(launch_cascade_prepare(c, head_dim, dtype, st), "cascade prepare launch"))
+    return e;
+
+  // both decodes leave partition states only; the merge writes `out`
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.out = out;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.seq_order = nullptr;
+  a.dev_error = dev_error;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.max_context_len = max_context_len;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.scale_log2 = scale * 1.4426950408889634f * k_scale;
+  a.out_scale = 1.f;
+  a.warp_parts = 0;
+  a.states_only = 1;
+  AuxStream* aux = nullptr;
+  if (num_groups > 0) {
+    if (int e = aux_stream(&aux)) return e;
+    if (int e = cuda_status(cudaEventRecord(aux->fork, st), "fork record")) return e;
+    if (int e = cuda_status(cudaStreamWaitEvent(aux->stream, aux->fork, 0), "fork wait"))
+      return e;
+    DecodeArgs gpre = a;
+    gpre.q = c.gq;
+    gpre.block_tables = c.g_tables;
+    gpre.context_lens = c.g_ctx;
+    gpre.ws_count = reinterpret_cast<int*>(ws + lay.gcount_off);
+    gpre.ws_m = gm;
+    gpre.ws_l = const_cast<float*>(c.g_l);
+    gpre.ws_acc = const_cast<float*>(c.g_acc);
+    gpre.num_seqs = num_groups;
+    gpre.num_q_heads = num_kv_heads * gg;
+    gpre.part_blocks = lay.g_part_blocks;
+    gpre.max_parts = lay.g_parts;
+    if (int e = cuda_status(launch_paged_decode(gpre, head_dim, gg, dtype, cache_dtype,
+                                                aux->stream),
+                            "cascade prefix decode launch"))
+      return e;
+    if (int e = cuda_status(cudaEventRecord(aux->join, aux->stream), "join record")) return e;
+  }
+  DecodeArgs own = a;
+  own.q = q;
+  own.block_tables = c.s_tables;
+  own.context_lens = c.s_ctx;
+  own.ws_count = reinterpret_cast<int*>(ws + lay.scount_off);
+  own.ws_m = sm;
+  own.ws_l = const_cast<float*>(c.s_l);
+  own.ws_acc = const_cast<float*>(c.s_acc);
+  own.num_seqs = num_seqs;
+  own.num_q_heads = num_q_heads;
+  own.part_blocks = lay.s_part_blocks;
+  own.max_parts = lay.s_parts;
+  if (int e = cuda_status(launch_paged_decode(own, head_dim, gh, dtype, cache_dtype, st),
+                          "cascade own-block decode launch"))
+    return e;
+  if (aux) {
+    if (int e = cuda_status(cudaStreamWaitEvent(st, aux->join, 0), "join wait")) return e;
+  }
+  return cuda_status(launch_cascade_merge(c, head_dim, dtype, st), "cascade merge launch");
+}
+
 }  // namespace
 
 extern "C" {
+
+int pa_paged_decode_cascade_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                           int head_dim, int max_context_len,
+                                           int max_blocks_per_seq, int block_size, int num_groups,
+                                           int group_size, int max_prefix_blocks, size_t* bytes) {
+  clear_error();
+  if (!bytes) return fail(PA_ERR_INVALID_ARG, "bytes must not be NULL");
+  if (block_size != kBlockSize)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d: only %d is supported", block_size,
+                kBlockSize);
+  CascadeLayout lay;
+  if (int st = cascade_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                              max_blocks_per_seq, num_groups, group_size, max_prefix_blocks, &lay))
+    return st;
+  *bytes = lay.bytes;
+  return PA_OK;
+}
+
+int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int max_context_len,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float scale, const int32_t* group_members,
+                            const int32_t* group_prefix_blocks, const int32_t* seq_group,
+                            const int32_t* seq_member, int num_groups, int group_size,
+                            int max_prefix_blocks, void* workspace, size_t workspace_bytes,
+                            int* dev_error, int dtype, void* stream) {
+  clear_error();
+  return paged_decode_cascade_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                   context_lens, num_seqs, max_context_len, num_q_heads,
+                                   num_kv_heads, head_dim, block_size, num_blocks, scale, 1.f, 1.f,
+                                   group_members, group_prefix_blocks, seq_group, seq_member,
+                                   num_groups, group_size, max_prefix_blocks, workspace,
+                                   workspace_bytes, dev_error, dtype, dtype, stream);
+}
+
+int pa_paged_decode_cascade_fp8(void* out, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                int max_context_len, int num_q_heads, int num_kv_heads,
+                                int head_dim, int block_size, int num_blocks, float scale,
+                                float k_scale, float v_scale, const int32_t* group_members,
+                                const int32_t* group_prefix_blocks, const int32_t* seq_group,
+                                const int32_t* seq_member, int num_groups, int group_size,
+                                int max_prefix_blocks, void* workspace, size_t workspace_bytes,
+                                int* dev_error, int dtype, void* stream) {
+  clear_error();
+  if (!positive_finite(k_scale) || !positive_finite(v_scale))
+    return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
+  return paged_decode_cascade_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                   context_lens, num_seqs, max_context_len, num_q_heads,
+                                   num_kv_heads, head_dim, block_size, num_blocks, scale, k_scale,
+                                   v_scale, group_members, group_prefix_blocks, seq_group,
+                                   seq_member, num_groups, group_size, max_prefix_blocks,
+                                   workspace, workspace_bytes, dev_error, dtype, PA_FP8_E4M3,
+                                   stream);
+}
 
 int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int max_blocks_per_seq,

@@ -50,6 +50,9 @@ struct DecodeArgs {
   float scale_log2;  // softmax scale * log2(e) (* the key scale of an E4M3 cache)
   float out_scale;   // 1, or the value scale of an E4M3 cache
   int warp_parts;    // split mode: one warp per partition + a merge launch (else one CTA)
+  int states_only;   // every partition leaves its state in the workspace; nothing writes
+                     // `out` and no partitions are merged (a sequence with no blocks
+                     // leaves no state): the caller merges them
 };
 
 // Split partitions of at most this many blocks, for batches whose longest
@@ -86,6 +89,44 @@ cudaError_t launch_reshape_and_cache_fp8(const void* key, const void* value, int
                                          int num_kv_heads, int head_dim, int num_blocks,
                                          int src_dtype, float k_scale, float v_scale,
                                          int* dev_error, cudaStream_t stream);
+
+// Cascade decode of sequences that share leading blocks: the prefix states of
+// every group come from one decode over the shared blocks (the members' query
+// heads stacked as one KV head's group), the rest of each sequence from its own
+// blocks, and a merge combines the two.
+struct CascadeArgs {
+  const void* q;                       // [B][Hq][D]
+  const int32_t* block_tables;         // [B][max_blocks]
+  const int32_t* context_lens;         // [B]
+  const int32_t* group_members;        // [num_groups][group_size], -1 pads
+  const int32_t* group_prefix_blocks;  // [num_groups]
+  const int32_t* seq_group;            // [B]: group of s, or -1
+  const int32_t* seq_member;           // [B]: slot of s in its group
+  void* gq;            // [num_groups][Hkv * group_size * Gh][D] stacked queries (written)
+  int32_t* g_tables;   // [num_groups][max_blocks] leader's prefix entries, -1 after (written)
+  int32_t* g_ctx;      // [num_groups] prefix tokens used, 0 for a rejected group (written)
+  int32_t* s_tables;   // [B][max_blocks] each sequence's blocks after its prefix (written)
+  int32_t* s_ctx;      // [B] tokens after the prefix (written)
+  int32_t* s_pbase;    // [B] first prefix-state row of s (kvh 0, head 0), -1 if none (written)
+  int32_t* s_np;       // [B] prefix partitions of s (written)
+  const float* g_m;    // group decode states [num_groups][Hkv][g_parts][Gg] (+ [D] for acc)
+  const float* g_l;
+  const float* g_acc;
+  const float* s_m;    // own-block decode states [B][Hkv][s_parts][Gh] (+ [D] for acc)
+  const float* s_l;
+  const float* s_acc;
+  void* out;           // [B][Hq][D]
+  int* dev_error;
+  int num_seqs, num_groups, group_size, num_q_heads, num_kv_heads;
+  int max_blocks_per_seq, max_prefix_blocks, max_context_len;
+  int g_parts, g_part_blocks, s_parts, s_part_blocks;
+  float out_scale;
+};
+
+cudaError_t launch_cascade_prepare(const CascadeArgs& c, int head_dim, int dtype,
+                                   cudaStream_t stream);
+cudaError_t launch_cascade_merge(const CascadeArgs& c, int head_dim, int dtype,
+                                 cudaStream_t stream);
 
 struct CopyPairs {
   int32_t src[kMaxCopyPairsPerLaunch];

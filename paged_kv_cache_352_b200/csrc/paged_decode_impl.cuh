@@ -74,7 +74,8 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   if (part >= (nparts > 0 ? nparts : 1)) return;
   T* out_rows = reinterpret_cast<T*>(a.out) + ((size_t)s * a.num_q_heads + (size_t)kvh * G) * D;
   if (nblk == 0) {
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) out_rows[i] = Storage<T>::from_f32(0.f);
+    if (!a.states_only)
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x) out_rows[i] = Storage<T>::from_f32(0.f);
     return;
   }
   const int nlocal = min(nblk, b_begin + a.part_blocks) - b_begin;
@@ -373,7 +374,7 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
     dim3 wgrid(a.num_kv_heads, (a.max_parts + WARPS - 1) / WARPS, a.num_seqs);
     wkern<<<wgrid, WARPS * 32, smem, stream>>>(a, tk, tv);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || a.states_only) return e;
     dim3 mgrid(a.num_kv_heads * G, a.num_seqs);
     merge_partitions_kernel<T, D, G><<<mgrid, kMergeThreads, 0, stream>>>(a);
     return cudaGetLastError();

@@ -74,6 +74,19 @@ class DecodeRunner:
         self.workspace = L.decode_workspace(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
                                             wl.head_dim, wl.max_context_len,
                                             self.partition_tokens, self.device)
+        # Samples forked from one prompt hold its full blocks in common: the step
+        # decodes them through pa_paged_decode_cascade, which reads each shared
+        # block once per group of samples (8 / G samples stacked per KV head).
+        self.groups = None
+        self.cascade_ws = None
+        g = wl.num_q_heads // wl.num_kv_heads
+        if wl.kind == "shared_prefix" and not duplicate and g <= 4:
+            groups = self.bm.prefix_groups(range(wl.num_seqs), 8 // g)
+            if groups.num_groups:
+                self.groups = groups.to(self.device)
+                self.cascade_ws = L.cascade_workspace(
+                    wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                    wl.max_context_len, self.max_blocks, self.groups, self.device)
         torch.cuda.synchronize(self.device)
 
     # -- set-up -----------------------------------------------------------------
@@ -173,17 +186,33 @@ class DecodeRunner:
                           self.dev_error, seq_order=self.seq_order if ordered else None)
         return out
 
+    def decode_cascade(self, out=None):
+        """The decode through pa_paged_decode_cascade (batches with groups only)."""
+        out = self.out if out is None else out
+        L.pa_paged_decode_cascade(out, self.q, self.k_cache, self.v_cache, self.block_tables,
+                                  self.context_lens, self.wl.max_context_len, self.wl.scale,
+                                  self.groups, self.cascade_ws, self.dev_error)
+        return out
+
+    def decode_step(self, out=None):
+        """The step's decode: the cascade when sequences share blocks, else plain."""
+        if self.groups is not None:
+            return self.decode_cascade(out)
+        return self.decode(out)
+
     def step(self):
         """One decode step: copy-on-write copies, cache writes, decode attention."""
         self.copy_blocks()
         self.reshape_and_cache()
-        return self.decode()
+        return self.decode_step()
 
     def launches_per_step(self) -> int:
         wl = self.wl
         _, _, decode = L.pa_paged_decode_plan(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
                                               wl.head_dim, wl.max_context_len,
                                               self.partition_tokens or 0, ordered=True)
+        if self.groups is not None:
+            decode = 4  # prepare, prefix decode, own-block decode, merge
         return int(len(self.cow_pairs) > 0) * -(-len(self.cow_pairs) // 1024) + \
             int(len(self.step_slots_host) > 0) + decode
 
@@ -294,7 +323,7 @@ class HostPipeline:
             setattr(r, name, v)
         r.copy_blocks()
         r.reshape_and_cache()
-        r.decode(out=sl["out"])
+        r.decode_step(out=sl["out"])
         sl["out_ready"].record(self.compute)
         with torch.cuda.stream(self.download):
             self.download.wait_event(sl["out_ready"])

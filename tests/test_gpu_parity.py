@@ -71,15 +71,21 @@ def test_physical_placement_is_invisible_bitwise(name):
 
 
 def test_shared_blocks_equal_duplicated_blocks_bitwise():
+    """pa_paged_decode gives the same bits whether samples share the prompt's
+    blocks or hold private copies. (The shared runner's step decodes through the
+    cascade, which sums in another order: equal within tolerance.)"""
     wl = workloads.workload("prefix_share_cow", small=True)
     shared = DecodeRunner(wl)
     dup = DecodeRunner(wl, duplicate=True)
     assert len(shared.cow_pairs) > 0 and len(dup.cow_pairs) == 0
     assert shared.bm.num_free() > dup.bm.num_free()
-    a = shared.step().clone()
+    assert shared.groups is not None and dup.groups is None
+    cascade = shared.step().clone()
+    a = shared.decode().clone()
     b = dup.step()
     _sync()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert_close(out_to_f64(cascade, wl.dtype), out_to_f64(b, wl.dtype), "cascade vs duplicated")
 
 
 @pytest.mark.parametrize("name", ["mha_7b_fp16", "gqa_32_8_bf16", "long_ctx_split_kv"])
