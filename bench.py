@@ -757,7 +757,9 @@ def run_ours(args):
     # an L2 flush that READS a buffer larger than L2: a write flush would leave
     # dirty lines whose write-back the next kernel would pay for.
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
-    flush_needed = decode_bytes(wl) < 4 * l2_bytes if args.l2 == "auto" else args.l2 == "flush"
+    # (sequences sharing blocks read only their distinct blocks from HBM: those decide)
+    read_bytes = unique_decode_bytes(wl, r) if r.groups is not None else decode_bytes(wl)
+    flush_needed = read_bytes < 4 * l2_bytes if args.l2 == "auto" else args.l2 == "flush"
     flush = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=device) \
         if flush_needed else None
     flush_sink = torch.empty(1, dtype=torch.int64, device=device)
@@ -914,7 +916,7 @@ def run_ours(args):
                    "partition_tokens": r.partition_tokens,
                    "l2": ("flushed between steps by reading a 256 MiB buffer, outside the "
                           "timed events" if flush_needed else
-                          f"inputs larger than L2 ({decode_bytes(wl) / 1e6:.0f} MB vs "
+                          f"inputs larger than L2 ({read_bytes / 1e6:.0f} MB vs "
                           f"{l2_bytes / 1e6:.0f} MB L2), no flush"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
