@@ -489,8 +489,7 @@ int cascade_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim
 // own-block decode on the caller's stream (the two read disjoint blocks and
 // write disjoint states), forked after the prepare kernel and joined before the
 // merge by events. One stream and two events per device and host thread, made
-// on first use and kept for the life of the process; the fork and join are
-// legal inside stream capture.
+// on first use and kept for the life of the process.
 struct AuxStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
