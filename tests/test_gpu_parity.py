@@ -18,7 +18,6 @@ import paged_kv_cache_352_b200 as pa
 from paged_kv_cache_352_b200.runner import DecodeRunner
 from tests.parity import assert_close, out_to_f64, tensor_bits
 import workloads
-from workloads import gen
 
 pytestmark = pytest.mark.gpu
 
