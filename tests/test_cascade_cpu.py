@@ -153,3 +153,17 @@ def test_cascade_workspace_covers_both_decodes():
     states_s = B * hkv * 1 * (d + 2) * 4
     tables = (ng + B) * mb * 4
     assert n >= gq + states_g + states_s + tables
+
+
+def test_prefix_groups_of_empty_and_unshared_batches():
+    bm = pa.BlockManager(256)
+    g = bm.prefix_groups([], 8)
+    assert g.num_groups == 0 and g.max_prefix_blocks == 0 and len(g.seq_group) == 0
+    for s, n in ((0, 40), (1, 16), (2, 0), (3, 300)):
+        bm.add_seq(s, n)
+    g = bm.prefix_groups([3, 0, 2, 1], 8)     # no two sequences share a block
+    assert g.num_groups == 0 and g.seq_group.tolist() == [-1] * 4
+    assert g.seq_member.tolist() == [-1] * 4
+    ws = pa.pa_paged_decode_cascade_workspace_size(4, 8, 8, 64, 300, 19, g.num_groups, 1,
+                                                   g.max_prefix_blocks)
+    assert ws > 0
