@@ -316,6 +316,14 @@ def rank_workload(name: str, rank: int, num_seqs: int = 0, num_blocks: int = 0):
 # CPU oracle timing (cpu_baseline leg and --impl reference)
 # --------------------------------------------------------------------------
 
+def _host_cpus() -> int:
+    """CPUs this process may run on (the oracle's BLAS pool is sized from them)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux
+        return os.cpu_count() or 1
+
+
 def _oracle_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -725,6 +733,7 @@ def run_reference(args):
                                            if k != "workload"}},
         "decode_tokens_per_s": round(nseq * args.steps / el, 3),
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": _oracle_threads(),
+                         "host_cpus": _host_cpus(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -948,6 +957,7 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         v, tps, desc, _ = time_oracle(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": _oracle_threads(),
+                                "host_cpus": _host_cpus(),
                                 "kind": "oracle", "sample": desc,
                                 "decode_tokens_per_s": round(tps, 3)}
         one = time_oracle_one_thread(wl, budget_s=min(5.0, args.cpu_budget / 3))
