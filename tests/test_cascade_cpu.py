@@ -50,7 +50,7 @@ def _fork_forest(seed, nb=3000):
 
 
 @pytest.mark.parametrize("seed", range(12))
-@pytest.mark.parametrize("group_size", [2, 4, 8])
+@pytest.mark.parametrize("group_size", [2, 3, 4, 5, 8])
 def test_prefix_groups_match_oracle(seed, group_size):
     cbm, obm, batch = _fork_forest(seed)
     g = cbm.prefix_groups(batch, group_size)
