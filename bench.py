@@ -533,6 +533,32 @@ def shared_prompt_trace(num_requests: int = 1000, seed: int = 353, systems: int 
     return trace
 
 
+def measure_host_planning(num_requests: int = 1000, num_blocks: int = 8192,
+                          max_num_seqs: int = 256, host_blocks: int = 4096):
+    """The scheduler's planning alone (block manager, slot mappings, copy-on-write
+    pairs, swaps, tables; C++ behind one binding call per step) over the
+    continuous-batching trace, host wall time: the host share of each step, which
+    the loop overlaps with the GPU's work on the previous plans."""
+    from paged_kv_cache_352_b200 import _lib as L
+    trace = continuous_batching_trace(num_requests)
+    sched = L.Scheduler(num_blocks, 16, np.random.default_rng(7).permutation(num_blocks),
+                        max_num_seqs=max_num_seqs, num_host_blocks=host_blocks)
+    for t in trace:
+        sched.submit(*t[:5])
+    steps = slots = 0
+    t0 = time.perf_counter()
+    while not sched.idle():
+        c = sched.step()
+        steps += 1
+        slots += c.num_seqs + c.num_prefill
+    el = time.perf_counter() - t0
+    return {"us_per_step": round(el / steps * 1e6, 2), "steps": steps, "slots": slots,
+            "slots_per_s": round(slots / el, 1),
+            "what": "pa_sched_step alone over the continuous-batching trace (1000 requests): "
+                    "admission, appends with copy-on-write, preemption by swap, slot mappings "
+                    "and tables; host wall time including the binding"}
+
+
 def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks: int = 8192,
                                 max_num_seqs: int = 256, host_blocks: int = 4096,
                                 max_model_len: int = 2048, fp8_scales=None, trace=None,
@@ -875,6 +901,7 @@ def run_ours(args):
     swap = measure_swap(wl, r, device) if extras else None
     prefix_cache = measure_prefix_cache(wl, device) if extras else None
     batching = measure_continuous_batching(wl, device) if extras else None
+    host_planning = measure_host_planning() if extras else None
     batching_fp8 = measure_continuous_batching(wl, device, fp8_scales=(0.05, 0.02)) \
         if extras else None
     batching_prefix = None
@@ -949,6 +976,7 @@ def run_ours(args):
         "swap": swap,
         "prefix_cache": prefix_cache,
         "continuous_batching": batching,
+        "host_planning": host_planning,
         "continuous_batching_fp8": batching_fp8,
         "continuous_batching_shared_prompts": batching_prefix,
         "fp8_kv": fp8,

@@ -168,3 +168,13 @@ def test_submit_tokens_checks_length():
     c = pa.Scheduler(8, 16)
     with pytest.raises(pa.PAError):
         c.submit(0, 5, 3, tokens=[1, 2, 3])
+
+
+def test_host_planning_measurement_runs_the_whole_trace():
+    """The bench's host-planning figure plans a whole trace: every request's
+    prompt and output tokens get slots."""
+    import bench
+    trace = bench.continuous_batching_trace(60)
+    r = bench.measure_host_planning(num_requests=60)
+    want = sum(t[2] * t[3] for t in trace)   # generated tokens: output length x samples
+    assert r["steps"] > 0 and r["slots"] >= want and r["us_per_step"] > 0
