@@ -318,6 +318,11 @@ int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache, const
  *      per KV head), leaving its partition states in the workspace;
  *   3. one decode over every sequence's remaining blocks, likewise;
  *   4. a merge of the two sets of softmax states per output row.
+ * Step 2 runs on a second stream of the library's, beside step 3 on `stream`,
+ * forked after step 1 and joined before step 4 by events; the call is ordered
+ * on `stream` like any other. The library makes that stream and its two events
+ * on a host thread's first cascade call on a device and keeps them for the
+ * life of the process.
  * The result is the decode of pa_paged_decode up to floating-point rounding
  * (the same fp32 arithmetic summed in another order).
  *
