@@ -138,6 +138,14 @@ def test_cascade_argument_checks():
     assert call() == L.PA_ERR_INVALID_ARG                # no workspace
     assert "workspace" in L.last_error()
     assert call(B=0) == L.PA_OK                          # nothing to do
+    ws = ctypes.c_void_p(256 * 4096)                     # aligned, never dereferenced
+    big = 1 << 40
+    assert call(ws=ws, wsb=big, hq=32, hkv=16) == L.PA_ERR_UNSUPPORTED  # 8 x 2 stacked heads
+    assert call(ws=ctypes.c_void_p(256 * 4096 + 16), wsb=big) == L.PA_ERR_INVALID_ARG
+    assert "256-byte" in L.last_error()
+    assert call(ws=ws, wsb=1) == L.PA_ERR_INVALID_ARG    # workspace too small
+    assert call(ws=ws, wsb=big, dt=7) == L.PA_ERR_UNSUPPORTED
+    assert call(ws=ws, wsb=big, ng=-1) == L.PA_ERR_INVALID_ARG
     n = pa.pa_paged_decode_cascade_workspace_size(8, 32, 32, 128, 1200, 76, 1, 8, 62)
     assert n > 0
     assert pa.pa_paged_decode_cascade_workspace_size(8, 32, 32, 128, 1200, 76, 0, 1, 0) < n
