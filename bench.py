@@ -3,9 +3,12 @@
 One step = the whole decode-step path of one attention layer for a batch:
 copy-on-write block copies (when the workload has any), writing each new
 token's K/V into its slot, and paged decode attention with the split-KV merge.
-The default workload is the 7B-like MHA batch (64 sequences, 32 heads,
-head_dim 128, fp16, contexts U[128, 2048], 16384-block pool, one new token
-per sequence).
+The default (headline) workload is the largest single-GPU batch: long-context
+split-KV decode (8 sequences, contexts U[32768, 131072], 64 query / 8 KV heads,
+head_dim 128, bf16, 512-token split-KV partitions, one new token per sequence).
+Every other workload (tiny MHA, 7B-like MHA, GQA 32/8, prompts forked into
+samples sharing blocks) is timed at full size with the same protocol in the
+line's ``per_config`` object.
 
 Metric: KV-read GB/s (algorithmic bytes of the step / device time of the
 step; % of measured HBM peak alongside) and decode tokens/s.
@@ -52,7 +55,12 @@ if ROOT not in sys.path:
 
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode tokens/s"
 UNIT = "GB/s"
-DEFAULT_WORKLOAD = "mha_7b_fp16"
+DEFAULT_WORKLOAD = "long_ctx_split_kv"
+# every other workload is timed at full size in the line's per_config object
+PER_CONFIG = ("tiny_mha_d64", "mha_7b_fp16", "gqa_32_8_bf16", "prefix_share_cow",
+              "long_ctx_split_kv")
+# head shape of the serving-loop, prefix-cache and batching measurements
+LOOP_SHAPE = "mha_7b_fp16"
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -334,17 +342,20 @@ def _oracle_threads():
         return 1
 
 
-def time_oracle(wl, budget_s: float = 15.0, max_seq: int | None = None):
+def time_oracle(wl, budget_s: float = 15.0, max_seq: int | None = None, chunks=None,
+                setup_budget_s: float = 20.0):
     """Times the oracle's paged decode on the first sequences of the workload.
 
-    Grows the sample one sequence at a time until ``budget_s`` of oracle time is
-    used; a batch that ends first is decoded again, pass after pass, until the
-    budget is spent. Returns (GB/s, tokens/s, description, oracle seconds)."""
+    Grows the sample one sequence at a time (in chunks of 1, 2, 4, 8) until
+    ``budget_s`` of oracle time is used, or until building the sample's pools has
+    taken ``setup_budget_s`` (long contexts); a batch that ends first is decoded
+    again, pass after pass, until the budget is spent. ``chunks`` (from an earlier
+    call) reuses a built sample instead. Returns (GB/s, tokens/s, description,
+    oracle seconds, chunks)."""
     from oracle.attention import paged_decode
     import time as _t
     total_t, total_b, total_seq, total_tok = 0.0, 0, 0, 0
     limit = wl.num_seqs if max_seq is None else min(max_seq, wl.num_seqs)
-    chunks = []
 
     def run(sub, st):
         nonlocal total_t, total_b, total_seq, total_tok
@@ -356,15 +367,22 @@ def time_oracle(wl, budget_s: float = 15.0, max_seq: int | None = None):
         total_seq += sub.num_seqs
         total_tok += int(sub.context_lens.sum())
 
-    first, chunk = 0, 1
-    while first < limit and (total_seq == 0 or total_t < budget_s):
-        n = min(chunk, limit - first)
-        chunks.append(oracle_sample_setup_range(wl, first, n))
-        run(*chunks[-1])
-        first += n
-        chunk = min(8, chunk * 2)
-    unique = first
     passes = 1
+    if chunks is None:
+        chunks = []
+        first, chunk, setup_t = 0, 1, 0.0
+        while first < limit and (total_seq == 0 or (total_t < budget_s and
+                                                    setup_t < setup_budget_s)):
+            n = min(chunk, limit - first)
+            t0 = _t.perf_counter()
+            chunks.append(oracle_sample_setup_range(wl, first, n))
+            setup_t += _t.perf_counter() - t0
+            run(*chunks[-1])
+            first += n
+            chunk = min(8, chunk * 2)
+    else:
+        passes = 0
+    unique = sum(sub.num_seqs for sub, _ in chunks)
     while total_t < budget_s and passes < 100000:
         passes += 1
         for c in chunks:
@@ -374,10 +392,10 @@ def time_oracle(wl, budget_s: float = 15.0, max_seq: int | None = None):
     desc = (f"oracle paged_decode (fp64 NumPy) on {unique} of {wl.num_seqs} sequences, "
             f"{total_seq} sequence decodes in {passes} pass(es) ({total_tok} context tokens, "
             f"all {wl.num_q_heads} query heads), {total_t:.1f} s of oracle time")
-    return total_b / total_t / 1e9, total_seq / total_t, desc, total_t
+    return total_b / total_t / 1e9, total_seq / total_t, desc, total_t, chunks
 
 
-def time_oracle_one_thread(wl, budget_s: float = 5.0):
+def time_oracle_one_thread(wl, budget_s: float = 5.0, chunks=None):
     """The same oracle sample timing with the BLAS pool limited to one thread,
     so the multi-core figure can be read per core. None without threadpoolctl."""
     try:
@@ -385,7 +403,7 @@ def time_oracle_one_thread(wl, budget_s: float = 5.0):
     except ImportError:
         return None
     with threadpool_limits(limits=1):
-        v, tps, desc, _ = time_oracle(wl, budget_s=budget_s)
+        v, tps, desc, _, _ = time_oracle(wl, budget_s=budget_s, chunks=chunks)
     return {"value": round(v, 4), "unit": UNIT, "cores": 1, "sample": desc,
             "decode_tokens_per_s": round(tps, 3)}
 
@@ -724,15 +742,25 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
                     "k_scale 0.05, v_scale 0.02), CUDA events per launch"}
 
 
+def line_config(wl, args) -> dict:
+    """The ``config`` object of a bench line: the workload's name and shape. Both
+    arms print exactly this for the same arguments."""
+    cfg = {"workload": wl.name, **{k: v for k, v in wl.describe().items() if k != "workload"}}
+    pt = getattr(args, "partition_tokens", -1)
+    if pt is not None and pt >= 0:
+        cfg["partition_tokens"] = pt
+    return cfg
+
+
 def run_reference(args):
     rank, world, _ = _rank_info()
     if rank != 0:
         return 0
     import workloads
     wl = workloads.workload(args.workload)
-    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    per_step_budget = max(0.5, 90.0 / max(1, args.steps + args.warmup))
     # calibrate the sample size per step on one sequence
-    _, _, _, t1 = time_oracle(wl, budget_s=0.0, max_seq=1)
+    _, _, _, t1, _ = time_oracle(wl, budget_s=0.0, max_seq=1)
     nseq = int(max(1, min(wl.num_seqs, per_step_budget / max(t1, 1e-3))))
     from oracle.attention import paged_decode
     sub, st = oracle_sample_setup_range(wl, 0, nseq)
@@ -755,8 +783,7 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, **{k: v for k, v in wl.describe().items()
-                                           if k != "workload"}},
+        "config": line_config(wl, args),
         "decode_tokens_per_s": round(nseq * args.steps / el, 3),
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": _oracle_threads(),
                          "host_cpus": _host_cpus(),
@@ -766,6 +793,172 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _l2_flusher(wl, r, device, mode: str):
+    """The L2 rule between timed launches. Inputs several times larger than L2
+    need no flush (a cyclic scan larger than the cache leaves nothing to reuse);
+    smaller ones get a flush that READS a buffer larger than L2, outside the
+    timing events (a write flush would leave dirty lines whose write-back the
+    next kernel would pay for). Sequences sharing blocks read only their distinct
+    blocks from HBM, so those decide. Returns (flush callable, description)."""
+    import torch
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    read_bytes = unique_decode_bytes(wl, r) if r.groups is not None else decode_bytes(wl)
+    needed = read_bytes < 4 * l2_bytes if mode == "auto" else mode == "flush"
+    flush = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=device) if needed else None
+    sink = torch.empty(1, dtype=torch.int64, device=device)
+
+    def l2_flush():
+        if flush is not None:
+            torch.sum(flush, dim=0, out=sink)
+    desc = ("flushed between steps by reading a 256 MiB buffer, outside the timed events"
+            if needed else f"inputs larger than L2 ({read_bytes / 1e6:.0f} MB vs "
+                           f"{l2_bytes / 1e6:.0f} MB L2), no flush")
+    return l2_flush, desc
+
+
+def time_steps(r, steps: int, device, l2_flush):
+    """``steps`` steps (copy-on-write copies, cache writes, decode), each bracketed
+    by CUDA events on the launching stream, launched back to back behind a GPU
+    hold every HOLD_EVERY steps. Returns per-step (step seconds, decode seconds)."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        if k % HOLD_EVERY == 0:
+            gpu_hold(HOLD_EVERY * HOLD_PER_STEP_S)
+        l2_flush()
+        ev[k][0].record(stream)
+        r.copy_blocks()
+        r.reshape_and_cache()
+        ev[k][1].record(stream)
+        r.decode_step()
+        ev[k][2].record(stream)
+    torch.cuda.synchronize(device)
+    t_step = np.array([ev[k][0].elapsed_time(ev[k][2]) for k in range(steps)]) / 1e3
+    t_dec = np.array([ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)]) / 1e3
+    return t_step, t_dec
+
+
+def time_copy_blocks(r, wl, device):
+    """pa_copy_blocks of the step's copy-on-write pairs alone (idempotent: each pair
+    copies the same source), 20 launches back to back behind a GPU hold."""
+    import torch
+    if len(r.cow_pairs) == 0:
+        return None
+    stream = torch.cuda.current_stream(device)
+    ca, cb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_hold(20 * HOLD_PER_STEP_S)
+    ca.record(stream)
+    for _ in range(20):
+        r.copy_blocks()
+    cb.record(stream)
+    torch.cuda.synchronize(device)
+    tc = ca.elapsed_time(cb) / 20 / 1e3
+    nbytes = len(r.cow_pairs) * 2 * 2 * wl.num_kv_heads * 16 * wl.head_dim * wl.elem_bytes
+    return {"pairs": len(r.cow_pairs), "ms": round(tc * 1e3, 4), "bytes": nbytes,
+            "gbs": round(nbytes / tc / 1e9, 1),
+            "what": "pa_copy_blocks of the step's copy-on-write pairs (K and V, read + write), "
+                    "CUDA events around 20 back-to-back launches"}
+
+
+def time_plain_decode(r, device, l2_flush, cascade_s: float):
+    """For batches decoded through the cascade: the same batch through
+    pa_paged_decode, in which every sequence reads its shared blocks itself."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(20)]
+    gpu_hold(20 * HOLD_PER_STEP_S)
+    for a_, b_ in pe:
+        l2_flush()
+        a_.record(stream)
+        r.decode()
+        b_.record(stream)
+    torch.cuda.synchronize(device)
+    tp = float(np.mean([a_.elapsed_time(b_) for a_, b_ in pe])) / 1e3
+    return {"ms": round(tp * 1e3, 4), "cascade_speedup": round(tp / cascade_s, 3),
+            "what": "pa_paged_decode of the same batch (every sequence reads its "
+                    "shared blocks itself), CUDA events, mean of 20"}
+
+
+def decode_roofline(wl, r, dec_s: float, peak: float, peak_kind: str, read_ref):
+    """The decode call against the HBM roofline: algorithmic bytes per call (distinct
+    blocks for batches whose sequences share blocks) over its mean device time."""
+    db = decode_bytes(wl)
+    kernel = "paged_decode_kernel"
+    if r.groups is None and r.decode_launches() == 2:
+        kernel = "paged_decode_warp_parts_kernel + merge_partitions_kernel"
+    if r.groups is not None:
+        db = unique_decode_bytes(wl, r)
+        kernel = ("pa_paged_decode_cascade: cascade_prepare_kernel, paged_decode_kernel over "
+                  "the groups' shared blocks and over the own blocks, cascade_merge_kernel")
+    achieved = db / dec_s / 1e9
+    roof = {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": _traffic_for(wl.name + (":cascade" if r.groups is not None else "")),
+            "algorithmic_bytes_per_launch": db, "launch_ms": round(dec_s * 1e3, 4),
+            "peak_kind": peak_kind,
+            "pct_of_nominal_8tbs": round(100 * achieved / 8000.0, 2)}
+    if read_ref:
+        # the copy peak counts read + write bytes; a read-only stream measured in
+        # the same run is the tighter ceiling for a read-dominated kernel
+        roof["read_stream_gbs"] = round(read_ref, 1)
+        roof["frac_of_read_stream"] = round(achieved / read_ref, 4)
+    return roof
+
+
+def measure_config(name: str, args, device, peak: float, peak_kind: str, read_ref):
+    """One workload's step at full size (set-up, warm-up, ``args.steps`` timed steps
+    with the headline's protocol) and its decode against the roofline. For the
+    per-workload object of the bench line; everything it allocates is released."""
+    import torch
+    from paged_kv_cache_352_b200.runner import DecodeRunner
+    import workloads
+    wl = workloads.workload(name)
+    r = DecodeRunner(wl, device=device)
+    l2_flush, l2_desc = _l2_flusher(wl, r, device, "auto")
+    for _ in range(max(3, args.warmup)):
+        r.step()
+    torch.cuda.synchronize(device)
+    if r.error_bits():
+        raise RuntimeError(f"{name}: device error bits {r.error_bits()} during warm-up")
+    t_step, t_dec = time_steps(r, args.steps, device, l2_flush)
+    if r.error_bits():
+        raise RuntimeError(f"{name}: device error bits {r.error_bits()} during timing")
+    step_s, dec_s = float(t_step.mean()), float(t_dec.mean())
+    sb = step_bytes(wl, r)
+    if r.groups is not None:
+        sb = sb - decode_bytes(wl) + unique_decode_bytes(wl, r)
+    roof = decode_roofline(wl, r, dec_s, peak, peak_kind, read_ref)
+    res = {
+        "decode_us": {"mean": round(1e6 * dec_s, 2),
+                      "median": round(1e6 * float(np.median(t_dec)), 2),
+                      "min": round(1e6 * float(t_dec.min()), 2)},
+        "decode_gbs": roof["achieved"], "frac": roof["frac"],
+        "pct_of_nominal_8tbs": roof["pct_of_nominal_8tbs"],
+        "frac_of_read_stream": roof.get("frac_of_read_stream"),
+        "algorithmic_bytes": roof["algorithmic_bytes_per_launch"], "traffic": roof["traffic"],
+        "decode_tokens_per_s": round(wl.num_seqs / dec_s, 1),
+        "step_ms": round(1e3 * step_s, 4), "step_gbs": round(sb / step_s / 1e9, 2),
+        "step_tokens_per_s": round(wl.num_seqs / step_s, 1),
+        "kernel": roof["kernel"], "partition_tokens": r.partition_tokens, "l2": l2_desc,
+        "dtype": wl.dtype, "steps": args.steps,
+    }
+    if name == "tiny_mha_d64":
+        res["note"] = ("0.11 MB per launch: one launch latency, so the 70 % bandwidth target "
+                       "cannot apply")
+    if r.groups is not None:
+        res["logical_decode_gbs"] = round(decode_bytes(wl) / dec_s / 1e9, 2)
+        res["plain_decode"] = time_plain_decode(r, device, l2_flush, dec_s)
+        res["copy_blocks"] = time_copy_blocks(r, wl, device)
+    elif wl.num_seqs > 4:
+        res["fp8_kv"] = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak,
+                                           iters=max(args.steps, 20))
+    del r
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args):
@@ -782,26 +975,12 @@ def run_ours(args):
     from paged_kv_cache_352_b200 import build as pabuild
     pabuild.build()
     from paged_kv_cache_352_b200.runner import DecodeRunner, HostPipeline
+    import workloads
 
     wl = rank_workload(args.workload, rank, args.num_seqs, args.num_blocks)
     r = DecodeRunner(wl, device=device,
                      partition_tokens=args.partition_tokens if args.partition_tokens >= 0 else None)
-    stream = torch.cuda.current_stream(device)
-    # Inputs several times larger than L2 need no flush between steps (a cyclic
-    # scan larger than the cache leaves nothing to reuse). Smaller workloads get
-    # an L2 flush that READS a buffer larger than L2: a write flush would leave
-    # dirty lines whose write-back the next kernel would pay for.
-    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
-    # (sequences sharing blocks read only their distinct blocks from HBM: those decide)
-    read_bytes = unique_decode_bytes(wl, r) if r.groups is not None else decode_bytes(wl)
-    flush_needed = read_bytes < 4 * l2_bytes if args.l2 == "auto" else args.l2 == "flush"
-    flush = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=device) \
-        if flush_needed else None
-    flush_sink = torch.empty(1, dtype=torch.int64, device=device)
-
-    def l2_flush():
-        if flush is not None:
-            torch.sum(flush, dim=0, out=flush_sink)
+    l2_flush, l2_desc = _l2_flusher(wl, r, device, args.l2)
 
     for _ in range(max(3, args.warmup)):
         r.step()
@@ -816,24 +995,11 @@ def run_ours(args):
         return 0
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     _barrier(world)
     torch.cuda.synchronize(device)
     with ClockSampler(device) as clocks:
-        for k in range(K):
-            if k % HOLD_EVERY == 0:
-                gpu_hold(HOLD_EVERY * HOLD_PER_STEP_S)
-            l2_flush()
-            ev[k][0].record(stream)
-            r.copy_blocks()
-            r.reshape_and_cache()
-            ev[k][1].record(stream)
-            r.decode_step()
-            ev[k][2].record(stream)
-        torch.cuda.synchronize(device)
+        t_step, t_dec = time_steps(r, K, device, l2_flush)
     _barrier(world)
-    t_step = np.array([ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]) / 1e3
-    t_dec = np.array([ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]) / 1e3
     step_s = _max_over_ranks(float(t_step.mean()), world, device)
     dec_s = _max_over_ranks(float(t_dec.mean()), world, device)
     if r.error_bits():
@@ -843,39 +1009,9 @@ def run_ours(args):
                  "min": round(1e3 * float(t_dec.min()), 4)}
     # the step's cache writes (copy-on-write copies + new tokens) before the decode
     cache_write_ms = round(1e3 * float((t_step - t_dec).mean()), 4)
-    copy_blocks = None
-    if len(r.cow_pairs) > 0 and world == 1:
-        # copy-on-write copies alone (idempotent: each pair copies the same source)
-        ca, cb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        gpu_hold(20 * HOLD_PER_STEP_S)
-        ca.record(stream)
-        for _ in range(20):
-            r.copy_blocks()
-        cb.record(stream)
-        torch.cuda.synchronize(device)
-        tc = ca.elapsed_time(cb) / 20 / 1e3
-        nbytes = len(r.cow_pairs) * 2 * 2 * wl.num_kv_heads * 16 * wl.head_dim * wl.elem_bytes
-        copy_blocks = {"pairs": len(r.cow_pairs), "ms": round(tc * 1e3, 4),
-                       "bytes": nbytes, "gbs": round(nbytes / tc / 1e9, 1),
-                       "what": "pa_copy_blocks of the step's copy-on-write pairs (K and V, "
-                               "read + write), CUDA events around 20 back-to-back launches"}
-
-    plain_decode = None
-    if r.groups is not None and world == 1:
-        # the same batch through pa_paged_decode, which reads shared blocks per sequence
-        pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(20)]
-        gpu_hold(20 * HOLD_PER_STEP_S)
-        for a_, b_ in pe:
-            l2_flush()
-            a_.record(stream)
-            r.decode()
-            b_.record(stream)
-        torch.cuda.synchronize(device)
-        tp = float(np.mean([a_.elapsed_time(b_) for a_, b_ in pe])) / 1e3
-        plain_decode = {"ms": round(tp * 1e3, 4), "cascade_speedup": round(tp / dec_s, 3),
-                        "what": "pa_paged_decode of the same batch (every sequence reads its "
-                                "shared blocks itself), CUDA events, mean of 20"}
+    copy_blocks = time_copy_blocks(r, wl, device) if world == 1 else None
+    plain_decode = time_plain_decode(r, device, l2_flush, dec_s) \
+        if r.groups is not None and world == 1 else None
 
     # e2e: the same step fed from pinned host buffers, result read back to the
     # host, with the next step's input copy overlapping this step's kernels
@@ -897,27 +1033,11 @@ def run_ours(args):
     _barrier(world)
     e2e_s = _max_over_ranks(e_start.elapsed_time(e_end) / 1e3 / E, world, device)
 
-    extras = world == 1 and args.only == "all"
-    swap = measure_swap(wl, r, device) if extras else None
-    prefix_cache = measure_prefix_cache(wl, device) if extras else None
-    batching = measure_continuous_batching(wl, device) if extras else None
-    host_planning = measure_host_planning() if extras else None
-    batching_fp8 = measure_continuous_batching(wl, device, fp8_scales=(0.05, 0.02)) \
-        if extras else None
-    batching_prefix = None
-    if extras:
-        spt = shared_prompt_trace()
-        batching_prefix = {
-            "with_cache": measure_continuous_batching(wl, device, trace=spt, use_tokens=True),
-            "without_cache": measure_continuous_batching(wl, device, trace=spt),
-        }
     peak, peak_kind = _peaks()
-    fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) if extras else None
-
+    read_ref = read_stream_gbs(device) if world == 1 else None
     sb = step_bytes(wl, r)
     db = decode_bytes(wl)
     effective = None
-    kernel = "paged_decode_kernel"
     if r.groups is not None:
         # Sequences share blocks: the bytes that must leave HBM are those of the
         # distinct blocks read; the logical rate is reported beside them.
@@ -926,15 +1046,50 @@ def run_ours(args):
                      "step_gbs_logical": round(world * sb / step_s / 1e9, 2),
                      "logical_decode_bytes": db, "unique_decode_bytes": ub}
         sb = sb - db + ub
-        db = ub
-        kernel = ("pa_paged_decode_cascade: cascade_prepare_kernel, paged_decode_kernel over "
-                  "the groups' shared blocks and over the own blocks, cascade_merge_kernel")
     value = world * sb / step_s / 1e9
-    achieved = db / dec_s / 1e9
-    traffic = _traffic_for(wl.name + (":cascade" if r.groups is not None else ""))
-    read_ref = read_stream_gbs(device) if world == 1 else None
+    roofline = decode_roofline(wl, r, dec_s, peak, peak_kind, read_ref)
     csum = clocks.summary()
     launches_per_step = r.launches_per_step()
+    fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) \
+        if world == 1 and args.only == "all" and r.groups is None else None
+    e2e = {"value": round(world * sb / e2e_s / 1e9, 2), "unit": UNIT,
+           "h2d_bytes_per_step": hs.h2d_bytes, "d2h_bytes_per_step": hs.d2h_bytes,
+           "ms_per_step": round(e2e_s * 1e3, 4),
+           "what": "the step through the C interface fed from pinned host buffers (queries, new "
+                   "keys/values, slot mapping, block tables, lengths, order copied host -> device "
+                   "every step, output copied back); the block tables and slots are the "
+                   "workload's, planned once before timing (host planning per step is measured "
+                   "in host_planning)"}
+    del hs
+    extras = world == 1 and args.only == "all"
+    # 512 MiB of whole blocks each way between the pool and pinned host memory
+    blk_bytes = 2 * r.k_cache[0].numel() * r.k_cache.element_size()
+    swap = measure_swap(wl, r, device, nblocks=(512 << 20) // blk_bytes) if extras else None
+    del r
+    torch.cuda.empty_cache()
+
+    # every other workload at full size, with the same protocol (one GPU only)
+    per_config = None
+    if extras:
+        per_config = {}
+        for name in PER_CONFIG:
+            if name != wl.name:
+                per_config[name] = measure_config(name, args, device, peak, peak_kind, read_ref)
+    # the serving-loop extras run on 7B-like MHA heads (32/32, d 128, fp16)
+    loop_wl = workloads.workload(LOOP_SHAPE) if extras else None
+    prefix_cache = measure_prefix_cache(loop_wl, device) if extras else None
+    batching = measure_continuous_batching(loop_wl, device) if extras else None
+    host_planning = measure_host_planning() if extras else None
+    batching_fp8 = measure_continuous_batching(loop_wl, device, fp8_scales=(0.05, 0.02)) \
+        if extras else None
+    batching_prefix = None
+    if extras:
+        spt = shared_prompt_trace()
+        batching_prefix = {
+            "with_cache": measure_continuous_batching(loop_wl, device, trace=spt,
+                                                      use_tokens=True),
+            "without_cache": measure_continuous_batching(loop_wl, device, trace=spt),
+        }
 
     if world > 1:
         import torch.distributed as dist
@@ -947,14 +1102,9 @@ def run_ours(args):
         "warmup": max(3, args.warmup), "ms_per_step": round(step_s * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.name, **{k: v for k, v in wl.describe().items()
-                                           if k != "workload"},
-                   "partition_tokens": r.partition_tokens,
-                   "l2": ("flushed between steps by reading a 256 MiB buffer, outside the "
-                          "timed events" if flush_needed else
-                          f"inputs larger than L2 ({read_bytes / 1e6:.0f} MB vs "
-                          f"{l2_bytes / 1e6:.0f} MB L2), no flush"),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": line_config(wl, args),
+        "l2_policy": l2_desc,
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
         "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
@@ -964,31 +1114,26 @@ def run_ours(args):
         "decode_only_tokens_per_s": round(world * wl.num_seqs / dec_s, 1),
         "bytes_per_step": sb,
         "shared_blocks": effective, "plain_decode": plain_decode,
-        "roofline": {"bound": "hbm", "kernel": kernel,
-                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes_per_launch": db,
-                     "launch_ms": round(dec_s * 1e3, 4), "peak_kind": peak_kind},
-        "e2e": {"value": round(world * sb / e2e_s / 1e9, 2), "unit": UNIT,
-                "h2d_bytes_per_step": hs.h2d_bytes, "d2h_bytes_per_step": hs.d2h_bytes,
-                "ms_per_step": round(e2e_s * 1e3, 4)},
+        "roofline": roofline,
+        "e2e": e2e,
         "gpu_launches": K * launches_per_step,
+        "per_config": per_config,
+        "fp8_kv": fp8,
         "swap": swap,
         "prefix_cache": prefix_cache,
         "continuous_batching": batching,
         "host_planning": host_planning,
         "continuous_batching_fp8": batching_fp8,
         "continuous_batching_shared_prompts": batching_prefix,
-        "fp8_kv": fp8,
         "clocks": csum,
     }
     if world == 1 and not args.no_cpu_baseline:
-        v, tps, desc, _ = time_oracle(wl, budget_s=args.cpu_budget)
+        v, tps, desc, _, chunks = time_oracle(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": _oracle_threads(),
                                 "host_cpus": _host_cpus(),
                                 "kind": "oracle", "sample": desc,
                                 "decode_tokens_per_s": round(tps, 3)}
-        one = time_oracle_one_thread(wl, budget_s=min(5.0, args.cpu_budget / 3))
+        one = time_oracle_one_thread(wl, budget_s=min(5.0, args.cpu_budget / 3), chunks=chunks)
         if one is not None:
             line["cpu_baseline"]["one_thread"] = one
     print(json.dumps(line), flush=True)

@@ -206,13 +206,18 @@ class DecodeRunner:
         self.reshape_and_cache()
         return self.decode_step()
 
-    def launches_per_step(self) -> int:
-        wl = self.wl
-        _, _, decode = L.pa_paged_decode_plan(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
-                                              wl.head_dim, wl.max_context_len,
-                                              self.partition_tokens or 0, ordered=True)
+    def decode_launches(self) -> int:
+        """Kernel launches of the step's decode call."""
         if self.groups is not None:
-            decode = 4  # prepare, prefix decode, own-block decode, merge
+            return 4  # prepare, prefix decode, own-block decode, merge
+        wl = self.wl
+        _, _, n = L.pa_paged_decode_plan(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                         wl.head_dim, wl.max_context_len,
+                                         self.partition_tokens or 0, ordered=True)
+        return n
+
+    def launches_per_step(self) -> int:
+        decode = self.decode_launches()
         return int(len(self.cow_pairs) > 0) * -(-len(self.cow_pairs) // 1024) + \
             int(len(self.step_slots_host) > 0) + decode
 

@@ -91,3 +91,26 @@ def test_byte_accounting_matches_definition():
     qo = 2 * 4 * 4 * 64 * 2
     tables = 4 * (1 + 1 + 2 + 5)
     assert bench.decode_bytes(wl) == kv + qo + tables + 4 * 4
+
+
+def test_both_arms_print_the_same_config(monkeypatch, capsys):
+    """The repo arm and the reference arm describe the workload with one function,
+    so the driver sees the same ``config`` for the same arguments."""
+    import json
+    import workloads
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    args = type("A", (), {"workload": "tiny_mha_d64", "steps": 1, "warmup": 0,
+                          "partition_tokens": -1})
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["config"] == bench.line_config(workloads.workload("tiny_mha_d64"), args)
+    assert "l2" not in line["config"] and "parallelism" not in line["config"]
+    src = open(bench.__file__).read()
+    assert src.count('"config": line_config(wl, args)') == 2
+
+
+def test_default_workload_is_the_largest_single_gpu_batch():
+    import workloads
+    sizes = {n: bench.decode_bytes(workloads.workload(n)) for n in bench.PER_CONFIG}
+    assert bench.DEFAULT_WORKLOAD == max(sizes, key=sizes.get) == "long_ctx_split_kv"
