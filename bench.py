@@ -580,7 +580,7 @@ def measure_host_planning(num_requests: int = 1000, num_blocks: int = 8192,
 def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks: int = 8192,
                                 max_num_seqs: int = 256, host_blocks: int = 4096,
                                 max_model_len: int = 2048, fp8_scales=None, trace=None,
-                                use_tokens: bool = False):
+                                use_tokens: bool = False, cascade=None):
     """The iteration-level batching loop end to end on one GPU: the library's
     scheduler plans each step and its executor runs swap-out/in, prefill writes,
     copy-on-write, new-token writes and decode (7B-like heads of ``wl``). Keys,
@@ -590,7 +590,9 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     to what a contiguous ``max_model_len`` reservation per sequence would give.
     ``fp8_scales = (k_scale, v_scale)`` runs the same trace over E4M3 caches;
     ``trace`` replaces the default trace, and ``use_tokens`` submits its token ids
-    so that admission goes through the prefix cache."""
+    so that admission goes through the prefix cache. ``cascade`` sets the
+    executor's mode for sequences sharing blocks (PA_SCHED_CASCADE_*; default
+    auto)."""
     import torch
     from paged_kv_cache_352_b200 import _lib as L
     trace = continuous_batching_trace(num_requests) if trace is None else trace
@@ -602,6 +604,8 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     for t in trace:
         sched.submit(*t[:5], tokens=t[5] if use_tokens else None)
     sched.attach(hq, hkv, d, dt, max_model_len, fp8_scales=fp8_scales)
+    if cascade is not None:
+        sched.set_cascade(cascade)
     cdt = torch.uint8 if fp8_scales else dt
     kc = torch.zeros(num_blocks, hkv, 16, d, dtype=cdt, device=device)
     vc = torch.zeros_like(kc)
@@ -613,7 +617,7 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     err = torch.zeros(1, dtype=torch.int32, device=device)
     scale = 1.0 / math.sqrt(d)
     tot = {"steps": 0, "tokens": 0, "prefill_tokens": 0, "preempt": 0, "swap_blocks": 0,
-           "cow": 0, "context": 0, "cached": 0}
+           "cow": 0, "context": 0, "cached": 0, "cascade_steps": 0, "saved_blocks": 0}
     util, contiguous = [], []
     row_bytes = hkv * d * (1 if fp8_scales else 2)   # cached bytes of one (token, K or V) row
     torch.cuda.synchronize(device)
@@ -624,6 +628,9 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
     while not sched.idle():
         c = sched.step()
         sched.execute(kc, vc, hk, hv, bank, bank, bank, bank, qbank, out, scale, dev_error=err)
+        ng, saved = sched.last_cascade()
+        tot["cascade_steps"] += ng > 0
+        tot["saved_blocks"] += saved
         tot["steps"] += 1
         tot["tokens"] += c.num_seqs
         tot["prefill_tokens"] += c.num_prefill
@@ -656,6 +663,8 @@ def measure_continuous_batching(wl, device, num_requests: int = 1000, num_blocks
         "cached_prompt_tokens": tot["cached"],
         "preemptions": tot["preempt"], "swapped_blocks": tot["swap_blocks"],
         "cow_copies": tot["cow"],
+        "cascade_steps": tot["cascade_steps"],
+        "cascade_saved_block_reads": tot["saved_blocks"],
         "kv_utilization": round(float(np.mean(util)), 4) if util else None,
         "contiguous_reservation_utilization": (round(float(np.mean(contiguous)), 4)
                                                if contiguous else None),
@@ -892,8 +901,9 @@ def decode_roofline(wl, r, dec_s: float, peak: float, peak_kind: str, read_ref):
         kernel = "paged_decode_warp_parts_kernel + merge_partitions_kernel"
     if r.groups is not None:
         db = unique_decode_bytes(wl, r)
-        kernel = ("pa_paged_decode_cascade: cascade_prepare_kernel, paged_decode_kernel over "
-                  "the groups' shared blocks and over the own blocks, cascade_merge_kernel")
+        kernel = ("pa_paged_decode_cascade: cascade_prepare_kernel, cascade_decode_kernel (the "
+                  "groups' shared blocks and every sequence's own blocks in one launch), "
+                  "cascade_merge_kernel")
     achieved = db / dec_s / 1e9
     roof = {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -1078,16 +1088,24 @@ def run_ours(args):
     # the serving-loop extras run on 7B-like MHA heads (32/32, d 128, fp16)
     loop_wl = workloads.workload(LOOP_SHAPE) if extras else None
     prefix_cache = measure_prefix_cache(loop_wl, device) if extras else None
-    batching = measure_continuous_batching(loop_wl, device) if extras else None
+
+    def loop(**kw):
+        """The loop with the executor's default cascade rule, and the generated
+        tokens/s of the same trace with the cascade off beside it."""
+        res = measure_continuous_batching(loop_wl, device, **kw)
+        import paged_kv_cache_352_b200 as pa
+        off = measure_continuous_batching(loop_wl, device, cascade=pa.PA_SCHED_CASCADE_OFF, **kw)
+        res["cascade_off"] = {"value": off["value"], "ms_per_step": off["ms_per_step"]}
+        return res
+
+    batching = loop() if extras else None
     host_planning = measure_host_planning() if extras else None
-    batching_fp8 = measure_continuous_batching(loop_wl, device, fp8_scales=(0.05, 0.02)) \
-        if extras else None
+    batching_fp8 = loop(fp8_scales=(0.05, 0.02)) if extras else None
     batching_prefix = None
     if extras:
         spt = shared_prompt_trace()
         batching_prefix = {
-            "with_cache": measure_continuous_batching(loop_wl, device, trace=spt,
-                                                      use_tokens=True),
+            "with_cache": loop(trace=spt, use_tokens=True),
             "without_cache": measure_continuous_batching(loop_wl, device, trace=spt),
         }
 

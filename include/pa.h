@@ -83,6 +83,27 @@ const char* pa_last_error(void);
 int pa_version(void);
 
 /* ---------------------------------------------------------------------------
+ * pa_test_stall_next_decode — test hook for the device-side failure path.
+ *
+ * The pages tie failure handling to memory running short ("PagedAttention: The
+ * vLLM Paper", "Implementation Essentials", preemption); on the device, every
+ * on-chip wait of the decode kernels is bounded and gives up with
+ * PA_DEVERR_WAIT_TIMEOUT instead of spinning. This call lets a test drive that
+ * path without a fault: the next decode kernel launch in the process (by any
+ * pa_paged_decode* call) has each warp arm the barrier of its first block
+ * without issuing the block's copy, and lowers the limit of the main loop's
+ * waits to wait_limit_ns. That wait runs out, the warp reports
+ * PA_DEVERR_WAIT_TIMEOUT, still waits (with the normal 1 s limit) for the
+ * copies it did issue, and the kernel returns; that launch's output is invalid.
+ * The request applies to one launch and is then cleared.
+ *
+ *   wait_limit_ns   in [1000, 1e8] (1 us .. 100 ms), else PA_ERR_INVALID_ARG
+ *
+ * Not for production use: it exists so that tests can check the error path.
+ * ------------------------------------------------------------------------- */
+int pa_test_stall_next_decode(unsigned long long wait_limit_ns);
+
+/* ---------------------------------------------------------------------------
  * pa_reshape_and_cache — store new tokens' keys and values in their slots.
  *
  * Every generated token's K/V is cached so decode need not recompute it
@@ -282,8 +303,14 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
  *
  * The call allocates nothing:
  *   - The first call on each device looks up the array's device address and
- *     caches it. Make that first call, with the device current, before any
- *     stream capture on that device.
+ *     caches it with the id of the device's current context. A call that finds
+ *     another context current (after cudaDeviceReset, for example) looks the
+ *     address up again, since a new context holds the array elsewhere. Make the
+ *     first call on a device, and the first after a reset, with the device
+ *     current and before any stream capture on that device.
+ *   - The call runs on the current device. out, q, both caches, the tables and
+ *     the lengths must be device memory of that device and `stream` one of its
+ *     streams; otherwise it returns PA_ERR_INVALID_ARG and launches nothing.
  *   - Each call clears the array's merge counters with an async memset on
  *     `stream`, then launches the decode kernel.
  *   - All calls share the one array, so calls whose kernels overlap on the GPU
@@ -641,6 +668,33 @@ int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim
 int pa_sched_attach_fp8(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim, int dtype,
                         int max_context_len, float k_scale, float v_scale);
 
+/* Decode of sequences that share leading blocks, inside the executor. Samples
+ * forked from one prompt share its full blocks, and so do requests whose
+ * prompts were found in the prefix cache ("PagedAttention: The vLLM Paper",
+ * "Implementation Essentials", prefix sharing). The executor groups a step's
+ * batch with pa_bm_prefix_groups (8 / G members per group, G query heads per KV
+ * head; no grouping when G = 8) and, when a group exists, decodes the step with
+ * pa_paged_decode_cascade (pa_paged_decode_cascade_fp8 over 8-bit caches),
+ * which reads each group's shared blocks once:
+ *   PA_SCHED_CASCADE_OFF   never (always pa_paged_decode)
+ *   PA_SCHED_CASCADE_ON    whenever the batch has a group
+ *   PA_SCHED_CASCADE_AUTO  (default) when the shared blocks it reads once
+ *                          instead of once per member from another request
+ *                          than the group's first add up to 32 MiB (about the
+ *                          cost of its two extra launches). Samples of one
+ *                          request are left out: they have equal contexts, so
+ *                          the plain decode runs them side by side and L2
+ *                          serves their shared prompt once.
+ * The results equal the plain decode's up to floating-point rounding order.
+ * pa_sched_attach sizes the cascade's workspace once. pa_sched_last_cascade
+ * reports the groups the last executed step decoded through the cascade (0 when
+ * it used pa_paged_decode) and the block reads that saved. */
+#define PA_SCHED_CASCADE_OFF 0
+#define PA_SCHED_CASCADE_ON 1
+#define PA_SCHED_CASCADE_AUTO 2
+int pa_sched_set_cascade(pa_sched* s, int mode);
+int pa_sched_last_cascade(const pa_sched* s, int* num_groups, int64_t* shared_blocks);
+
 /* Runs the last planned step on `stream` in device order: pa_swap_blocks for
  * the swap pairs (device pool k_cache/v_cache <-> pinned host pool
  * host_k/host_v, [num_host_blocks][Hkv][16][d]; may be NULL when the plan has
@@ -648,7 +702,7 @@ int pa_sched_attach_fp8(pa_sched* s, int num_q_heads, int num_kv_heads, int head
  * ([num_prefill][Hkv][d], contiguous, device), pa_copy_blocks, pa_reshape_and_cache
  * of key/value ([num_writes][Hkv][d]), then pa_paged_decode of q
  * ([num_seqs][Hq][d]) into out ([num_seqs][Hq][d]) through the plan's tables,
- * longest context first. Row i of each input belongs to write / sequence i of
+ * longest context first (or the cascade, above, when sequences share blocks). Row i of each input belongs to write / sequence i of
  * the plan. Block tables, context lengths, slots and the order reach the device
  * through the pinned ring with one host-to-device copy per step; the call
  * waits only for the copy that last used the ring slot. Never synchronises the

@@ -20,6 +20,9 @@ from ._lib import (  # noqa: F401
     PA_FP8_E4M3,
     PA_PREEMPT_RECOMPUTE,
     PA_PREEMPT_SWAP,
+    PA_SCHED_CASCADE_AUTO,
+    PA_SCHED_CASCADE_OFF,
+    PA_SCHED_CASCADE_ON,
     PrefixGroups,
     Scheduler,
     cascade_workspace,
@@ -32,6 +35,8 @@ from ._lib import (  # noqa: F401
     pa_paged_decode_cascade,
     pa_paged_decode_cascade_workspace_size,
     pa_paged_decode_fp8,
+    pa_paged_decode_noalloc,
+    pa_paged_decode_plan,
     pa_paged_decode_workspace_size,
     pa_reshape_and_cache,
     pa_reshape_and_cache_fp8,

@@ -51,6 +51,7 @@ _vp = ctypes.c_void_p
 _SIGS = {
     "pa_last_error": (ctypes.c_char_p, []),
     "pa_version": (_c_int, []),
+    "pa_test_stall_next_decode": (_c_int, [ctypes.c_ulonglong]),
     "pa_reshape_and_cache": (_c_int, [_vp, _vp, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int,
                                       _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -127,6 +128,9 @@ _SIGS = {
     "pa_sched_attach": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "pa_sched_attach_fp8": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
                                      ctypes.c_float]),
+    "pa_sched_set_cascade": (_c_int, [_vp, _c_int]),
+    "pa_sched_last_cascade": (_c_int, [_vp, ctypes.POINTER(_c_int),
+                                       ctypes.POINTER(ctypes.c_int64)]),
     "pa_sched_execute": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                   ctypes.c_float, _vp, _vp]),
 }
@@ -191,6 +195,17 @@ def _dev_ptr(t, name, dtype=None, contiguous=True):
     return t.data_ptr()
 
 
+def _device(*tensors):
+    """Context in which a call runs: the device of the first CUDA tensor given,
+    made current, so that the library's kernels launch on the GPU that holds the
+    data and the default stream is that GPU's current stream."""
+    import contextlib
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return _torch().cuda.device(t.device)
+    return contextlib.nullcontext()
+
+
 def _stream(stream):
     torch = _torch()
     if stream is None:
@@ -224,22 +239,24 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, dev_error=N
         raise PAError(PA_ERR_INVALID_ARG, "key/value rows must be dense per token")
     if slot_mapping.shape != (T,):
         raise PAError(PA_ERR_INVALID_ARG, "slot_mapping must be [T]")
-    _check(lib().pa_reshape_and_cache(
-        _dev_ptr(key, "key", k_cache.dtype, contiguous=False),
-        _dev_ptr(value, "value", k_cache.dtype, contiguous=False),
-        key.stride(0), value.stride(0),
-        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
-        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, hkv, d, bs, nb,
-        dtype_code(k_cache), _dev_ptr(dev_error, "dev_error", torch.int32), _stream(stream)))
+    with _device(k_cache):
+        _check(lib().pa_reshape_and_cache(
+            _dev_ptr(key, "key", k_cache.dtype, contiguous=False),
+            _dev_ptr(value, "value", k_cache.dtype, contiguous=False),
+            key.stride(0), value.stride(0),
+            _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+            _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, hkv, d, bs, nb,
+            dtype_code(k_cache), _dev_ptr(dev_error, "dev_error", torch.int32), _stream(stream)))
 
 
 def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
     """Copy blocks ``pairs[i, 0] -> pairs[i, 1]`` (host int64 array ``[n, 2]``)."""
     nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
     p = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
-    _check(lib().pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
-                                p.ctypes.data if len(p) else None, len(p), hkv, d, bs, nb,
-                                dtype_code(k_cache), _stream(stream)))
+    with _device(k_cache):
+        _check(lib().pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+                                    p.ctypes.data if len(p) else None, len(p), hkv, d, bs, nb,
+                                    dtype_code(k_cache), _stream(stream)))
 
 
 def _pool_ptr(t, name):
@@ -259,10 +276,11 @@ def pa_swap_blocks(src_k, src_v, dst_k, dst_v, pairs, stream=None):
     if (hkv, bs, d) != (hkv2, bs2, d2) or src_k.dtype != dst_k.dtype:
         raise PAError(PA_ERR_INVALID_ARG, "source and destination pools differ in layout")
     p = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
-    _check(lib().pa_swap_blocks(_pool_ptr(src_k, "src_k"), _pool_ptr(src_v, "src_v"), s_nb,
-                                _pool_ptr(dst_k, "dst_k"), _pool_ptr(dst_v, "dst_v"), d_nb,
-                                p.ctypes.data if len(p) else None, len(p), hkv, d, bs,
-                                dtype_code(src_k), _stream(stream)))
+    with _device(src_k, dst_k):
+        _check(lib().pa_swap_blocks(_pool_ptr(src_k, "src_k"), _pool_ptr(src_v, "src_v"), s_nb,
+                                    _pool_ptr(dst_k, "dst_k"), _pool_ptr(dst_v, "dst_v"), d_nb,
+                                    p.ctypes.data if len(p) else None, len(p), hkv, d, bs,
+                                    dtype_code(src_k), _stream(stream)))
 
 
 def pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
@@ -325,13 +343,14 @@ def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_co
     ws_bytes = 0
     if workspace is not None:
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().pa_paged_decode(
-        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
-        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
-        _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
-        int(partition_tokens), _dev_ptr(workspace, "workspace"), ws_bytes,
-        _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
+    with _device(q):
+        _check(lib().pa_paged_decode(
+            _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
+            block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
+            _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+            int(partition_tokens), _dev_ptr(workspace, "workspace"), ws_bytes,
+            _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(k_cache), _stream(stream)))
 
 
 def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
@@ -349,12 +368,14 @@ def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale
         raise PAError(PA_ERR_INVALID_ARG, "key/value rows must be dense per token")
     if value.dtype != key.dtype or slot_mapping.shape != (T,):
         raise PAError(PA_ERR_INVALID_ARG, "value must match key; slot_mapping must be [T]")
-    _check(lib().pa_reshape_and_cache_fp8(
-        _dev_ptr(key, "key", contiguous=False), _dev_ptr(value, "value", contiguous=False),
-        key.stride(0), value.stride(0), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
-        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, hkv, d, bs, nb, dtype_code(key),
-        float(k_scale), float(v_scale), _dev_ptr(dev_error, "dev_error", torch.int32),
-        _stream(stream)))
+    with _device(k_cache):
+        _check(lib().pa_reshape_and_cache_fp8(
+            _dev_ptr(key, "key", contiguous=False), _dev_ptr(value, "value", contiguous=False),
+            key.stride(0), value.stride(0), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"),
+            _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, hkv, d, bs, nb, dtype_code(key),
+            float(k_scale), float(v_scale), _dev_ptr(dev_error, "dev_error", torch.int32),
+            _stream(stream)))
 
 
 def pa_paged_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
@@ -372,13 +393,15 @@ def pa_paged_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, ma
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().pa_paged_decode_fp8(
-        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
-        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
-        _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
-        float(k_scale), float(v_scale), int(partition_tokens), _dev_ptr(workspace, "workspace"),
-        ws_bytes, _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(q), _stream(stream)))
+    with _device(q):
+        _check(lib().pa_paged_decode_fp8(
+            _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
+            block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
+            _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+            float(k_scale), float(v_scale), int(partition_tokens), _dev_ptr(workspace, "workspace"),
+            ws_bytes, _dev_ptr(dev_error, "dev_error", torch.int32), dtype_code(q),
+            _stream(stream)))
 
 
 def pa_paged_decode_cascade_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
@@ -450,23 +473,25 @@ def pa_paged_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens
         raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
     if groups.dev is None or groups.seq_group.shape != (B,):
         raise PAError(PA_ERR_INVALID_ARG, "groups must describe this batch and be on the device")
-    members, prefix, sgroup, smember = groups.dev
-    i32 = torch.int32
-    head = [_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
-            _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", i32),
-            block_tables.shape[1], _dev_ptr(context_lens, "context_lens", i32), B,
-            int(max_context_len), hq, hkv, d, bs, nb, float(scale)]
-    tail = [_dev_ptr(members, "group_members", i32), _dev_ptr(prefix, "group_prefix_blocks", i32),
-            _dev_ptr(sgroup, "seq_group", i32), _dev_ptr(smember, "seq_member", i32),
-            groups.num_groups, groups.group_size, groups.max_prefix_blocks,
-            _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-            _dev_ptr(dev_error, "dev_error", i32), dtype_code(q), _stream(stream)]
-    if fp8:
-        if k_scale is None or v_scale is None:
-            raise PAError(PA_ERR_INVALID_ARG, "E4M3 caches need k_scale and v_scale")
-        _check(lib().pa_paged_decode_cascade_fp8(*head, float(k_scale), float(v_scale), *tail))
-    else:
-        _check(lib().pa_paged_decode_cascade(*head, *tail))
+    with _device(q):
+        members, prefix, sgroup, smember = groups.dev
+        i32 = torch.int32
+        head = [_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", i32),
+                block_tables.shape[1], _dev_ptr(context_lens, "context_lens", i32), B,
+                int(max_context_len), hq, hkv, d, bs, nb, float(scale)]
+        tail = [_dev_ptr(members, "group_members", i32),
+                _dev_ptr(prefix, "group_prefix_blocks", i32), _dev_ptr(sgroup, "seq_group", i32),
+                _dev_ptr(smember, "seq_member", i32),
+                groups.num_groups, groups.group_size, groups.max_prefix_blocks,
+                _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                _dev_ptr(dev_error, "dev_error", i32), dtype_code(q), _stream(stream)]
+        if fp8:
+            if k_scale is None or v_scale is None:
+                raise PAError(PA_ERR_INVALID_ARG, "E4M3 caches need k_scale and v_scale")
+            _check(lib().pa_paged_decode_cascade_fp8(*head, float(k_scale), float(v_scale), *tail))
+        else:
+            _check(lib().pa_paged_decode_cascade(*head, *tail))
 
 
 NOALLOC_WORKSPACE_BYTES = 16 << 20
@@ -488,7 +513,9 @@ def pa_paged_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens
     For callers that cannot allocate device memory: the split-KV scratch comes
     from a fixed array built into libpa (``NOALLOC_WORKSPACE_BYTES`` per GPU).
     Calls share that array, so calls that overlap on the GPU must not be issued
-    (use one stream). Batches that need more scratch raise ``PAError``.
+    (use one stream). Batches that need more scratch raise ``PAError``. The call
+    runs on the device of ``q`` (made current for it), and the library refuses
+    tensors or a stream of any other device.
     """
     torch = _torch()
     nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
@@ -498,13 +525,14 @@ def pa_paged_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens
                                           "cache's dtype")
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise PAError(PA_ERR_INVALID_ARG, "block_tables must be [B, max_blocks], context_lens [B]")
-    _check(lib().pa_paged_decode_noalloc(
-        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
-        block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
-        _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
-        int(partition_tokens), _dev_ptr(dev_error, "dev_error", torch.int32),
-        dtype_code(k_cache), _stream(stream)))
+    with _device(q):
+        _check(lib().pa_paged_decode_noalloc(
+            _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", torch.int32),
+            block_tables.shape[1], _dev_ptr(context_lens, "context_lens", torch.int32),
+            _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+            int(partition_tokens), _dev_ptr(dev_error, "dev_error", torch.int32),
+            dtype_code(k_cache), _stream(stream)))
 
 
 # --------------------------------------------------------------------------
@@ -696,6 +724,9 @@ class BlockManager:
 # --------------------------------------------------------------------------
 
 PA_SCHED_MAX_SAMPLES = 64
+PA_SCHED_CASCADE_OFF = 0
+PA_SCHED_CASCADE_ON = 1
+PA_SCHED_CASCADE_AUTO = 2
 PA_PREEMPT_SWAP = 0
 PA_PREEMPT_RECOMPUTE = 1
 
@@ -839,6 +870,18 @@ class Scheduler:
         self.io_dtype = code
         self.fp8 = fp8_scales is not None
 
+    def set_cascade(self, mode: int) -> None:
+        """When the executor decodes sequences that share leading blocks through
+        the cascade: PA_SCHED_CASCADE_OFF, _ON or _AUTO (the default)."""
+        _check(self._lib.pa_sched_set_cascade(self._h, int(mode)))
+
+    def last_cascade(self):
+        """(groups decoded through the cascade in the last executed step, block
+        reads that saved); (0, 0) when that step used the plain decode."""
+        ng, saved = _c_int(0), ctypes.c_int64(0)
+        _check(self._lib.pa_sched_last_cascade(self._h, ctypes.byref(ng), ctypes.byref(saved)))
+        return ng.value, saved.value
+
     def execute(self, k_cache, v_cache, host_k, host_v, prefill_key, prefill_value, key, value,
                 q, out, scale: float, dev_error=None, stream=None) -> None:
         """Run the last planned step (pa_sched_execute). Inputs are device tensors
@@ -850,10 +893,12 @@ class Scheduler:
         cdt = k_cache.dtype
         dt = q.dtype
         host = lambda t, n: None if t is None else _pool_ptr(t, n)
-        _check(self._lib.pa_sched_execute(
-            self._h, _dev_ptr(k_cache, "k_cache", cdt), _dev_ptr(v_cache, "v_cache", cdt),
-            host(host_k, "host_k"), host(host_v, "host_v"),
-            _dev_ptr(prefill_key, "prefill_key", dt), _dev_ptr(prefill_value, "prefill_value", dt),
-            _dev_ptr(key, "key", dt), _dev_ptr(value, "value", dt), _dev_ptr(q, "q", dt),
-            _dev_ptr(out, "out", dt), scale, _dev_ptr(dev_error, "dev_error", torch.int32),
-            _stream(stream)))
+        with _device(k_cache):
+            _check(self._lib.pa_sched_execute(
+                self._h, _dev_ptr(k_cache, "k_cache", cdt), _dev_ptr(v_cache, "v_cache", cdt),
+                host(host_k, "host_k"), host(host_v, "host_v"),
+                _dev_ptr(prefill_key, "prefill_key", dt),
+                _dev_ptr(prefill_value, "prefill_value", dt),
+                _dev_ptr(key, "key", dt), _dev_ptr(value, "value", dt), _dev_ptr(q, "q", dt),
+                _dev_ptr(out, "out", dt), scale, _dev_ptr(dev_error, "dev_error", torch.int32),
+                _stream(stream)))

@@ -12,13 +12,15 @@ namespace pa {
 namespace {
 
 // Second pass of the warp-per-partition split: one CTA per (sequence, query
-// head) merges that row's partition states in logical order,
+// head) merges that row's states in logical order,
 //   out = sum_p exp2(m_p - M) acc_p / sum_p exp2(m_p - M) l_p,  M = max_p m_p,
-// each thread owning a float4 of columns for the partitions p = set (mod kSets);
-// the sets are added in a fixed order.
+// each thread owning a float4 of columns for the states p = set (mod kSets);
+// the sets are added in a fixed order. A state covers the WARPS consecutive
+// partitions of one decode CTA (merged on chip), so a sequence of n partitions
+// has ceil(n / WARPS) of them.
 constexpr int kMergeThreads = 512;
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int WARPS>
 __global__ void __launch_bounds__(kMergeThreads) merge_partitions_kernel(const DecodeArgs a) {
   constexpr int kCols = D / 4;
   constexpr int kSets = kMergeThreads / kCols;
@@ -31,7 +33,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partitions_kernel(const D
   int ctx = __ldg(a.context_lens + s);
   if (ctx < 0 || ctx > a.max_blocks_per_seq * kBlockSize || ctx > a.max_context_len) ctx = 0;
   const int nblk = (ctx + kBlockSize - 1) / kBlockSize;
-  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  const int nparts = ((nblk + a.part_blocks - 1) / a.part_blocks + WARPS - 1) / WARPS;
   T* out = reinterpret_cast<T*>(a.out) + ((size_t)s * a.num_q_heads + (size_t)kvh * G + g) * D;
   if (nparts == 0) {
     for (int i = tid; i < D; i += blockDim.x) out[i] = Storage<T>::from_f32(0.f);

@@ -416,13 +416,18 @@ struct TensorPolicy {
       }
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
-    const float mnew = fmaxf(m, bmax);
-    const float mref = mnew == -INFINITY ? 0.f : mnew;
-    const float alpha = exp2f(m - mref);
-    m = mnew;
+    float alpha;
+    const float mref = lazy_reference(m, bmax, alpha);
     const float p0 = exp2f(x[0][0] - mref), p1 = exp2f(x[0][1] - mref);
     const float p2 = exp2f(x[1][0] - mref), p3 = exp2f(x[1][1] - mref);
     l = fmaf(l, alpha, (p0 + p1) + (p2 + p3));
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+      for (int n = 0; n < NTO; ++n) {
+        o[n][0] *= alpha;
+        o[n][1] *= alpha;
+      }
+    }
     uint32_t pa0, pa0_lo, pa2, pa2_lo;
     MmaOps<T>::split(p0, p1, pa0, pa0_lo);
     MmaOps<T>::split(p2, p3, pa2, pa2_lo);
@@ -433,10 +438,6 @@ struct TensorPolicy {
       const int t = (mi & 1) * 8 + ri;
       uint32_t v0, v1, v2, v3;
       ldsm_x4_trans(vbase + swz(t, 2 * pp + (mi >> 1)), v0, v1, v2, v3);
-      o[2 * pp][0] *= alpha;
-      o[2 * pp][1] *= alpha;
-      o[2 * pp + 1][0] *= alpha;
-      o[2 * pp + 1][1] *= alpha;
       MmaOps<T>::run(o[2 * pp], pa0_lo, pa2_lo, v0, v1);
       MmaOps<T>::run(o[2 * pp + 1], pa0_lo, pa2_lo, v2, v3);
       MmaOps<T>::run(o[2 * pp], pa0, pa2, v0, v1);

@@ -190,13 +190,18 @@ struct Fp8TensorPolicy {
       }
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
-    const float mnew = fmaxf(m, bmax);
-    const float mref = mnew == -INFINITY ? 0.f : mnew;
-    const float alpha = exp2f(m - mref);
-    m = mnew;
+    float alpha;
+    const float mref = lazy_reference(m, bmax, alpha);
     const float p0 = exp2f(x[0][0] - mref), p1 = exp2f(x[0][1] - mref);
     const float p2 = exp2f(x[1][0] - mref), p3 = exp2f(x[1][1] - mref);
     l = fmaf(l, alpha, (p0 + p1) + (p2 + p3));
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+      for (int n = 0; n < NTO; ++n) {
+        o[n][0] *= alpha;
+        o[n][1] *= alpha;
+      }
+    }
     uint32_t pa0, pa2;
     {
       const __half2 h0 = __floats2half2_rn(p0, p1);
@@ -245,8 +250,6 @@ struct Fp8TensorPolicy {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int nt = 4 * w + i;
-        o[nt][0] *= alpha;
-        o[nt][1] *= alpha;
         uint32_t b0, b1;
         e4m3x4_to_half2x2(y[i], b0, b1);
         MmaOps<__half>::run(o[nt], pa0, pa2, b0, b1);

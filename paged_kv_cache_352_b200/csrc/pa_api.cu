@@ -11,6 +11,8 @@
 #include <unordered_set>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "pa_internal.h"
 
 namespace pa {
@@ -157,19 +159,32 @@ int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
 
 }  // namespace pa
 
+pa::NvtxRange::NvtxRange(const char* name) { nvtxRangePushA(name); }
+pa::NvtxRange::~NvtxRange() { nvtxRangePop(); }
+
 using namespace pa;
 
 extern "C" {
 
 const char* pa_last_error(void) { return g_last_error.c_str(); }
 
-int pa_version(void) { return 110; }
+int pa_version(void) { return 111; }
+
+int pa_test_stall_next_decode(unsigned long long wait_limit_ns) {
+  clear_error();
+  if (wait_limit_ns < 1000ull || wait_limit_ns > 100000000ull)
+    return fail(PA_ERR_INVALID_ARG, "wait_limit_ns %llu: must be in [1 us, 100 ms]",
+                wait_limit_ns);
+  set_stall_request(wait_limit_ns);
+  return PA_OK;
+}
 
 int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_stride,
                          int64_t value_token_stride, void* k_cache, void* v_cache,
                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                          int head_dim, int block_size, int num_blocks, int dtype,
                          int* dev_error, void* stream) {
+  const NvtxRange nvtx_range("pa_reshape_and_cache");
   clear_error();
   if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype)) return st;
   if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens must be >= 0");
@@ -195,6 +210,7 @@ int pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_s
 int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                    void* stream) {
+  const NvtxRange nvtx_range("pa_copy_blocks");
   clear_error();
   if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype, true))
     return st;
@@ -238,6 +254,7 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_p
 int pa_swap_blocks(const void* src_k, const void* src_v, int src_num_blocks, void* dst_k,
                    void* dst_v, int dst_num_blocks, const int64_t* pairs, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int dtype, void* stream) {
+  const NvtxRange nvtx_range("pa_swap_blocks");
   clear_error();
   if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, src_num_blocks, dtype, true))
     return st;
@@ -592,8 +609,7 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
     return e;
 
   // both decodes leave partition states only; the merge writes `out`
-  DecodeArgs a;
-  memset(&a, 0, sizeof(a));
+  DecodeArgs a{};
   a.out = out;
   a.k_cache = k_cache;
   a.v_cache = v_cache;
@@ -607,30 +623,6 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
   a.out_scale = 1.f;
   a.warp_parts = 0;
   a.states_only = 1;
-  AuxStream* aux = nullptr;
-  if (num_groups > 0) {
-    if (int e = aux_stream(&aux)) return e;
-    if (int e = cuda_status(cudaEventRecord(aux->fork, st), "fork record")) return e;
-    if (int e = cuda_status(cudaStreamWaitEvent(aux->stream, aux->fork, 0), "fork wait"))
-      return e;
-    DecodeArgs gpre = a;
-    gpre.q = c.gq;
-    gpre.block_tables = c.g_tables;
-    gpre.context_lens = c.g_ctx;
-    gpre.ws_count = reinterpret_cast<int*>(ws + lay.gcount_off);
-    gpre.ws_m = gm;
-    gpre.ws_l = const_cast<float*>(c.g_l);
-    gpre.ws_acc = const_cast<float*>(c.g_acc);
-    gpre.num_seqs = num_groups;
-    gpre.num_q_heads = num_kv_heads * gg;
-    gpre.part_blocks = lay.g_part_blocks;
-    gpre.max_parts = lay.g_parts;
-    if (int e = cuda_status(launch_paged_decode(gpre, head_dim, gg, dtype, cache_dtype,
-                                                aux->stream),
-                            "cascade prefix decode launch"))
-      return e;
-    if (int e = cuda_status(cudaEventRecord(aux->join, aux->stream), "join record")) return e;
-  }
   DecodeArgs own = a;
   own.q = q;
   own.block_tables = c.s_tables;
@@ -643,6 +635,38 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
   own.num_q_heads = num_q_heads;
   own.part_blocks = lay.s_part_blocks;
   own.max_parts = lay.s_parts;
+  DecodeArgs gpre = a;
+  gpre.q = c.gq;
+  gpre.block_tables = c.g_tables;
+  gpre.context_lens = c.g_ctx;
+  gpre.ws_count = reinterpret_cast<int*>(ws + lay.gcount_off);
+  gpre.ws_m = gm;
+  gpre.ws_l = const_cast<float*>(c.g_l);
+  gpre.ws_acc = const_cast<float*>(c.g_acc);
+  gpre.num_seqs = num_groups;
+  gpre.num_q_heads = num_kv_heads * gg;
+  gpre.part_blocks = lay.g_part_blocks;
+  gpre.max_parts = lay.g_parts;
+  // Both decodes in one launch where the shapes allow (8 stacked query heads
+  // per KV head over a 16-bit cache), else on two streams.
+  if (num_groups > 0 && gg == 8 && gh < 8) {
+    const cudaError_t e = launch_cascade_decode(gpre, own, head_dim, gh, dtype, cache_dtype, st);
+    if (e == cudaSuccess)
+      return cuda_status(launch_cascade_merge(c, head_dim, dtype, st), "cascade merge launch");
+    if (e != cudaErrorNotSupported) return cuda_status(e, "cascade decode launch");
+  }
+  AuxStream* aux = nullptr;
+  if (num_groups > 0) {
+    if (int e = aux_stream(&aux)) return e;
+    if (int e = cuda_status(cudaEventRecord(aux->fork, st), "fork record")) return e;
+    if (int e = cuda_status(cudaStreamWaitEvent(aux->stream, aux->fork, 0), "fork wait"))
+      return e;
+    if (int e = cuda_status(launch_paged_decode(gpre, head_dim, gg, dtype, cache_dtype,
+                                                aux->stream),
+                            "cascade prefix decode launch"))
+      return e;
+    if (int e = cuda_status(cudaEventRecord(aux->join, aux->stream), "join record")) return e;
+  }
   if (int e = cuda_status(launch_paged_decode(own, head_dim, gh, dtype, cache_dtype, st),
                           "cascade own-block decode launch"))
     return e;
@@ -682,6 +706,7 @@ int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const
                             const int32_t* seq_member, int num_groups, int group_size,
                             int max_prefix_blocks, void* workspace, size_t workspace_bytes,
                             int* dev_error, int dtype, void* stream) {
+  const NvtxRange nvtx_range("pa_paged_decode_cascade");
   clear_error();
   return paged_decode_cascade_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                    context_lens, num_seqs, max_context_len, num_q_heads,
@@ -701,6 +726,7 @@ int pa_paged_decode_cascade_fp8(void* out, const void* q, const void* k_cache,
                                 const int32_t* seq_member, int num_groups, int group_size,
                                 int max_prefix_blocks, void* workspace, size_t workspace_bytes,
                                 int* dev_error, int dtype, void* stream) {
+  const NvtxRange nvtx_range("pa_paged_decode_cascade_fp8");
   clear_error();
   if (!positive_finite(k_scale) || !positive_finite(v_scale))
     return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
@@ -720,6 +746,7 @@ int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v
                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                     int num_blocks, float scale, int partition_tokens, void* workspace,
                     size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
+  const NvtxRange nvtx_range("pa_paged_decode");
   clear_error();
   return paged_decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
                            context_lens, seq_order, num_seqs, max_context_len, num_q_heads,
@@ -735,6 +762,7 @@ int pa_paged_decode_fp8(void* out, const void* q, const void* k_cache, const voi
                         int block_size, int num_blocks, float scale, float k_scale,
                         float v_scale, int partition_tokens, void* workspace,
                         size_t workspace_bytes, int* dev_error, int dtype, void* stream) {
+  const NvtxRange nvtx_range("pa_paged_decode_fp8");
   clear_error();
   if (!positive_finite(k_scale) || !positive_finite(v_scale))
     return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
@@ -750,6 +778,7 @@ int pa_reshape_and_cache_fp8(const void* key, const void* value, int64_t key_tok
                              const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                              int head_dim, int block_size, int num_blocks, int src_dtype,
                              float k_scale, float v_scale, int* dev_error, void* stream) {
+  const NvtxRange nvtx_range("pa_reshape_and_cache_fp8");
   clear_error();
   if (int st = check_cache_shape(num_kv_heads, head_dim, block_size, num_blocks, src_dtype))
     return st;

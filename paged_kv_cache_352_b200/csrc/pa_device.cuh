@@ -63,13 +63,16 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Waits for the barrier phase with the given parity; returns false when the
-// phase has not completed within kWaitLimitNs (the caller reports the timeout).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// phase has not completed within `limit_ns` (0: kWaitLimitNs), and the caller
+// reports the timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t limit = limit_ns ? limit_ns : kWaitLimitNs;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit) return false;
   }
 }
 
@@ -174,6 +177,25 @@ struct CacheElem<E4M3> {
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return static_cast<uint32_t>(
       __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Online-softmax reference of one row, updated lazily: the reference (base 2)
+// moves up only when the block's largest logit passes it by more than
+// kLazyRescaleLog2, so every exponential stays at most 2^kLazyRescaleLog2 and
+// most blocks keep the reference, when the caller's rescale of its accumulators
+// can be skipped. Any reference gives the same softmax once the accumulators
+// and the sum agree with it. Returns the reference for this block's exponentials
+// (0 while every logit so far is -inf); alpha is the factor to bring the
+// accumulators to it, exactly 1 when the reference did not move (and while
+// nothing has accumulated).
+constexpr float kLazyRescaleLog2 = 8.f;
+
+__device__ __forceinline__ float lazy_reference(float& m, float bmax, float& alpha) {
+  const float mnew = bmax > m + kLazyRescaleLog2 ? bmax : m;
+  const float mref = mnew == -INFINITY ? 0.f : mnew;
+  alpha = m == -INFINITY ? 1.f : exp2f(m - mref);
+  m = mnew;
+  return mref;
 }
 
 // gpu-scope fetch-and-add with acquire + release semantics.

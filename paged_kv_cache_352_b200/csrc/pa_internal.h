@@ -22,6 +22,16 @@ constexpr int kMaxPartitionBlocksOrdered = 256;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // bounded on-chip waits: 1 s
 constexpr int kMaxCopyPairsPerLaunch = 1024;   // pairs carried in one kernel parameter block
 
+// Names the enclosing library call in profiler timelines (an NVTX range pushed
+// on entry and popped on return). Without an attached profiler the calls are
+// no-ops behind a function pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name);
+  ~NvtxRange();
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Records a message for pa_last_error() and returns `code`.
 int fail(int code, const char* fmt, ...);
 void clear_error();
@@ -53,7 +63,18 @@ struct DecodeArgs {
   int states_only;   // every partition leaves its state in the workspace; nothing writes
                      // `out` and no partitions are merged (a sequence with no blocks
                      // leaves no state): the caller merges them
+  // Failure-detection test hook (pa_test_stall_next_decode); both 0 in normal use.
+  // stall_first_block: each warp arms the barrier of its first block without
+  // issuing the block's copy, so that wait runs out; wait_limit_ns: the limit of
+  // the main loop's waits (0 = kWaitLimitNs).
+  unsigned long long wait_limit_ns = 0;
+  int stall_first_block = 0;
 };
+
+// The wait limit a pending pa_test_stall_next_decode request asked for (0 when
+// none); taking it clears the request, so it applies to one decode launch.
+unsigned long long take_stall_request();
+void set_stall_request(unsigned long long wait_limit_ns);
 
 // Split partitions of at most this many blocks, for batches whose longest
 // context spans at least 16 of them, run one warp per partition when that grid
@@ -70,6 +91,13 @@ struct DecodeLayout {
 // Workspace layout for a decode call (bytes == 0 when no sequence can split).
 int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                   int max_context_len, int partition_tokens, bool ordered, DecodeLayout* lay);
+
+// The cascade's decode over the groups' prefixes (`pre`, 8 stacked query heads
+// per KV head) and over every sequence's own blocks (`own`, g_own query heads)
+// as one launch; cudaErrorNotSupported for shapes without that form, for which
+// the two decodes are launched separately.
+cudaError_t launch_cascade_decode(const DecodeArgs& pre, const DecodeArgs& own, int head_dim,
+                                  int g_own, int dtype, int cache_dtype, cudaStream_t stream);
 
 // dtype: query/output type (PA_F16 or PA_BF16); cache_dtype: dtype or PA_FP8_E4M3.
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,

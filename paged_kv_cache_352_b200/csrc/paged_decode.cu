@@ -36,6 +36,8 @@
 // (query type, head_dim) over E4M3 caches in paged_decode_<type>_d<dim>_e4m3.cu.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "pa_internal.h"
 
 namespace pa {
@@ -48,9 +50,33 @@ cudaError_t launch_decode_f16_d64_e4m3(const DecodeArgs& a, int group, cudaStrea
 cudaError_t launch_decode_f16_d128_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
 cudaError_t launch_decode_bf16_d64_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
 cudaError_t launch_decode_bf16_d128_e4m3(const DecodeArgs& a, int group, cudaStream_t stream);
+cudaError_t launch_cascade_decode_f16_d64(const DecodeArgs& pre, const DecodeArgs& own,
+                                          int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_f16_d128(const DecodeArgs& pre, const DecodeArgs& own,
+                                           int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_bf16_d64(const DecodeArgs& pre, const DecodeArgs& own,
+                                           int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_bf16_d128(const DecodeArgs& pre, const DecodeArgs& own,
+                                            int g_own, cudaStream_t stream);
 
-cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
+namespace {
+std::atomic<unsigned long long> g_stall_request{0};
+}  // namespace
+
+unsigned long long take_stall_request() {
+  if (g_stall_request.load(std::memory_order_relaxed) == 0) return 0;
+  return g_stall_request.exchange(0);
+}
+
+void set_stall_request(unsigned long long wait_limit_ns) { g_stall_request.store(wait_limit_ns); }
+
+cudaError_t launch_paged_decode(const DecodeArgs& args, int head_dim, int group, int dtype,
                                 int cache_dtype, cudaStream_t stream) {
+  DecodeArgs a = args;
+  if (const unsigned long long ns = take_stall_request()) {
+    a.stall_first_block = 1;
+    a.wait_limit_ns = ns;
+  }
   const bool fp8 = cache_dtype == PA_FP8_E4M3;
   if (!fp8 && cache_dtype != dtype) return cudaErrorInvalidValue;
   if (dtype == PA_F16) {
@@ -65,6 +91,19 @@ cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, in
                                     : launch_decode_bf16_d128(a, group, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_cascade_decode(const DecodeArgs& pre, const DecodeArgs& own, int head_dim,
+                                  int g_own, int dtype, int cache_dtype, cudaStream_t stream) {
+  if (cache_dtype != dtype) return cudaErrorNotSupported;  // 8-bit caches: two launches
+  if (dtype == PA_F16) {
+    if (head_dim == 64) return launch_cascade_decode_f16_d64(pre, own, g_own, stream);
+    if (head_dim == 128) return launch_cascade_decode_f16_d128(pre, own, g_own, stream);
+  } else {
+    if (head_dim == 64) return launch_cascade_decode_bf16_d64(pre, own, g_own, stream);
+    if (head_dim == 128) return launch_cascade_decode_bf16_d128(pre, own, g_own, stream);
+  }
+  return cudaErrorNotSupported;
 }
 
 }  // namespace pa

@@ -31,19 +31,19 @@ constexpr int min_ctas_hint() {
   return P::kMinCtasPerSm * 4 / WARPS > 0 ? P::kMinCtasPerSm * 4 / WARPS : 1;
 }
 
+// One CTA's work: (KV head kvh, partition part) of the sequence that grid row z
+// serves. The body of paged_decode_kernel, and of each half of the cascade's
+// two-part kernel.
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
-    paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v) {
+__device__ __forceinline__ void decode_unit(const DecodeArgs& a, const CUtensorMap* tm_k,
+                                            const CUtensorMap* tm_v, int kvh, int part, int z) {
   constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + P::kAlign - 1) & ~(uintptr_t)(P::kAlign - 1));
-  const int kvh = blockIdx.x;
-  const int part = blockIdx.y;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int s = a.seq_order ? __ldg(a.seq_order + blockIdx.z) : (int)blockIdx.z;
+  const int s = a.seq_order ? __ldg(a.seq_order + z) : z;
   if ((unsigned)s >= (unsigned)a.num_seqs) {
     if (part == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
     return;
@@ -110,11 +110,13 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
       uint64_t* bar = &wbars[st];
       const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
       wvalid[st] = ok;  // published to the consumers by the arrive below
-      if (!ok) {
+      if (a.stall_first_block && j == 0) {
+        mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
+      } else if (!ok) {
         report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
         mbar_arrive(bar);  // complete the phase without data; the block is skipped
       } else {
-        P::issue(a, &tm_k, &tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
+        P::issue(a, tm_k, tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
       }
     }
   };
@@ -122,9 +124,12 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   int issued = my_n < STAGES ? my_n : STAGES;
   pol.begin(a.scale_log2);
 
-  bool aborted = false;
+  // test hook: the first stage was armed without a copy; its wait runs out
+  bool aborted = a.stall_first_block && my_n > 0 &&
+                 !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
+  if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
   int j = 0;
-  for (; j < my_n; ++j) {
+  for (; !aborted && j < my_n; ++j) {
     const int st = j % STAGES;
     if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
       if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
@@ -142,8 +147,10 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   }
   if (aborted) {
     // drain the copies still in flight into this warp's ring before leaving it
+    // (a stage the test hook armed without a copy has none)
     for (int k = j; k < issued; ++k)
-      mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
+      if (!(a.stall_first_block && k == 0))
+        mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
   }
 
   // merge the warps through shared memory, reusing the tile ring
@@ -155,6 +162,43 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   __syncthreads();
   finish_partition<T, D, G, WARPS>(a, red_m, red_m, red_l, red_acc, s, kvh, part, nparts,
                                    out_rows);
+}
+
+template <class P, typename T, int D, int G, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
+    paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v) {
+  decode_unit<P, T, D, G, WARPS, STAGES>(a, &tm_k, &tm_v, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+template <class P1, class P2, int WARPS>
+constexpr int min_ctas_hint2() {
+  return min_ctas_hint<P1, WARPS>() < min_ctas_hint<P2, WARPS>() ? min_ctas_hint<P1, WARPS>()
+                                                                 : min_ctas_hint<P2, WARPS>();
+}
+
+// The cascade's two decodes in one launch: CTAs [0, n1) serve `a1` (the
+// groups' shared prefixes, members' query heads stacked) and the rest serve
+// `a2` (every sequence's own blocks), each CTA index split into (KV head,
+// partition, sequence) with the KV head fastest. The long prefix partitions are
+// scheduled first and the short own-block CTAs fill the SMs behind them, so the
+// launch has one tail instead of two.
+template <class P1, int G1, class P2, int G2, typename T, int D, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint2<P1, P2, WARPS>()))
+    cascade_decode_kernel(const DecodeArgs a1, const DecodeArgs a2,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v) {
+  const int hkv = a1.num_kv_heads;
+  const int n1 = hkv * a1.max_parts * a1.num_seqs;
+  int i = blockIdx.x;
+  if (i < n1) {
+    decode_unit<P1, T, D, G1, WARPS, STAGES>(a1, &tm_k, &tm_v, i % hkv, (i / hkv) % a1.max_parts,
+                                             i / (hkv * a1.max_parts));
+  } else {
+    i -= n1;
+    decode_unit<P2, T, D, G2, WARPS, STAGES>(a2, &tm_k, &tm_v, i % hkv, (i / hkv) % a2.max_parts,
+                                             i / (hkv * a2.max_parts));
+  }
 }
 
 // Split-KV with one warp per partition, for short partitions (at most
@@ -198,8 +242,9 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   }
   const int nblk = (ctx + kBS - 1) / kBS;
   const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
-  if (part >= nparts) return;  // the whole warp: no barrier spans warps here
-  const int my_n = min(nblk, b_begin + a.part_blocks) - b_begin;
+  if ((int)blockIdx.y * WARPS >= nparts) return;  // the whole CTA
+  // a warp past the sequence's last partition streams nothing but joins the merge
+  const int my_n = part < nparts ? min(nblk, b_begin + a.part_blocks) - b_begin : 0;
 
   unsigned char* wring = smem + (size_t)warp * STAGES * P::kStageBytes;
   uint64_t* wbars = reinterpret_cast<uint64_t*>(smem + kRing) + warp * STAGES;
@@ -227,7 +272,9 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
       uint64_t* bar = &wbars[st];
       const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
       wvalid[st] = ok;
-      if (!ok) {
+      if (a.stall_first_block && j == 0) {
+        mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
+      } else if (!ok) {
         report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
         mbar_arrive(bar);
       } else {
@@ -239,9 +286,11 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   int issued = my_n < STAGES ? my_n : STAGES;
   pol.begin(a.scale_log2);
 
-  bool aborted = false;
+  bool aborted = a.stall_first_block && my_n > 0 &&
+                 !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
+  if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
   int j = 0;
-  for (; j < my_n; ++j) {
+  for (; !aborted && j < my_n; ++j) {
     const int st = j % STAGES;
     if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
       if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
@@ -258,11 +307,38 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   }
   if (aborted) {
     for (int k = j; k < issued; ++k)
-      mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
+      if (!(a.stall_first_block && k == 0))
+        mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
   }
-  // the partition's state straight from registers: rows [G] of m, l and [G][D] of acc
-  const size_t row = (((size_t)s * a.num_kv_heads + kvh) * a.max_parts + part) * G;
-  pol.to_red(a.ws_m + row, a.ws_l + row, a.ws_acc + row * D, 0, lane);
+  // The CTA's WARPS consecutive partitions merge on chip (through shared memory,
+  // reusing the tile ring) into one state row, row blockIdx.y of the sequence's
+  // rows: the merge kernel then reads WARPS times fewer states.
+  __syncthreads();
+  float* red_m = reinterpret_cast<float*>(smem);  // [WARPS][G]
+  float* red_l = red_m + WARPS * G;                // [WARPS][G]
+  float* red_acc = red_l + WARPS * G;              // [WARPS][G][D]
+  pol.to_red(red_m, red_l, red_acc, warp, lane);
+  __syncthreads();
+  const size_t row0 = (((size_t)s * a.num_kv_heads + kvh) * a.max_parts + blockIdx.y) * G;
+  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
+    const int g = item / D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_m[w * G + g]);
+    const float Mref = M == -INFINITY ? 0.f : M;
+    float L = 0.f, A = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      const float sc = exp2f(red_m[w * G + g] - Mref);
+      L = fmaf(sc, red_l[w * G + g], L);
+      A = fmaf(sc, red_acc[(w * G) * D + item], A);
+    }
+    a.ws_acc[(row0 + g) * D + (item % D)] = A;
+    if (item % D == 0) {
+      a.ws_m[row0 + g] = M;
+      a.ws_l[row0 + g] = L;
+    }
+  }
 }
 
 constexpr size_t kSmemLimit = 200 * 1024;
@@ -376,11 +452,51 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e != cudaSuccess || a.states_only) return e;
     dim3 mgrid(a.num_kv_heads * G, a.num_seqs);
-    merge_partitions_kernel<T, D, G><<<mgrid, kMergeThreads, 0, stream>>>(a);
+    merge_partitions_kernel<T, D, G, WARPS><<<mgrid, kMergeThreads, 0, stream>>>(a);
     return cudaGetLastError();
   }
   dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
   kern<<<grid, WARPS * 32, smem, stream>>>(a, tk, tv);
+  return cudaGetLastError();
+}
+
+// The cascade's two decodes as one launch of cascade_decode_kernel (4 x 2 tiles).
+template <class P1, int G1, class P2, int G2, typename T, int D>
+cudaError_t launch_dual(const DecodeArgs& a1, const DecodeArgs& a2, int dtype,
+                        cudaStream_t stream) {
+  constexpr int WARPS = 4, STAGES = 2;
+  const size_t s1 = smem_bytes<P1, WARPS, STAGES, G1, D>(a1.max_parts);
+  const size_t s2 = smem_bytes<P2, WARPS, STAGES, G2, D>(a2.max_parts);
+  const size_t smem = s1 > s2 ? s1 : s2;
+  if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
+  const long long n1 = (long long)a1.num_kv_heads * a1.max_parts * a1.num_seqs;
+  const long long n2 = (long long)a2.num_kv_heads * a2.max_parts * a2.num_seqs;
+  if (a1.num_kv_heads != a2.num_kv_heads || n1 + n2 > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (n1 + n2 == 0) return cudaSuccess;
+  auto kern = cascade_decode_kernel<P1, G1, P2, G2, T, D, WARPS, STAGES>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  static std::atomic<bool> ready[kMaxDevices];
+  if (!ready[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+    if (e != cudaSuccess) return e;
+    ready[dev].store(true, std::memory_order_release);
+  }
+  CUtensorMap tk, tv;
+  memset(&tk, 0, sizeof(tk));
+  memset(&tv, 0, sizeof(tv));
+  if (P1::kTma2D || P2::kTma2D) {
+    static_assert(!P1::kFp8Cache && !P2::kFp8Cache, "16-bit caches only");
+    const long long rows = (long long)a1.num_blocks * a1.num_kv_heads * kBS;
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA row coordinates are int32
+    e = make_cache_map(&tk, a1.k_cache, rows, D, dtype);
+    if (e != cudaSuccess) return e;
+    e = make_cache_map(&tv, a1.v_cache, rows, D, dtype);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<(unsigned)(n1 + n2), WARPS * 32, smem, stream>>>(a1, a2, tk, tv);
   return cudaGetLastError();
 }
 
@@ -472,6 +588,27 @@ cudaError_t launch_group(const DecodeArgs& a, int group, int dtype, cudaStream_t
 }
 
 }  // namespace
+
+// The cascade's decodes of a 16-bit cache in one launch: the groups' prefixes
+// with 8 stacked query heads (`pre`, tensor cores) and the own blocks with
+// g_own query heads per KV head (`own`, the policy paged_decode would pick).
+// cudaErrorNotSupported when that shape has no single-launch form (or a
+// PA_DECODE_PATH override is set): the caller then launches the two decodes.
+template <typename T, int D>
+cudaError_t launch_cascade_typed(const DecodeArgs& pre, const DecodeArgs& own, int g_own,
+                                 int dtype, cudaStream_t stream) {
+  if (!use_tensor_path(8) || getenv("PA_DECODE_PATH")) return cudaErrorNotSupported;
+  using Pre = TensorPolicy<T, D, 8>;
+  switch (g_own) {
+    case 1:
+      return launch_dual<Pre, 8, CudaCorePolicy<T, D, 1, T>, 1, T, D>(pre, own, dtype, stream);
+    case 2:
+      return launch_dual<Pre, 8, CudaCorePolicy<T, D, 2, T>, 2, T, D>(pre, own, dtype, stream);
+    case 4:
+      return launch_dual<Pre, 8, TensorPolicy<T, D, 4>, 4, T, D>(pre, own, dtype, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
 
 // Launches the decode kernel for one query/output type T, head_dim and cache
 // element type C (T itself, or E4M3).

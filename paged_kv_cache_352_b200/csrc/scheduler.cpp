@@ -27,6 +27,10 @@ using pa::fail;
 namespace {
 
 constexpr int kRing = 3;  // pinned staging buffers in flight
+// PA_SCHED_CASCADE_AUTO takes the cascade when the shared blocks it reads once
+// instead of once per member of another request add up to this many bytes:
+// about what its two extra launches cost at the copy bandwidth.
+constexpr double kCascadeMinSavedBytes = 32.0 * 1024 * 1024;
 
 struct Request {
   int64_t id = 0;
@@ -114,6 +118,14 @@ struct pa_sched {
   void* workspace = nullptr;
   size_t workspace_bytes = 0;
   std::vector<int32_t> order_tmp;
+  // decode through the cascade when batch sequences share leading blocks
+  int cascade_mode = PA_SCHED_CASCADE_AUTO;
+  void* cascade_ws = nullptr;
+  size_t cascade_ws_bytes = 0;
+  int last_groups = 0;
+  int64_t last_saved_blocks = 0;
+  std::vector<int64_t> ids_tmp;
+  std::vector<int32_t> gm_tmp, gp_tmp, sg_tmp, sm_tmp;
 
   static int64_t seq_of(int64_t request, int sample) {
     return request * PA_SCHED_MAX_SAMPLES + sample;
@@ -358,7 +370,9 @@ struct pa_sched {
     }
     if (dev_meta) cudaFree(dev_meta);
     if (workspace) cudaFree(workspace);
-    dev_meta = workspace = nullptr;
+    if (cascade_ws) cudaFree(cascade_ws);
+    dev_meta = workspace = cascade_ws = nullptr;
+    cascade_ws_bytes = 0;
     attached = false;
   }
 };
@@ -448,6 +462,7 @@ int pa_sched_submit_tokens(pa_sched* s, int64_t request_id, const int32_t* promp
 }
 
 int pa_sched_step(pa_sched* s, pa_sched_plan* plan) {
+  const pa::NvtxRange nvtx_range("pa_sched_step");
   pa::clear_error();
   if (!s || !plan) return fail(PA_ERR_INVALID_ARG, "null argument");
   if (s->failed) return fail(PA_ERR_NO_FREE_BLOCKS, "scheduler failed in an earlier step");
@@ -559,6 +574,24 @@ int pa_sched_kv_usage(const pa_sched* s, int64_t* filled, int64_t* allocated) {
 
 const pa_bm* pa_sched_block_manager(const pa_sched* s) { return s ? s->bm : nullptr; }
 
+int pa_sched_set_cascade(pa_sched* s, int mode) {
+  pa::clear_error();
+  if (!s) return fail(PA_ERR_INVALID_ARG, "null scheduler");
+  if (mode != PA_SCHED_CASCADE_OFF && mode != PA_SCHED_CASCADE_ON &&
+      mode != PA_SCHED_CASCADE_AUTO)
+    return fail(PA_ERR_INVALID_ARG, "cascade mode %d", mode);
+  s->cascade_mode = mode;
+  return PA_OK;
+}
+
+int pa_sched_last_cascade(const pa_sched* s, int* num_groups, int64_t* shared_blocks) {
+  pa::clear_error();
+  if (!s || !num_groups || !shared_blocks) return fail(PA_ERR_INVALID_ARG, "null argument");
+  *num_groups = s->last_groups;
+  *shared_blocks = s->last_saved_blocks;
+  return PA_OK;
+}
+
 int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim, int dtype,
                     int max_context_len) {
   pa::clear_error();
@@ -582,11 +615,36 @@ int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim
     }
   }
   const int64_t maxb = ceil_div(max_context_len, s->block_size);
+  // The cascade's workspace, for every batch size and number of groups (at most
+  // one per two sequences) over the same ladder of context lengths, each
+  // context's blocks all shareable.
+  const int gh = num_kv_heads > 0 ? num_q_heads / num_kv_heads : 0;
+  size_t cws = 0;
+  if (gh >= 1 && gh <= 4 && num_q_heads % num_kv_heads == 0) {
+    for (int b = 2; b <= s->max_num_seqs; ++b) {
+      for (int64_t c = 16;; c = std::min<int64_t>(2 * c, max_context_len)) {
+        const int mb = (int)ceil_div(c, s->block_size);
+        for (int ng = 1; ng <= b / 2; ++ng) {
+          size_t bytes = 0;
+          if (pa_paged_decode_cascade_workspace_size(b, num_q_heads, num_kv_heads, head_dim,
+                                                     (int)c, mb, s->block_size, ng, 8 / gh, mb,
+                                                     &bytes) == PA_OK)
+            cws = std::max(cws, bytes);
+        }
+        if (c == max_context_len) break;
+      }
+    }
+    pa::clear_error();
+  }
   const size_t cap_prefill = (size_t)s->bm->num_blocks * s->block_size;
   const size_t cap_tokens = (size_t)s->max_num_seqs;
   size_t bytes = 8 * (cap_prefill + cap_tokens);
   bytes = align_up(bytes, 16) + 4 * (size_t)s->max_num_seqs * maxb;
   bytes = align_up(bytes, 16) + 4 * 2 * (size_t)s->max_num_seqs;
+  // group descriptors: members (<= 8 per group, <= one group per two sequences),
+  // prefix lengths, and each sequence's group and slot
+  bytes = align_up(bytes, 16) + 4 * (size_t)(4 * s->max_num_seqs + s->max_num_seqs / 2 +
+                                             2 * s->max_num_seqs) + 64;
   bytes = align_up(bytes, 256);
   s->hq = num_q_heads;
   s->hkv = num_kv_heads;
@@ -600,6 +658,7 @@ int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim
   cudaError_t e = cudaMalloc(&s->dev_meta, bytes);
   if (e == cudaSuccess && ws) e = cudaMalloc(&s->workspace, ws);
   if (e == cudaSuccess && ws) e = cudaMemset(s->workspace, 0, ws);
+  if (e == cudaSuccess && cws) e = cudaMalloc(&s->cascade_ws, cws);
   for (int k = 0; k < kRing && e == cudaSuccess; ++k) {
     e = cudaHostAlloc(&s->host_meta[k], bytes, cudaHostAllocDefault);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s->ring_ev[k], cudaEventDisableTiming);
@@ -609,6 +668,7 @@ int pa_sched_attach(pa_sched* s, int num_q_heads, int num_kv_heads, int head_dim
     return fail(PA_ERR_CUDA, "executor allocation failed: %s", cudaGetErrorString(e));
   }
   s->workspace_bytes = ws;
+  s->cascade_ws_bytes = cws;
   s->cache_dtype = dtype;
   s->attached = true;
   return PA_OK;
@@ -632,6 +692,7 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
                      const void* prefill_key, const void* prefill_value, const void* key,
                      const void* value, const void* q, void* out, float scale, int* dev_error,
                      void* stream) {
+  const pa::NvtxRange nvtx_range("pa_sched_execute");
   pa::clear_error();
   if (!s) return fail(PA_ERR_INVALID_ARG, "null scheduler");
   if (!s->attached) return fail(PA_ERR_INVALID_ARG, "no executor attached");
@@ -650,6 +711,64 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
       (!p.writes.empty() && (!key || !value)) || (nseq && (!q || !out)))
     return fail(PA_ERR_INVALID_ARG, "null input for a non-empty part of the step");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // Sequences of the batch that hold the same leading blocks (samples forked
+  // from one prompt, requests whose prompts were found in the prefix cache) are
+  // decoded through the cascade, which reads their shared blocks once.
+  int ng = 0, maxp = 0;
+  const int gh = s->hq / hkv;
+  const int gsz = 8 / gh;  // members stacked per KV head: 8 query heads in all
+  s->last_groups = 0;
+  s->last_saved_blocks = 0;
+  if (s->cascade_mode != PA_SCHED_CASCADE_OFF && s->cascade_ws && nseq >= 2 && gsz >= 2) {
+    s->ids_tmp.resize(nseq);
+    for (int i = 0; i < nseq; ++i)
+      s->ids_tmp[i] = pa_sched::seq_of(p.batch_request[i], p.batch_sample[i]);
+    s->gm_tmp.resize((size_t)nseq * gsz);
+    s->gp_tmp.resize(nseq);
+    s->sg_tmp.resize(nseq);
+    s->sm_tmp.resize(nseq);
+    if (pa_bm_prefix_groups(s->bm, s->ids_tmp.data(), nseq, gsz, s->gm_tmp.data(),
+                            s->gp_tmp.data(), s->sg_tmp.data(), s->sm_tmp.data(), &ng,
+                            &maxp) != PA_OK)
+      return fail(PA_ERR_INVALID_ARG, "grouping the batch: %s", pa_last_error());
+    // Block reads saved per group: (members - 1) x its prefix. The automatic
+    // rule counts only members of other requests than the group's first: the
+    // samples of one request have equal contexts, so the plain decode's
+    // longest-first order runs them side by side and L2 already serves their
+    // shared prompt once; requests that share a cached prompt are not adjacent.
+    int64_t saved = 0, saved_across = 0;
+    for (int g = 0; g < ng; ++g) {
+      const int32_t* row = s->gm_tmp.data() + (size_t)g * gsz;
+      int m = 0, others = 0;
+      for (int j = 0; j < gsz && row[j] >= 0; ++j) {
+        ++m;
+        bool seen = p.batch_request[row[j]] == p.batch_request[row[0]];
+        for (int k = 1; k < j && !seen; ++k)
+          seen = p.batch_request[row[k]] == p.batch_request[row[j]];
+        others += !seen;
+      }
+      saved += (int64_t)(m - 1) * s->gp_tmp[g];
+      saved_across += (int64_t)others * s->gp_tmp[g];
+    }
+    const double block_bytes =
+        2.0 * hkv * bs * d * (s->cache_dtype == PA_FP8_E4M3 ? 1 : 2);
+    if (s->cascade_mode == PA_SCHED_CASCADE_AUTO &&
+        saved_across * block_bytes < kCascadeMinSavedBytes)
+      ng = 0;
+    if (ng) {
+      size_t need = 0;
+      if (pa_paged_decode_cascade_workspace_size(nseq, s->hq, hkv, d, p.max_ctx, p.max_blocks,
+                                                 bs, ng, gsz, maxp, &need) != PA_OK ||
+          need > s->cascade_ws_bytes)
+        ng = 0;
+    }
+    pa::clear_error();
+    if (ng) {
+      s->last_groups = ng;
+      s->last_saved_blocks = saved;
+    }
+  }
 
   // stage slots, tables, context lengths and the order in one pinned buffer
   const int k = s->ring_next;
@@ -677,6 +796,27 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
   if (nseq) pa_longest_first_order(p.batch_ctx.data(), nseq, s->order_tmp.data());
   memcpy(h + off, s->order_tmp.data(), 4 * (size_t)nseq);
   off += 4 * (size_t)nseq;
+  // group descriptors (cascade steps only): members, prefix lengths, group and slot
+  const size_t off_gm = off = align_up(off, 16);
+  if (ng) {
+    memcpy(h + off, s->gm_tmp.data(), 4 * (size_t)ng * gsz);
+    off += 4 * (size_t)ng * gsz;
+  }
+  const size_t off_gp = off;
+  if (ng) {
+    memcpy(h + off, s->gp_tmp.data(), 4 * (size_t)ng);
+    off += 4 * (size_t)ng;
+  }
+  const size_t off_sg = off;
+  if (ng) {
+    memcpy(h + off, s->sg_tmp.data(), 4 * (size_t)nseq);
+    off += 4 * (size_t)nseq;
+  }
+  const size_t off_sm = off;
+  if (ng) {
+    memcpy(h + off, s->sm_tmp.data(), 4 * (size_t)nseq);
+    off += 4 * (size_t)nseq;
+  }
   char* dm = static_cast<char*>(s->dev_meta);
   if (off) {
     e = cudaMemcpyAsync(dm, h, off, cudaMemcpyHostToDevice, st);
@@ -718,6 +858,21 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
     const int32_t* tables = reinterpret_cast<const int32_t*>(dm + off_tables);
     const int32_t* ctx = reinterpret_cast<const int32_t*>(dm + off_ctx);
     const int32_t* order = reinterpret_cast<const int32_t*>(dm + off_order);
+    if (ng) {
+      const int32_t* gm = reinterpret_cast<const int32_t*>(dm + off_gm);
+      const int32_t* gp = reinterpret_cast<const int32_t*>(dm + off_gp);
+      const int32_t* sg = reinterpret_cast<const int32_t*>(dm + off_sg);
+      const int32_t* sm = reinterpret_cast<const int32_t*>(dm + off_sm);
+      return fp8 ? pa_paged_decode_cascade_fp8(
+                       out, q, k_cache, v_cache, tables, p.max_blocks, ctx, nseq, p.max_ctx,
+                       s->hq, hkv, d, bs, nb, scale, s->k_scale, s->v_scale, gm, gp, sg, sm, ng,
+                       gsz, maxp, s->cascade_ws, s->cascade_ws_bytes, dev_error, s->dtype,
+                       stream)
+                 : pa_paged_decode_cascade(out, q, k_cache, v_cache, tables, p.max_blocks, ctx,
+                                           nseq, p.max_ctx, s->hq, hkv, d, bs, nb, scale, gm, gp,
+                                           sg, sm, ng, gsz, maxp, s->cascade_ws,
+                                           s->cascade_ws_bytes, dev_error, s->dtype, stream);
+    }
     const int r =
         fp8 ? pa_paged_decode_fp8(out, q, k_cache, v_cache, tables, p.max_blocks, ctx, order, nseq,
                                   p.max_ctx, s->hq, hkv, d, bs, nb, scale, s->k_scale, s->v_scale,

@@ -209,7 +209,10 @@ class DecodeRunner:
     def decode_launches(self) -> int:
         """Kernel launches of the step's decode call."""
         if self.groups is not None:
-            return 4  # prepare, prefix decode, own-block decode, merge
+            # prepare, both decodes in one launch (8 stacked query heads per KV
+            # head over a 16-bit cache; else two launches), merge
+            g = self.wl.num_q_heads // self.wl.num_kv_heads
+            return 3 if g * self.groups.group_size == 8 and g < 8 else 4
         wl = self.wl
         _, _, n = L.pa_paged_decode_plan(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
                                          wl.head_dim, wl.max_context_len,

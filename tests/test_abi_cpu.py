@@ -27,11 +27,19 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert len(names) >= 18
     missing = [n for n in names if not hasattr(h, n)]
     assert not missing, missing
-    assert h.pa_version() == 110
+    assert h.pa_version() == 111
 
 
 def test_binding_covers_every_declared_symbol():
     assert set(_declared_symbols()) <= set(L._SIGS)
+
+
+def test_stall_hook_rejects_limits_out_of_range():
+    # (a valid limit would arm the next decode launch of this process: not done here)
+    assert L.lib().pa_test_stall_next_decode(0) == L.PA_ERR_INVALID_ARG
+    assert L.lib().pa_test_stall_next_decode(999) == L.PA_ERR_INVALID_ARG
+    assert L.lib().pa_test_stall_next_decode(10**9) == L.PA_ERR_INVALID_ARG
+    assert "wait_limit_ns" in L.last_error()
 
 
 # ---- host-side argument checks (return before any CUDA call) --------------------

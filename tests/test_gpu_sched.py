@@ -21,9 +21,10 @@ from workloads import gen
 pytestmark = pytest.mark.gpu
 
 
-def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
+def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None, cascade=None):
     """fp8 = (k_scale, v_scale) runs the loop over E4M3 caches; the oracle then
-    attends to the quantized-then-dequantized rows."""
+    attends to the quantized-then-dequantized rows. cascade sets the executor's
+    cascade mode (PA_SCHED_CASCADE_*; the library's default otherwise)."""
     tdt = torch.float16 if dt == "f16" else torch.bfloat16
     cdt = torch.uint8 if fp8 else tdt
     order = np.random.default_rng(seed).permutation(nb)
@@ -35,6 +36,8 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
         o.submit(*t[:5], tokens=toks)
     max_ctx = max(t[1] + t[2] for t in trace)
     c.attach(hq, hkv, d, tdt, max_ctx, fp8_scales=fp8)
+    if cascade is not None:
+        c.set_cascade(cascade)
     kc = torch.zeros(nb, hkv, 16, d, dtype=cdt, device="cuda")
     vc = torch.zeros_like(kc)
     hk = torch.zeros(max(host, 1), hkv, 16, d, dtype=cdt).pin_memory() if host else None
@@ -44,7 +47,8 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     scale = 1 / math.sqrt(d)
     G = hq // hkv
-    stats = {"steps": 0, "preempt": 0, "swap": 0, "cow": 0, "seqs": 0, "cached": 0}
+    stats = {"steps": 0, "preempt": 0, "swap": 0, "cow": 0, "seqs": 0, "cached": 0,
+             "cascade_steps": 0, "cascade_groups": 0}
     while not o.idle():
         c.step()
         op = o.step()
@@ -68,6 +72,9 @@ def _run_trace(trace, nb, cap, host, mode, hq, hkv, d, dt, seed, fp8=None):
         out = torch.empty(len(op.batch), hq, d, dtype=tdt, device="cuda")
         c.execute(kc, vc, hk, hv, pk, pv, wk, wv, q, out, scale, dev_error=err)
         torch.cuda.synchronize()
+        ng, _ = c.last_cascade()
+        stats["cascade_steps"] += ng > 0
+        stats["cascade_groups"] += ng
         got = out_to_f64(out, dt)
         for i, (r, s, ctx) in enumerate(op.batch):
             K, V = toks.rows(r, s, range(ctx))
@@ -150,3 +157,44 @@ def test_prefix_cached_recompute_over_fp8_cache():
                     mode=pa.PA_PREEMPT_RECOMPUTE, hq=4, hkv=4, d=64, dt="f16", seed=45,
                     fp8=(0.02, 0.02))
     assert st["cached"] > 0 and st["preempt"] > 0, st
+
+
+def test_parallel_samples_decoded_through_the_cascade():
+    """Samples forked from one prompt share its full blocks; with the cascade on,
+    every step that has such a group reads them once per group, and every output
+    still matches the oracle (8 / G = 2 samples per group at G = 4)."""
+    st = _run_trace(_trace(31, 24, 4, prompt=(40, 200)), nb=120, cap=12, host=400,
+                    mode=pa.PA_PREEMPT_SWAP, hq=8, hkv=2, d=128, dt="bf16", seed=51,
+                    cascade=pa.PA_SCHED_CASCADE_ON)
+    assert st["cascade_steps"] > 0 and st["cow"] > 0, st
+
+
+def test_parallel_samples_through_the_cascade_mha_f16():
+    """One query head per KV head: groups of up to 8 samples stack 8 heads."""
+    st = _run_trace(_trace(32, 16, 6, prompt=(30, 300), arrive=8), nb=400, cap=16, host=400,
+                    mode=pa.PA_PREEMPT_SWAP, hq=4, hkv=4, d=64, dt="f16", seed=52,
+                    cascade=pa.PA_SCHED_CASCADE_ON)
+    assert st["cascade_steps"] > 0, st
+
+
+def test_prefix_cached_requests_through_the_cascade():
+    """Requests sharing system prompts hold the same cached blocks: they are
+    grouped across requests and decoded through the cascade."""
+    from tests.test_oracle_scheduler import _prompt_trace
+    st = _run_trace(_prompt_trace(23, 24, 3), nb=30, cap=12, host=400, mode=pa.PA_PREEMPT_SWAP,
+                    hq=8, hkv=2, d=128, dt="bf16", seed=44, cascade=pa.PA_SCHED_CASCADE_ON)
+    assert st["cached"] > 0 and st["cascade_steps"] > 0, st
+
+
+def test_cascade_in_the_loop_over_fp8_cache():
+    st = _run_trace(_trace(31, 24, 4, prompt=(40, 200)), nb=120, cap=12, host=400,
+                    mode=pa.PA_PREEMPT_SWAP, hq=8, hkv=2, d=128, dt="bf16", seed=51,
+                    fp8=(0.02, 0.015), cascade=pa.PA_SCHED_CASCADE_ON)
+    assert st["cascade_steps"] > 0, st
+
+
+def test_cascade_off_decodes_plainly():
+    st = _run_trace(_trace(31, 12, 4, prompt=(40, 200)), nb=120, cap=12, host=400,
+                    mode=pa.PA_PREEMPT_SWAP, hq=8, hkv=2, d=128, dt="bf16", seed=51,
+                    cascade=pa.PA_SCHED_CASCADE_OFF)
+    assert st["cascade_steps"] == 0, st
