@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(256)
                              uint4* v_cache, const int64_t* __restrict__ slot_mapping,
                              int64_t total_chunks, int chunks_per_row, int num_kv_heads,
                              int64_t num_slots, int* dev_error) {
+  allow_dependents();  // a following decode may launch; it waits for this kernel
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= total_chunks) return;
   const int64_t per_token = (int64_t)chunks_per_row * num_kv_heads;
@@ -68,6 +69,7 @@ __global__ void __launch_bounds__(256)
                                  int64_t total_chunks, int chunks_per_row, int num_kv_heads,
                                  int64_t num_slots, float k_scale, float v_scale,
                                  int* dev_error) {
+  allow_dependents();  // a following decode may launch; it waits for this kernel
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= total_chunks) return;
   const int64_t per_token = (int64_t)chunks_per_row * num_kv_heads;
@@ -118,6 +120,7 @@ constexpr int kCopyUnroll = 4;
 __global__ void __launch_bounds__(kCopyThreads)
     copy_pool_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* dst_v,
                             const __grid_constant__ CopyPairs pairs, int64_t vecs_per_block) {
+  allow_dependents();  // a following decode may launch; it waits for this kernel
   const int pair = blockIdx.y;
   const int64_t src = pairs.src[pair];
   const int64_t dst = pairs.dst[pair];

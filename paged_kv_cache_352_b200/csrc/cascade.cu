@@ -65,6 +65,7 @@ __device__ void write_own_table(const CascadeArgs& c, int s, int first) {
 template <int D>
 __global__ void __launch_bounds__(kPrepThreads) cascade_prepare_kernel(const CascadeArgs c,
                                                                         int gh, int copy_ctas) {
+  allow_dependents();  // the decode launch may start; it waits for this kernel
   constexpr int kVec = D / 8;  // 16-byte vectors per query row
   constexpr int kMaxGroup = kPrepThreads / 32;
   const int tid = threadIdx.x;
@@ -183,6 +184,8 @@ __global__ void __launch_bounds__(kPrepThreads) cascade_prepare_kernel(const Cas
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) cascade_merge_kernel(const CascadeArgs c,
                                                                          int gh) {
+  grid_dependency_wait();  // the partition states come from the decodes
+  allow_dependents();
   constexpr int kSet = 4;
   const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -273,18 +276,15 @@ cudaError_t launch_cascade_merge(const CascadeArgs& c, int head_dim, int dtype,
   const long long rows = (long long)c.num_seqs * c.num_q_heads;
   const dim3 grid((unsigned)((rows + kMergeWarps - 1) / kMergeWarps));
   const int threads = kMergeWarps * 32;
-  if (dtype == PA_F16) {
-    if (head_dim == 64) cascade_merge_kernel<__half, 64><<<grid, threads, 0, stream>>>(c, gh);
-    else if (head_dim == 128) cascade_merge_kernel<__half, 128><<<grid, threads, 0, stream>>>(c, gh);
-    else return cudaErrorInvalidValue;
-  } else {
-    if (head_dim == 64)
-      cascade_merge_kernel<__nv_bfloat16, 64><<<grid, threads, 0, stream>>>(c, gh);
-    else if (head_dim == 128)
-      cascade_merge_kernel<__nv_bfloat16, 128><<<grid, threads, 0, stream>>>(c, gh);
-    else return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  void (*kern)(const CascadeArgs, int) = nullptr;
+  if (dtype == PA_F16)
+    kern = head_dim == 64 ? cascade_merge_kernel<__half, 64>
+           : head_dim == 128 ? cascade_merge_kernel<__half, 128> : nullptr;
+  else
+    kern = head_dim == 64 ? cascade_merge_kernel<__nv_bfloat16, 64>
+           : head_dim == 128 ? cascade_merge_kernel<__nv_bfloat16, 128> : nullptr;
+  if (!kern) return cudaErrorInvalidValue;
+  return launch_dependent(kern, grid, dim3(threads), 0, stream, c, gh);
 }
 
 }  // namespace pa

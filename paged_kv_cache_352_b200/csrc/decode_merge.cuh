@@ -22,6 +22,8 @@ constexpr int kMergeThreads = 512;
 
 template <typename T, int D, int G, int WARPS>
 __global__ void __launch_bounds__(kMergeThreads) merge_partitions_kernel(const DecodeArgs a) {
+  grid_dependency_wait();  // the partition states come from the decode kernel
+  allow_dependents();
   constexpr int kCols = D / 4;
   constexpr int kSets = kMergeThreads / kCols;
   __shared__ float red[kMergeThreads];

@@ -206,6 +206,20 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
   return old;
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization (launch_dependent) may start while the kernel ahead of it in
+// the stream is still running; grid_dependency_wait() returns once that kernel
+// has completed and its memory operations are visible, and is a no-op in an
+// ordinary launch. allow_dependents() lets the next kernel in the stream launch
+// early (it still waits for this one before reading anything).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void report(int* dev_error, int bit) {
   if (dev_error != nullptr) atomicOr(dev_error, bit);
 }

@@ -37,6 +37,8 @@ constexpr int min_ctas_hint() {
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
 __device__ __forceinline__ void decode_unit(const DecodeArgs& a, const CUtensorMap* tm_k,
                                             const CUtensorMap* tm_v, int kvh, int part, int z) {
+  grid_dependency_wait();  // every input may come from the kernel ahead in the stream
+  allow_dependents();
   constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -171,6 +173,122 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   decode_unit<P, T, D, G, WARPS, STAGES>(a, &tm_k, &tm_v, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
+// One CTA's work with one KV head per warp: warp w serves KV head kvh0 + w of
+// partition `part` of the sequence grid row z serves, streams the whole
+// partition through its own ring and leaves its state (m, l, unnormalised rows)
+// in the workspace: a states-only decode whose warps never wait for each
+// other. The warps of a CTA read the same table entries and have the same
+// number of blocks. Used for the cascade's own blocks: short runs of blocks per
+// (sequence, KV head), WARPS of them per CTA instead of one.
+template <class P, typename T, int D, int G, int WARPS, int STAGES>
+__device__ __forceinline__ void decode_heads_unit(const DecodeArgs& a, const CUtensorMap* tm_k,
+                                                  const CUtensorMap* tm_v, int kvh0, int part,
+                                                  int z) {
+  grid_dependency_wait();
+  allow_dependents();
+  constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + P::kAlign - 1) & ~(uintptr_t)(P::kAlign - 1));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kvh = kvh0 + warp;
+  const int s = a.seq_order ? __ldg(a.seq_order + z) : z;
+  if ((unsigned)s >= (unsigned)a.num_seqs) {
+    if (part == 0 && kvh0 == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
+    return;
+  }
+  if (kvh >= a.num_kv_heads) return;  // the whole warp; no barrier spans warps here
+  const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+  const int b_begin = part * a.part_blocks;
+  int ctx = __ldg(a.context_lens + s);
+  int win = -1;  // lane i holds the table entry of the warp's block win_base + i
+  {
+    const int idx = b_begin + lane;
+    if (lane < a.part_blocks && idx < a.max_blocks_per_seq) win = __ldg(table + idx);
+  }
+  P pol;
+  pol.init(lane);
+  pol.prefetch_q(a, s, kvh);
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * kBS || ctx > a.max_context_len) {
+    if (part == 0 && kvh == 0 && lane == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
+    ctx = 0;
+  }
+  const int nblk = (ctx + kBS - 1) / kBS;
+  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
+  if (part >= nparts) return;  // a sequence with no blocks leaves no state
+  const int my_n = min(nblk, b_begin + a.part_blocks) - b_begin;
+
+  unsigned char* wring = smem + (size_t)warp * STAGES * P::kStageBytes;
+  uint64_t* wbars = reinterpret_cast<uint64_t*>(smem + kRing) + warp * STAGES;
+  int* wvalid = reinterpret_cast<int*>(smem + kRing + WARPS * STAGES * sizeof(uint64_t)) +
+                warp * STAGES;
+  constexpr size_t kHead = kRing + size_t(WARPS) * STAGES * (sizeof(uint64_t) + sizeof(int));
+  unsigned char* scratch =
+      smem + ((kHead + 127) & ~size_t(127)) + (size_t)warp * P::kScratchBytes;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&wbars[st], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  int win_base = 0;
+  auto issue = [&](int j) {
+    if (j >= win_base + 32) {
+      win_base = j & ~31;
+      win = win_base + lane < my_n ? __ldg(table + b_begin + win_base + lane) : -1;
+    }
+    const int phys = __shfl_sync(0xffffffffu, win, j - win_base);
+    if (lane == 0) {
+      const int st = j % STAGES;
+      uint64_t* bar = &wbars[st];
+      const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
+      wvalid[st] = ok;
+      if (a.stall_first_block && j == 0) {
+        mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
+      } else if (!ok) {
+        report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
+        mbar_arrive(bar);
+      } else {
+        P::issue(a, tm_k, tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
+      }
+    }
+  };
+  for (int j = 0; j < STAGES && j < my_n; ++j) issue(j);
+  int issued = my_n < STAGES ? my_n : STAGES;
+  pol.begin(a.scale_log2);
+
+  bool aborted = a.stall_first_block && my_n > 0 &&
+                 !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
+  if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+  int j = 0;
+  for (; !aborted && j < my_n; ++j) {
+    const int st = j % STAGES;
+    if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
+      if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+      aborted = true;
+      break;
+    }
+    if (wvalid[st])
+      pol.block(wring + (size_t)st * P::kStageBytes, ctx - (b_begin + j) * kBS, scratch);
+    __syncwarp();
+    if (j + STAGES < my_n) {
+      if (lane == 0) fence_proxy_async_smem();
+      issue(j + STAGES);
+      issued = j + STAGES + 1;
+    }
+  }
+  if (aborted) {
+    for (int k = j; k < issued; ++k)
+      if (!(a.stall_first_block && k == 0))
+        mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
+  }
+  // the partition's state straight from registers: rows [G] of m, l and [G][D] of acc
+  const size_t row = (((size_t)s * a.num_kv_heads + kvh) * a.max_parts + part) * G;
+  pol.to_red(a.ws_m + row, a.ws_l + row, a.ws_acc + row * D, 0, lane);
+}
+
 template <class P1, class P2, int WARPS>
 constexpr int min_ctas_hint2() {
   return min_ctas_hint<P1, WARPS>() < min_ctas_hint<P2, WARPS>() ? min_ctas_hint<P1, WARPS>()
@@ -178,17 +296,20 @@ constexpr int min_ctas_hint2() {
 }
 
 // The cascade's two decodes in one launch: CTAs [0, n1) serve `a1` (the
-// groups' shared prefixes, members' query heads stacked) and the rest serve
-// `a2` (every sequence's own blocks), each CTA index split into (KV head,
-// partition, sequence) with the KV head fastest. The long prefix partitions are
-// scheduled first and the short own-block CTAs fill the SMs behind them, so the
-// launch has one tail instead of two.
+// groups' shared prefixes, members' query heads stacked; one CTA per KV head and
+// partition, its warps on alternate blocks) and the rest serve `a2` (every
+// sequence's own blocks, states only; one warp per KV head, WARPS KV heads per
+// CTA), each CTA index split into (KV head or head group, partition, sequence)
+// with the first fastest. The long prefix partitions are scheduled first and
+// the short own-block CTAs fill the SMs behind them, so the launch has one tail
+// instead of two.
 template <class P1, int G1, class P2, int G2, typename T, int D, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint2<P1, P2, WARPS>()))
     cascade_decode_kernel(const DecodeArgs a1, const DecodeArgs a2,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v) {
   const int hkv = a1.num_kv_heads;
+  const int hg = (hkv + WARPS - 1) / WARPS;  // KV-head groups of the own-block half
   const int n1 = hkv * a1.max_parts * a1.num_seqs;
   int i = blockIdx.x;
   if (i < n1) {
@@ -196,8 +317,9 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint2<P1, P2, WARPS>()))
                                              i / (hkv * a1.max_parts));
   } else {
     i -= n1;
-    decode_unit<P2, T, D, G2, WARPS, STAGES>(a2, &tm_k, &tm_v, i % hkv, (i / hkv) % a2.max_parts,
-                                             i / (hkv * a2.max_parts));
+    decode_heads_unit<P2, T, D, G2, WARPS, STAGES>(a2, &tm_k, &tm_v, (i % hg) * WARPS,
+                                                   (i / hg) % a2.max_parts,
+                                                   i / (hg * a2.max_parts));
   }
 }
 
@@ -212,6 +334,8 @@ template <class P, typename T, int D, int G, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
     paged_decode_warp_parts_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                                    const __grid_constant__ CUtensorMap tm_v) {
+  grid_dependency_wait();
+  allow_dependents();
   constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -448,16 +572,14 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
       wready[dev].store(true, std::memory_order_release);
     }
     dim3 wgrid(a.num_kv_heads, (a.max_parts + WARPS - 1) / WARPS, a.num_seqs);
-    wkern<<<wgrid, WARPS * 32, smem, stream>>>(a, tk, tv);
-    e = cudaGetLastError();
+    e = launch_dependent(wkern, wgrid, dim3(WARPS * 32), smem, stream, a, tk, tv);
     if (e != cudaSuccess || a.states_only) return e;
     dim3 mgrid(a.num_kv_heads * G, a.num_seqs);
-    merge_partitions_kernel<T, D, G, WARPS><<<mgrid, kMergeThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(merge_partitions_kernel<T, D, G, WARPS>, mgrid, dim3(kMergeThreads),
+                            0, stream, a);
   }
   dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
-  kern<<<grid, WARPS * 32, smem, stream>>>(a, tk, tv);
-  return cudaGetLastError();
+  return launch_dependent(kern, grid, dim3(WARPS * 32), smem, stream, a, tk, tv);
 }
 
 // The cascade's two decodes as one launch of cascade_decode_kernel (4 x 2 tiles).
@@ -470,7 +592,8 @@ cudaError_t launch_dual(const DecodeArgs& a1, const DecodeArgs& a2, int dtype,
   const size_t smem = s1 > s2 ? s1 : s2;
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
   const long long n1 = (long long)a1.num_kv_heads * a1.max_parts * a1.num_seqs;
-  const long long n2 = (long long)a2.num_kv_heads * a2.max_parts * a2.num_seqs;
+  const long long n2 =
+      (long long)((a2.num_kv_heads + WARPS - 1) / WARPS) * a2.max_parts * a2.num_seqs;
   if (a1.num_kv_heads != a2.num_kv_heads || n1 + n2 > 0x7fffffffLL) return cudaErrorInvalidValue;
   if (n1 + n2 == 0) return cudaSuccess;
   auto kern = cascade_decode_kernel<P1, G1, P2, G2, T, D, WARPS, STAGES>;
@@ -496,8 +619,8 @@ cudaError_t launch_dual(const DecodeArgs& a1, const DecodeArgs& a2, int dtype,
     e = make_cache_map(&tv, a1.v_cache, rows, D, dtype);
     if (e != cudaSuccess) return e;
   }
-  kern<<<(unsigned)(n1 + n2), WARPS * 32, smem, stream>>>(a1, a2, tk, tv);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3((unsigned)(n1 + n2)), dim3(WARPS * 32), smem, stream, a1, a2,
+                          tk, tv);
 }
 
 // Warps per CTA x stages per warp. 4 x 2 (64 KiB of K/V in flight per CTA at

@@ -720,7 +720,14 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
   const int gsz = 8 / gh;  // members stacked per KV head: 8 query heads in all
   s->last_groups = 0;
   s->last_saved_blocks = 0;
-  if (s->cascade_mode != PA_SCHED_CASCADE_OFF && s->cascade_ws && nseq >= 2 && gsz >= 2) {
+  // Blocks are shared across requests only through the prefix cache, so the
+  // automatic rule has nothing to gain when no request of the batch came in with
+  // its prompt's token ids.
+  bool consider = s->cascade_mode == PA_SCHED_CASCADE_ON;
+  if (s->cascade_mode == PA_SCHED_CASCADE_AUTO)
+    for (int i = 0; i < nseq && !consider; ++i)
+      consider = !s->req(p.batch_request[i]).tokens.empty();
+  if (consider && s->cascade_ws && nseq >= 2 && gsz >= 2) {
     s->ids_tmp.resize(nseq);
     for (int i = 0; i < nseq; ++i)
       s->ids_tmp[i] = pa_sched::seq_of(p.batch_request[i], p.batch_sample[i]);
