@@ -718,6 +718,12 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
     stream = torch.cuda.current_stream(device)
 
     def launch():
+        if runner.groups is not None:   # blocks shared by forks: read once per group
+            L.pa_paged_decode_cascade(out, runner.q, kc, vc, runner.block_tables,
+                                      runner.context_lens, wl.max_context_len, wl.scale,
+                                      runner.groups, runner.cascade_ws, runner.dev_error,
+                                      k_scale=ks, v_scale=vs)
+            return
         L.pa_paged_decode_fp8(out, runner.q, kc, vc, runner.block_tables, runner.context_lens,
                               wl.max_context_len, wl.scale, ks, vs,
                               partition_tokens=runner.partition_tokens or 0,
@@ -741,8 +747,15 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
         raise RuntimeError(f"fp8 decode: device error bits {runner.error_bits()}")
     t = float(np.mean([a.elapsed_time(b) for a, b in ev])) / 1e3
     nbytes = fp8_decode_bytes(wl)
+    kernel = "paged_decode_kernel (E4M3 cache)"
+    if runner.groups is not None:
+        # distinct blocks at one byte per cached element (half the 16-bit K/V bytes)
+        ctx_sum = int(wl.context_lens.astype(np.int64).sum())
+        non_kv = decode_bytes(wl) - ctx_sum * wl.num_kv_heads * wl.head_dim * wl.elem_bytes * 2
+        nbytes = (unique_decode_bytes(wl, runner) - non_kv) // 2 + non_kv
+        kernel = "pa_paged_decode_cascade over E4M3 caches (distinct blocks)"
     achieved = nbytes / t / 1e9
-    return {"kernel": "paged_decode_kernel (E4M3 cache)", "launch_ms": round(t * 1e3, 4),
+    return {"kernel": kernel, "launch_ms": round(t * 1e3, 4),
             "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": round(achieved, 2),
             "frac_of_hbm_peak": round(achieved / peak, 4),
             "decode_tokens_per_s": round(wl.num_seqs / t, 1),
@@ -963,7 +976,7 @@ def measure_config(name: str, args, device, peak: float, peak_kind: str, read_re
         res["logical_decode_gbs"] = round(decode_bytes(wl) / dec_s / 1e9, 2)
         res["plain_decode"] = time_plain_decode(r, device, l2_flush, dec_s)
         res["copy_blocks"] = time_copy_blocks(r, wl, device)
-    elif wl.num_seqs > 4:
+    if wl.num_seqs > 4:
         res["fp8_kv"] = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak,
                                            iters=max(args.steps, 20))
     del r

@@ -42,22 +42,32 @@ __device__ __forceinline__ void e4m3x4_to_half2x2(uint32_t w, uint32_t& lo, uint
 // pairs), and the lane reads its 16 or 32 code bytes of a row in 16-byte loads.
 //
 // Token permutation. S column n of n-tile nt is token (n >> 1) + 4(n & 1) + 8nt,
-// so the S accumulator of lane j holds tokens j, j+4, j+8, j+12, which are also
-// the P.V k-slots 2j, 2j+1, 2j+8, 2j+9 the lane feeds back as the A operand.
-// For V the lane loads those four token rows at its 16 (d = 128) or 8 (d = 64)
-// output dimensions and transposes the 4 x 4 byte blocks with byte permutes:
-// each resulting word is one dimension's codes for the four tokens, low half
-// b0, high half b1.
+// so the S accumulator of lane j holds tokens j, j+4, j+8, j+12 of its head g.
 //
-// Output columns: lane group g (lane / 4) is B column n = g; at d = 128 it owns
-// dimensions 16 c(g) + nt, c(g) = 4(g & 1) + (g >> 1), at d = 64 dimensions
-// 8g + nt. With 128-byte-swizzled tiles (d = 128, 2-D TMA) these choices make
-// every K and V load of a warp bank-conflict free; d = 64 tiles arrive by 1-D
-// bulk copies.
+// P.V as O^T = V^T P^T. The product runs transposed, with the value tile as the
+// A operand (m-tiles of 16 head dimensions, k = tokens) and P^T as B (n = the 8
+// query heads): 8 mma per block at d = 128 instead of 16, with no padding rows.
+// B's k-slots 2j, 2j+1, 2j+8, 2j+9 are the lane's own tokens j, j+4, j+8, j+12,
+// so its p's feed B as they are. For A the lane loads those four token rows at
+// its 16 (d = 128) or 8 (d = 64) dimensions, base + 0 .. 15; row g of m-tile t
+// is dimension base + 2t and row g + 8 is base + 2t + 1, so one byte permute
+// of two rows' words gives a code pair per dimension, converted to the two
+// half pairs of a0 / a1 (tokens j, j+4) or a2 / a3 (tokens j+8, j+12). The
+// accumulator of m-tile t holds dimensions base + 2t, base + 2t + 1 of heads
+// 2j, 2j + 1; their softmax factors come from lanes 4(2j), 4(2j + 1).
+//
+// Lane groups and dimensions: at d = 128 lane group g (lane / 4) owns dimensions
+// 16 c(g) + 0 .. 15, c(g) = 4(g & 1) + (g >> 1), at d = 64 dimensions 8g + 0 .. 7.
+// With 128-byte-swizzled tiles (d = 128, 2-D TMA) these choices make every K and
+// V load of a warp bank-conflict free; d = 64 tiles arrive by 1-D bulk copies.
+// Measured against the former product (P as the 16-row A operand, the value
+// bytes transposed 4 x 4 per lane, 16 mma per block): long-context 275.3 ->
+// 244.3 us, GQA 100.6 -> 88.6 us per launch over 8-bit caches.
 template <typename T, int D, int G>
 struct Fp8TensorPolicy {
   static constexpr int KSTEPS = D / 16;
   static constexpr int NTO = D / 8;    // output n-tiles
+  static constexpr int MT = D / 16;    // m-tiles of O^T = V^T P^T (16 dimensions each)
   static constexpr int CPT = D / 64;   // 16-byte key chunks a lane reads per row
   static constexpr int kTileBytes = kBS * D;
   static constexpr int kStageBytes = 2 * kTileBytes;
@@ -67,17 +77,18 @@ struct Fp8TensorPolicy {
   static constexpr bool kTensorCores = true;
   static constexpr bool kTma2D = kSwizzled;
   static constexpr bool kFp8Cache = true;
-  // Three CTAs per SM (168 registers; the one-warp-per-partition kernels keep
-  // everything in registers). Four CTAs (128 registers) spilled 90-180 bytes a
-  // thread and measured 10 % slower at 4 query heads per KV head and 7 % at 8.
-  static constexpr int kMinCtasPerSm = 3;
+  // Four CTAs per SM (128 registers; at most 20 bytes a thread spill). With the
+  // transposed P.V product the policy needs about 140 registers; capped at 128,
+  // 16 warps per SM measured faster than 12 warps at 142 registers: GQA 88.6 ->
+  // 85.0 us, long-context 244.2 -> 242.0 us.
+  static constexpr int kMinCtasPerSm = 4;
   static_assert(D == 64 || D == 128, "unsupported head_dim");
 
   int g, j;
   uint4 qraw[CPT][2];      // the lane's 16 * CPT query elements of row g (raw T)
   uint32_t qa[KSTEPS][2];  // f16 A fragments (slots 2j,2j+1 and 2j+8,2j+9)
   float m, l, row_scale;
-  float o[NTO][2];
+  float o[MT][4];  // O^T m-tile mt: dims pi(mt, g), pi(mt, g + 8) x heads 2j, 2j + 1
 
   __device__ __forceinline__ void init(int lane) {
     g = lane >> 2;
@@ -127,7 +138,7 @@ struct Fp8TensorPolicy {
     m = -INFINITY;
     l = 0.f;
 #pragma unroll
-    for (int n = 0; n < NTO; ++n) o[n][0] = o[n][1] = 0.f;
+    for (int t = 0; t < MT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
   }
 
   static __device__ __forceinline__ void issue(const DecodeArgs& a, const CUtensorMap* tm_k,
@@ -196,10 +207,16 @@ struct Fp8TensorPolicy {
     const float p2 = exp2f(x[1][0] - mref), p3 = exp2f(x[1][1] - mref);
     l = fmaf(l, alpha, (p0 + p1) + (p2 + p3));
     if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      // this lane's outputs are heads 2j and 2j + 1, whose factors live in
+      // lanes 4(2j) and 4(2j + 1)
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * j);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * j + 4);
 #pragma unroll
-      for (int n = 0; n < NTO; ++n) {
-        o[n][0] *= alpha;
-        o[n][1] *= alpha;
+      for (int t = 0; t < MT; ++t) {
+        o[t][0] *= a0;
+        o[t][1] *= a1;
+        o[t][2] *= a0;
+        o[t][3] *= a1;
       }
     }
     uint32_t pa0, pa2;
@@ -209,7 +226,11 @@ struct Fp8TensorPolicy {
       memcpy(&pa0, &h0, 4);
       memcpy(&pa2, &h2, 4);
     }
-    // ---- O += P V: rows j, j+4, j+8, j+12 at this lane group's dimensions
+    // ---- O^T += V^T P^T: A = V^T (m-tile rows are dimensions, k-slots 2j, 2j+1,
+    // 2j+8, 2j+9 are tokens j, j+4, j+8, j+12), B = P^T (the lane's own p's:
+    // pa0 = tokens j, j+4 and pa2 = j+8, j+12 of head g), N = the 8 heads. Row
+    // g of m-tile mt is dimension base + 2mt, row g + 8 is base + 2mt + 1, where
+    // the lane's 16 (d = 128) or 8 (d = 64) dimensions start at base.
     constexpr int VW = D == 128 ? 4 : 2;  // 32-bit words of codes a lane reads per row
     uint32_t vr[4][VW];
 #pragma unroll
@@ -239,21 +260,16 @@ struct Fp8TensorPolicy {
         }
     }
 #pragma unroll
-    for (int w = 0; w < VW; ++w) {
-      // 4 x 4 byte transpose: y[i] = byte i of rows j, j+4, j+8, j+12
-      const uint32_t t0 = __byte_perm(vr[0][w], vr[1][w], 0x5140);
-      const uint32_t t1 = __byte_perm(vr[0][w], vr[1][w], 0x7362);
-      const uint32_t t2 = __byte_perm(vr[2][w], vr[3][w], 0x5140);
-      const uint32_t t3 = __byte_perm(vr[2][w], vr[3][w], 0x7362);
-      const uint32_t y[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
-                             __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632)};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int nt = 4 * w + i;
-        uint32_t b0, b1;
-        e4m3x4_to_half2x2(y[i], b0, b1);
-        MmaOps<__half>::run(o[nt], pa0, pa2, b0, b1);
-      }
+    for (int t = 0; t < MT; ++t) {
+      const int w = t >> 1;
+      const uint32_t sel = (t & 1) ? 0x7362u : 0x5140u;  // bytes 2(t&1), 2(t&1)+1 of both rows
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_half2x2(__byte_perm(vr[0][w], vr[1][w], sel), a0, a1);
+      e4m3x4_to_half2x2(__byte_perm(vr[2][w], vr[3][w], sel), a2, a3);
+      asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+          "{%8,%9}, {%0,%1,%2,%3};"
+          : "+f"(o[t][0]), "+f"(o[t][1]), "+f"(o[t][2]), "+f"(o[t][3])
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(pa0), "r"(pa2));
     }
   }
 
@@ -261,19 +277,22 @@ struct Fp8TensorPolicy {
                                          int) {
     float lsum = l + __shfl_xor_sync(0xffffffffu, l, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-    if (g < G) {
-      if (j == 0) {
-        red_m[warp * G + g] = m;
-        red_l[warp * G + g] = lsum;
-      }
-      // accumulator columns 2j and 2j+1 of every n-tile
-      const int base0 = 16 * j;
-      const int base1 = D == 128 ? 64 + 16 * j : 16 * j + 8;
-      float* dst = red_acc + (warp * G + g) * D;
+    if (g < G && j == 0) {
+      red_m[warp * G + g] = m;
+      red_l[warp * G + g] = lsum;
+    }
+    // O^T elements: dimensions base + 2t (+1) of heads 2j, 2j + 1
+    const int base = D == 128 ? 16 * (4 * (g & 1) + (g >> 1)) : 8 * g;
 #pragma unroll
-      for (int n = 0; n < NTO; ++n) {
-        dst[base0 + n] = o[n][0];
-        dst[base1 + n] = o[n][1];
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * j + e;
+      if (h < G) {
+        float* dst = red_acc + (warp * G + h) * D + base;
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          dst[2 * t] = o[t][e];
+          dst[2 * t + 1] = o[t][2 + e];
+        }
       }
     }
   }

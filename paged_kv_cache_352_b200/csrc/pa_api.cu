@@ -648,7 +648,7 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
   gpre.part_blocks = lay.g_part_blocks;
   gpre.max_parts = lay.g_parts;
   // Both decodes in one launch where the shapes allow (8 stacked query heads
-  // per KV head over a 16-bit cache), else on two streams.
+  // per KV head), else on two streams.
   if (num_groups > 0 && gg == 8 && gh < 8) {
     const cudaError_t e = launch_cascade_decode(gpre, own, head_dim, gh, dtype, cache_dtype, st);
     if (e == cudaSuccess)

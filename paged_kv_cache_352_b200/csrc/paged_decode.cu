@@ -58,6 +58,14 @@ cudaError_t launch_cascade_decode_bf16_d64(const DecodeArgs& pre, const DecodeAr
                                            int g_own, cudaStream_t stream);
 cudaError_t launch_cascade_decode_bf16_d128(const DecodeArgs& pre, const DecodeArgs& own,
                                             int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_f16_d64_e4m3(const DecodeArgs& pre, const DecodeArgs& own,
+                                               int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_f16_d128_e4m3(const DecodeArgs& pre, const DecodeArgs& own,
+                                                int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_bf16_d64_e4m3(const DecodeArgs& pre, const DecodeArgs& own,
+                                                int g_own, cudaStream_t stream);
+cudaError_t launch_cascade_decode_bf16_d128_e4m3(const DecodeArgs& pre, const DecodeArgs& own,
+                                                 int g_own, cudaStream_t stream);
 
 namespace {
 std::atomic<unsigned long long> g_stall_request{0};
@@ -95,13 +103,22 @@ cudaError_t launch_paged_decode(const DecodeArgs& args, int head_dim, int group,
 
 cudaError_t launch_cascade_decode(const DecodeArgs& pre, const DecodeArgs& own, int head_dim,
                                   int g_own, int dtype, int cache_dtype, cudaStream_t stream) {
-  if (cache_dtype != dtype) return cudaErrorNotSupported;  // 8-bit caches: two launches
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (!fp8 && cache_dtype != dtype) return cudaErrorNotSupported;
   if (dtype == PA_F16) {
-    if (head_dim == 64) return launch_cascade_decode_f16_d64(pre, own, g_own, stream);
-    if (head_dim == 128) return launch_cascade_decode_f16_d128(pre, own, g_own, stream);
+    if (head_dim == 64)
+      return fp8 ? launch_cascade_decode_f16_d64_e4m3(pre, own, g_own, stream)
+                 : launch_cascade_decode_f16_d64(pre, own, g_own, stream);
+    if (head_dim == 128)
+      return fp8 ? launch_cascade_decode_f16_d128_e4m3(pre, own, g_own, stream)
+                 : launch_cascade_decode_f16_d128(pre, own, g_own, stream);
   } else {
-    if (head_dim == 64) return launch_cascade_decode_bf16_d64(pre, own, g_own, stream);
-    if (head_dim == 128) return launch_cascade_decode_bf16_d128(pre, own, g_own, stream);
+    if (head_dim == 64)
+      return fp8 ? launch_cascade_decode_bf16_d64_e4m3(pre, own, g_own, stream)
+                 : launch_cascade_decode_bf16_d64(pre, own, g_own, stream);
+    if (head_dim == 128)
+      return fp8 ? launch_cascade_decode_bf16_d128_e4m3(pre, own, g_own, stream)
+                 : launch_cascade_decode_bf16_d128(pre, own, g_own, stream);
   }
   return cudaErrorNotSupported;
 }

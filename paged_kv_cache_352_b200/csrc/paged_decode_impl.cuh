@@ -611,12 +611,18 @@ cudaError_t launch_dual(const DecodeArgs& a1, const DecodeArgs& a2, int dtype,
   memset(&tk, 0, sizeof(tk));
   memset(&tv, 0, sizeof(tv));
   if (P1::kTma2D || P2::kTma2D) {
-    static_assert(!P1::kFp8Cache && !P2::kFp8Cache, "16-bit caches only");
+    static_assert(P1::kFp8Cache == P2::kFp8Cache, "one cache type");
     const long long rows = (long long)a1.num_blocks * a1.num_kv_heads * kBS;
     if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA row coordinates are int32
-    e = make_cache_map(&tk, a1.k_cache, rows, D, dtype);
-    if (e != cudaSuccess) return e;
-    e = make_cache_map(&tv, a1.v_cache, rows, D, dtype);
+    if constexpr (P1::kFp8Cache) {
+      e = make_fp8_cache_map(&tk, a1.k_cache, rows, D);
+      if (e != cudaSuccess) return e;
+      e = make_fp8_cache_map(&tv, a1.v_cache, rows, D);
+    } else {
+      e = make_cache_map(&tk, a1.k_cache, rows, D, dtype);
+      if (e != cudaSuccess) return e;
+      e = make_cache_map(&tv, a1.v_cache, rows, D, dtype);
+    }
     if (e != cudaSuccess) return e;
   }
   return launch_dependent(kern, dim3((unsigned)(n1 + n2)), dim3(WARPS * 32), smem, stream, a1, a2,
@@ -712,24 +718,38 @@ cudaError_t launch_group(const DecodeArgs& a, int group, int dtype, cudaStream_t
 
 }  // namespace
 
-// The cascade's decodes of a 16-bit cache in one launch: the groups' prefixes
-// with 8 stacked query heads (`pre`, tensor cores) and the own blocks with
-// g_own query heads per KV head (`own`, the policy paged_decode would pick).
-// cudaErrorNotSupported when that shape has no single-launch form (or a
-// PA_DECODE_PATH override is set): the caller then launches the two decodes.
-template <typename T, int D>
+// The cascade's decodes in one launch: the groups' prefixes with 8 stacked
+// query heads (`pre`, tensor cores) and the own blocks with g_own query heads
+// per KV head (`own`, the policy paged_decode would pick), over a cache of T
+// (C = T) or of E4M3 codes (C = E4M3). cudaErrorNotSupported when that shape
+// has no single-launch form (or a PA_DECODE_PATH override is set): the caller
+// then launches the two decodes.
+template <typename T, int D, typename C = T>
 cudaError_t launch_cascade_typed(const DecodeArgs& pre, const DecodeArgs& own, int g_own,
                                  int dtype, cudaStream_t stream) {
-  if (!use_tensor_path(8) || getenv("PA_DECODE_PATH")) return cudaErrorNotSupported;
-  using Pre = TensorPolicy<T, D, 8>;
-  switch (g_own) {
-    case 1:
-      return launch_dual<Pre, 8, CudaCorePolicy<T, D, 1, T>, 1, T, D>(pre, own, dtype, stream);
-    case 2:
-      return launch_dual<Pre, 8, CudaCorePolicy<T, D, 2, T>, 2, T, D>(pre, own, dtype, stream);
-    case 4:
-      return launch_dual<Pre, 8, TensorPolicy<T, D, 4>, 4, T, D>(pre, own, dtype, stream);
-    default: return cudaErrorNotSupported;
+  if (getenv("PA_DECODE_PATH")) return cudaErrorNotSupported;
+  if constexpr (std::is_same<C, E4M3>::value) {
+    using Pre = Fp8TensorPolicy<T, D, 8>;
+    switch (g_own) {
+      case 1:
+        return launch_dual<Pre, 8, Fp8CudaCorePolicy<T, D, 1>, 1, T, D>(pre, own, dtype, stream);
+      case 2:
+        return launch_dual<Pre, 8, Fp8CudaCorePolicy<T, D, 2>, 2, T, D>(pre, own, dtype, stream);
+      case 4:
+        return launch_dual<Pre, 8, Fp8TensorPolicy<T, D, 4>, 4, T, D>(pre, own, dtype, stream);
+      default: return cudaErrorNotSupported;
+    }
+  } else {
+    using Pre = TensorPolicy<T, D, 8>;
+    switch (g_own) {
+      case 1:
+        return launch_dual<Pre, 8, CudaCorePolicy<T, D, 1, T>, 1, T, D>(pre, own, dtype, stream);
+      case 2:
+        return launch_dual<Pre, 8, CudaCorePolicy<T, D, 2, T>, 2, T, D>(pre, own, dtype, stream);
+      case 4:
+        return launch_dual<Pre, 8, TensorPolicy<T, D, 4>, 4, T, D>(pre, own, dtype, stream);
+      default: return cudaErrorNotSupported;
+    }
   }
 }
 

@@ -210,7 +210,7 @@ class DecodeRunner:
         """Kernel launches of the step's decode call."""
         if self.groups is not None:
             # prepare, both decodes in one launch (8 stacked query heads per KV
-            # head over a 16-bit cache; else two launches), merge
+            # head; else two launches), merge
             g = self.wl.num_q_heads // self.wl.num_kv_heads
             return 3 if g * self.groups.group_size == 8 and g < 8 else 4
         wl = self.wl
