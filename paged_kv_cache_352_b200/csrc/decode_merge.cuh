@@ -13,11 +13,13 @@ namespace {
 
 // Second pass of the warp-per-partition split: one CTA per (sequence, query
 // head) merges that row's states in logical order,
-//   out = sum_p exp2(m_p - M) acc_p / sum_p exp2(m_p - M) l_p,  M = max_p m_p,
-// each thread owning a float4 of columns for the states p = set (mod kSets);
-// the sets are added in a fixed order. A state covers the WARPS consecutive
-// partitions of one decode CTA (merged on chip), so a sequence of n partitions
-// has ceil(n / WARPS) of them.
+//   out = sum_p exp2(m_p - M) acc_p / sum_p exp2(m_p - M) l_p,  M = max_p m_p.
+// A state covers the WARPS consecutive partitions of one decode CTA (merged on
+// chip), so a sequence of n partitions has ceil(n / WARPS) of them. Thread
+// (set, col) owns a float4 of columns and the states p = set (mod kSets), which
+// it merges in one pass with a running maximum, loading kInFlight states per
+// round; the kSets partial states then merge in shared memory in set order.
+// The result depends only on the number of states.
 constexpr int kMergeThreads = 512;
 
 template <typename T, int D, int G, int WARPS>
@@ -26,8 +28,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partitions_kernel(const D
   allow_dependents();
   constexpr int kCols = D / 4;
   constexpr int kSets = kMergeThreads / kCols;
-  __shared__ float red[kMergeThreads];
-  __shared__ float4 part_sum[kSets][kCols];
+  constexpr int kInFlight = 4;
+  __shared__ float set_m[kSets], set_l[kSets];
+  __shared__ float4 set_acc[kSets][kCols];
   const int kvh = blockIdx.x / G;
   const int g = blockIdx.x - kvh * G;
   const int s = blockIdx.y;
@@ -42,81 +45,76 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partitions_kernel(const D
     return;
   }
   const size_t base = ((size_t)s * a.num_kv_heads + kvh) * a.max_parts * G + g;
-  // M, then L, by fixed-order block reductions
-  float m = -INFINITY;
-  for (int p = tid; p < nparts; p += blockDim.x) m = fmaxf(m, __ldcg(a.ws_m + base + (size_t)p * G));
-  red[tid] = m;
-  __syncthreads();
-  for (int w = kMergeThreads / 2; w > 0; w >>= 1) {
-    if (tid < w) red[tid] = fmaxf(red[tid], red[tid + w]);
-    __syncthreads();
-  }
-  const float M = red[0] == -INFINITY ? 0.f : red[0];
-  __syncthreads();
-  float l = 0.f;
-  for (int p = tid; p < nparts; p += blockDim.x)
-    l += exp2f(__ldcg(a.ws_m + base + (size_t)p * G) - M) * __ldcg(a.ws_l + base + (size_t)p * G);
-  red[tid] = l;
-  __syncthreads();
-  for (int w = kMergeThreads / 2; w > 0; w >>= 1) {
-    if (tid < w) red[tid] += red[tid + w];
-    __syncthreads();
-  }
-  const float L = red[0];
+  const float4* acc = reinterpret_cast<const float4*>(a.ws_acc) + base * kCols;
   const int col = tid % kCols;
   const int set = tid / kCols;
-  const float4* acc = reinterpret_cast<const float4*>(a.ws_acc) + base * kCols;
-  float4 sum[4];
+  float M = -INFINITY, L = 0.f;
+  float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p0 = set; p0 < nparts; p0 += kInFlight * kSets) {
+    float m[kInFlight], l[kInFlight];
+    float4 v[kInFlight];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-  int p = set;
-  for (; p + 3 * kSets < nparts; p += 4 * kSets) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int q = p + u * kSets;
-      const float w = exp2f(__ldcg(a.ws_m + base + (size_t)q * G) - M);
-      const float4 v = __ldcg(acc + (size_t)q * G * kCols + col);
-      sum[u].x = fmaf(w, v.x, sum[u].x);
-      sum[u].y = fmaf(w, v.y, sum[u].y);
-      sum[u].z = fmaf(w, v.z, sum[u].z);
-      sum[u].w = fmaf(w, v.w, sum[u].w);
+    for (int u = 0; u < kInFlight; ++u) {
+      const int p = p0 + u * kSets;
+      m[u] = -INFINITY;
+      l[u] = 0.f;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (p < nparts) {
+        m[u] = __ldcg(a.ws_m + base + (size_t)p * G);
+        l[u] = __ldcg(a.ws_l + base + (size_t)p * G);
+        v[u] = __ldcg(acc + (size_t)p * G * kCols + col);
+      }
     }
-  }
+    float Mn = M;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {  // at most three partitions of this set are left
-    const int q = p + u * kSets;
-    if (q < nparts) {
-      const float w = exp2f(__ldcg(a.ws_m + base + (size_t)q * G) - M);
-      const float4 v = __ldcg(acc + (size_t)q * G * kCols + col);
-      sum[u].x = fmaf(w, v.x, sum[u].x);
-      sum[u].y = fmaf(w, v.y, sum[u].y);
-      sum[u].z = fmaf(w, v.z, sum[u].z);
-      sum[u].w = fmaf(w, v.w, sum[u].w);
+    for (int u = 0; u < kInFlight; ++u) Mn = fmaxf(Mn, m[u]);
+    if (Mn == -INFINITY) continue;  // only empty partitions so far
+    const float sc = exp2f(M - Mn);  // 0 while M is still -inf
+    L *= sc;
+    A.x *= sc;
+    A.y *= sc;
+    A.z *= sc;
+    A.w *= sc;
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      const float w = exp2f(m[u] - Mn);
+      L = fmaf(w, l[u], L);
+      A.x = fmaf(w, v[u].x, A.x);
+      A.y = fmaf(w, v[u].y, A.y);
+      A.z = fmaf(w, v[u].z, A.z);
+      A.w = fmaf(w, v[u].w, A.w);
     }
+    M = Mn;
   }
-  float4 t;
-  t.x = (sum[0].x + sum[1].x) + (sum[2].x + sum[3].x);
-  t.y = (sum[0].y + sum[1].y) + (sum[2].y + sum[3].y);
-  t.z = (sum[0].z + sum[1].z) + (sum[2].z + sum[3].z);
-  t.w = (sum[0].w + sum[1].w) + (sum[2].w + sum[3].w);
-  part_sum[set][col] = t;
+  set_acc[set][col] = A;
+  if (col == 0) {
+    set_m[set] = M;
+    set_l[set] = L;
+  }
   __syncthreads();
-  if (set == 0) {
-    float4 r = part_sum[0][col];
+  if (set != 0) return;
+  float Mt = -INFINITY;
 #pragma unroll
-    for (int k = 1; k < kSets; ++k) {
-      r.x += part_sum[k][col].x;
-      r.y += part_sum[k][col].y;
-      r.z += part_sum[k][col].z;
-      r.w += part_sum[k][col].w;
-    }
-    const float f = L > 0.f ? a.out_scale / L : 0.f;
-    T o[4] = {Storage<T>::from_f32(r.x * f), Storage<T>::from_f32(r.y * f),
-              Storage<T>::from_f32(r.z * f), Storage<T>::from_f32(r.w * f)};
-    uint2 packed;
-    memcpy(&packed, o, sizeof(packed));
-    *reinterpret_cast<uint2*>(out + 4 * col) = packed;
+  for (int k = 0; k < kSets; ++k) Mt = fmaxf(Mt, set_m[k]);
+  const float Mref = Mt == -INFINITY ? 0.f : Mt;
+  float Lt = 0.f;
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < kSets; ++k) {
+    const float w = exp2f(set_m[k] - Mref);  // 0 for a set that saw no state
+    const float4 x = set_acc[k][col];
+    Lt = fmaf(w, set_l[k], Lt);
+    r.x = fmaf(w, x.x, r.x);
+    r.y = fmaf(w, x.y, r.y);
+    r.z = fmaf(w, x.z, r.z);
+    r.w = fmaf(w, x.w, r.w);
   }
+  const float f = Lt > 0.f ? a.out_scale / Lt : 0.f;
+  T o[4] = {Storage<T>::from_f32(r.x * f), Storage<T>::from_f32(r.y * f),
+            Storage<T>::from_f32(r.z * f), Storage<T>::from_f32(r.w * f)};
+  uint2 packed;
+  memcpy(&packed, o, sizeof(packed));
+  *reinterpret_cast<uint2*>(out + 4 * col) = packed;
 }
 
 }  // namespace
