@@ -90,7 +90,8 @@ int pa_version(void);
  * on-chip wait of the decode kernels is bounded and gives up with
  * PA_DEVERR_WAIT_TIMEOUT instead of spinning. This call lets a test drive that
  * path without a fault: the next decode kernel launch in the process (by any
- * pa_paged_decode* call) has each warp arm the barrier of its first block
+ * pa_paged_decode* call; for pa_paged_decode_cascade* the launch that decodes
+ * the shared and the own blocks) has each warp arm the barrier of its first block
  * without issuing the block's copy, and lowers the limit of the main loop's
  * waits to wait_limit_ns. That wait runs out, the warp reports
  * PA_DEVERR_WAIT_TIMEOUT, still waits (with the normal 1 s limit) for the

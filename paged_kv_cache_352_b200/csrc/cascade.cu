@@ -65,7 +65,8 @@ __device__ void write_own_table(const CascadeArgs& c, int s, int first) {
 template <int D>
 __global__ void __launch_bounds__(kPrepThreads) cascade_prepare_kernel(const CascadeArgs c,
                                                                         int gh, int copy_ctas) {
-  allow_dependents();  // the decode launch may start; it waits for this kernel
+  grid_dependency_wait();  // tables, lengths and queries may come from the kernel ahead
+  allow_dependents();      // the decode launch may start; it waits for this kernel
   constexpr int kVec = D / 8;  // 16-byte vectors per query row
   constexpr int kMaxGroup = kPrepThreads / 32;
   const int tid = threadIdx.x;
@@ -194,9 +195,12 @@ __global__ void __launch_bounds__(kMergeWarps * 32) cascade_merge_kernel(const C
   const int h = row - s * c.num_q_heads;
   const int kvh = h / gh, hh = h - kvh * gh;
   const int gg = c.group_size * gh;
+  // three independent loads in one round (prepare writes all three for every sequence)
   const int pb = __ldcg(c.s_pbase + s);
-  const int np = pb < 0 ? 0 : __ldcg(c.s_np + s);
-  const int ob = (__ldcg(c.s_ctx + s) + kBlockSize - 1) / kBlockSize;
+  const int np_raw = __ldcg(c.s_np + s);
+  const int own_ctx = __ldcg(c.s_ctx + s);
+  const int np = pb < 0 ? 0 : np_raw;
+  const int ob = (own_ctx + kBlockSize - 1) / kBlockSize;
   const int no = (ob + c.s_part_blocks - 1) / c.s_part_blocks;
   const size_t pbase = pb < 0 ? 0 : (size_t)pb + (size_t)kvh * c.g_parts * gg + hh;
   const size_t obase = ((size_t)s * c.num_kv_heads + kvh) * c.s_parts * gh + hh;
@@ -261,13 +265,9 @@ cudaError_t launch_cascade_prepare(const CascadeArgs& c, int head_dim, int /*dty
   const long long ctas = (long long)c.num_groups * (1 + copy_ctas) + c.num_seqs;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const dim3 grid((unsigned)ctas);
-  if (head_dim == 64)
-    cascade_prepare_kernel<64><<<grid, kPrepThreads, 0, stream>>>(c, gh, copy_ctas);
-  else if (head_dim == 128)
-    cascade_prepare_kernel<128><<<grid, kPrepThreads, 0, stream>>>(c, gh, copy_ctas);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (head_dim != 64 && head_dim != 128) return cudaErrorInvalidValue;
+  return launch_dependent(head_dim == 64 ? cascade_prepare_kernel<64> : cascade_prepare_kernel<128>,
+                          grid, dim3(kPrepThreads), 0, stream, c, gh, copy_ctas);
 }
 
 cudaError_t launch_cascade_merge(const CascadeArgs& c, int head_dim, int dtype,

@@ -101,10 +101,16 @@ cudaError_t launch_paged_decode(const DecodeArgs& args, int head_dim, int group,
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_cascade_decode(const DecodeArgs& pre, const DecodeArgs& own, int head_dim,
-                                  int g_own, int dtype, int cache_dtype, cudaStream_t stream) {
+cudaError_t launch_cascade_decode(const DecodeArgs& pre_args, const DecodeArgs& own_args,
+                                  int head_dim, int g_own, int dtype, int cache_dtype,
+                                  cudaStream_t stream) {
   const bool fp8 = cache_dtype == PA_FP8_E4M3;
   if (!fp8 && cache_dtype != dtype) return cudaErrorNotSupported;
+  DecodeArgs pre = pre_args, own = own_args;
+  if (const unsigned long long ns = take_stall_request()) {
+    pre.stall_first_block = own.stall_first_block = 1;
+    pre.wait_limit_ns = own.wait_limit_ns = ns;
+  }
   if (dtype == PA_F16) {
     if (head_dim == 64)
       return fp8 ? launch_cascade_decode_f16_d64_e4m3(pre, own, g_own, stream)

@@ -90,3 +90,36 @@ def test_wait_runs_out_and_reports(name, ctx, hq, hkv, dtype, pt, launches):
     assert int(err.item()) == 0
     want = oracle_decode(qb, kb, vb, tables, ctx, scale, dtype)
     assert_close(out_to_f64(out, dtype), want, f"{name}: decode after a timed-out launch")
+
+
+def test_wait_runs_out_in_the_cascade():
+    """The cascade's single decode launch: CTAs over the groups' shared prefixes
+    (tensor cores) and warps over each sample's own blocks, one per KV head."""
+    from tests.test_gpu_cascade import _forest
+    nb, hq, hkv, d = 1200, 4, 4, 128
+    bm, batch, ctx = _forest(21, nb)
+    tables = bm.block_tables(batch, max(1, max(-(-int(c) // 16) for c in ctx)))
+    groups = bm.prefix_groups(batch, 8)
+    assert groups.num_groups >= 1
+    kb = gen.normal_bits([61, 1], (nb, hkv, 16, d), "f16")
+    vb = gen.normal_bits([61, 2], (nb, hkv, 16, d), "f16")
+    qb = gen.normal_bits([61, 3], (len(batch), hq, d), "f16")
+    dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.float16).cuda()
+    q, kc, vc = dev(qb), dev(kb), dev(vb)
+    t, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(ctx).cuda()
+    g = groups.to("cuda")
+    ws = pa.cascade_workspace(len(batch), hq, hkv, d, int(ctx.max()), tables.shape[1], g)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    scale = 1 / np.sqrt(d)
+    assert L.lib().pa_test_stall_next_decode(LIMIT_NS) == L.PA_OK
+    pa.pa_paged_decode_cascade(out, q, kc, vc, t, cl, int(ctx.max()), scale, g, ws, dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pa.PA_DEVERR_WAIT_TIMEOUT, "the stalled wait was not reported"
+    err.zero_()
+    pa.pa_paged_decode_cascade(out, q, kc, vc, t, cl, int(ctx.max()), scale, g, ws, dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    want = oracle_decode(qb, kb, vb, tables, ctx, scale, "f16")
+    assert_close(out_to_f64(out, "f16"), want, "cascade after a timed-out launch")
+
