@@ -13,9 +13,10 @@ line's ``per_config`` object.
 Metric: KV-read GB/s (algorithmic bytes of the step / device time of the
 step; % of measured HBM peak alongside) and decode tokens/s.
 
-Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events
-on the launching stream; a barrier + synchronize on both sides of the timed
-region; max over ranks. Every 32 steps a GPU spin (outside the events) keeps
+Timing: W untimed warm-up steps; then K steps, each bracketed by one pair of
+CUDA events on the launching stream, and K decodes alone the same way (the
+roofline); a barrier + synchronize on both sides of the timed region; max over
+ranks. Every 32 steps a GPU spin (outside the events) keeps
 the stream busy while the host enqueues them, so the steps run back to back
 and the events measure device time rather than host issue gaps. Workloads whose inputs exceed 4x the 126 MB L2 run
 without a flush (a cyclic scan larger than the cache reuses nothing); smaller
@@ -841,25 +842,35 @@ def _l2_flusher(wl, r, device, mode: str):
 
 
 def time_steps(r, steps: int, device, l2_flush):
-    """``steps`` steps (copy-on-write copies, cache writes, decode), each bracketed
-    by CUDA events on the launching stream, launched back to back behind a GPU
-    hold every HOLD_EVERY steps. Returns per-step (step seconds, decode seconds)."""
+    """Two timed loops of ``steps`` iterations each, launched back to back behind a
+    GPU hold every HOLD_EVERY iterations, with the L2 rule applied before each.
+    First whole steps (copy-on-write copies, cache writes, decode), one pair of
+    CUDA events around each on the launching stream, so that the step's launches
+    run as they do in use (the decode may start while the cache write ahead of it
+    drains); then the decode alone, for the roofline. Returns per-iteration
+    (step seconds, decode seconds)."""
     import torch
     stream = torch.cuda.current_stream(device)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    for k in range(steps):
-        if k % HOLD_EVERY == 0:
-            gpu_hold(HOLD_EVERY * HOLD_PER_STEP_S)
-        l2_flush()
-        ev[k][0].record(stream)
+
+    def loop(body):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for k in range(steps):
+            if k % HOLD_EVERY == 0:
+                gpu_hold(HOLD_EVERY * HOLD_PER_STEP_S)
+            l2_flush()
+            ev[k][0].record(stream)
+            body()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize(device)
+        return np.array([a.elapsed_time(b) for a, b in ev]) / 1e3
+
+    def step():
         r.copy_blocks()
         r.reshape_and_cache()
-        ev[k][1].record(stream)
         r.decode_step()
-        ev[k][2].record(stream)
-    torch.cuda.synchronize(device)
-    t_step = np.array([ev[k][0].elapsed_time(ev[k][2]) for k in range(steps)]) / 1e3
-    t_dec = np.array([ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)]) / 1e3
+    t_step = loop(step)
+    t_dec = loop(r.decode_step)
     return t_step, t_dec
 
 
@@ -1030,8 +1041,9 @@ def run_ours(args):
     decode_ms = {"mean": round(1e3 * float(t_dec.mean()), 4),
                  "median": round(1e3 * float(np.median(t_dec)), 4),
                  "min": round(1e3 * float(t_dec.min()), 4)}
-    # the step's cache writes (copy-on-write copies + new tokens) before the decode
-    cache_write_ms = round(1e3 * float((t_step - t_dec).mean()), 4)
+    # the step's cache writes (copy-on-write copies + new tokens) before the decode:
+    # what the step costs beyond the decode alone
+    cache_write_ms = round(1e3 * float(t_step.mean() - t_dec.mean()), 4)
     copy_blocks = time_copy_blocks(r, wl, device) if world == 1 else None
     plain_decode = time_plain_decode(r, device, l2_flush, dec_s) \
         if r.groups is not None and world == 1 else None
@@ -1072,7 +1084,8 @@ def run_ours(args):
     value = world * sb / step_s / 1e9
     roofline = decode_roofline(wl, r, dec_s, peak, peak_kind, read_ref)
     csum = clocks.summary()
-    launches_per_step = r.launches_per_step()
+    # the timed region holds K whole steps and then K decodes alone
+    launches_timed = K * (r.launches_per_step() + r.decode_launches())
     fp8 = measure_fp8_decode(wl, r, device, l2_flush, dec_s, peak) \
         if world == 1 and args.only == "all" and r.groups is None else None
     e2e = {"value": round(world * sb / e2e_s / 1e9, 2), "unit": UNIT,
@@ -1147,7 +1160,7 @@ def run_ours(args):
         "shared_blocks": effective, "plain_decode": plain_decode,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": K * launches_per_step,
+        "gpu_launches": launches_timed,
         "per_config": per_config,
         "fp8_kv": fp8,
         "swap": swap,
