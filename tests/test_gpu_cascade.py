@@ -161,8 +161,10 @@ def test_cascade_rejects_a_slot_that_does_not_name_back():
     assert err & pa.PA_DEVERR_GROUP
 
 
-@pytest.mark.parametrize("hq,hkv,d,dt,gs", [(4, 4, 128, "f16", 8), (16, 4, 128, "bf16", 2),
-                                            (4, 4, 64, "f16", 2)])
+# 8 stacked heads (one launch) at 1, 2 and 4 query heads per KV head, and 2 (two launches)
+@pytest.mark.parametrize("hq,hkv,d,dt,gs", [(4, 4, 128, "f16", 8), (8, 4, 128, "bf16", 4),
+                                            (16, 4, 128, "bf16", 2), (4, 4, 64, "f16", 2),
+                                            (8, 4, 64, "f16", 4)])
 def test_cascade_fp8_matches_oracle(hq, hkv, d, dt, gs):
     nb = 900
     bm, batch, ctx = _forest(11 + hq, nb)
