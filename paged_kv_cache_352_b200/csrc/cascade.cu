@@ -12,9 +12,12 @@
 //                                    (2^(m_p - M) l_p + 2^(m_o - M) l_o),
 // which is the decode over the whole context up to floating-point rounding.
 //
-// This file holds the two small kernels around the two decode launches:
-//   cascade_prepare_kernel  validates each group, stacks its queries, writes
-//                           its prefix table and every sequence's own-block table;
+// This file holds the two small kernels around the decode launch(es):
+//   cascade_prepare_kernel  validates each group, writes its prefix table and
+//                           every sequence's own-block table, and stacks the
+//                           members' queries when the prefix decode runs as a
+//                           launch of its own (the single-launch form reads
+//                           them in place and does not wait for this kernel);
 //   cascade_merge_kernel    one warp per output row merges the prefix
 //                           partitions and the own-block partitions.
 #include <cuda_bf16.h>
@@ -58,7 +61,8 @@ __device__ void write_own_table(const CascadeArgs& c, int s, int first) {
 //                                   prefix-state rows;
 //   [num_groups, + num_seqs)        sequence s when no group owns it: its whole table;
 //   [.., + num_groups * copy_ctas)  one query vector per thread of group g's stacked
-//                                   queries.
+//                                   queries (none when the prefix decode reads the
+//                                   members' rows itself: copy_ctas = 0).
 // Every own-block table is written by exactly one CTA. A group CTA loads its
 // members' ids, then their lengths, ownership and prefix entries in one round,
 // and copies the tables in a third.
@@ -257,11 +261,11 @@ __global__ void __launch_bounds__(kMergeWarps * 32) cascade_merge_kernel(const C
 
 }  // namespace
 
-cudaError_t launch_cascade_prepare(const CascadeArgs& c, int head_dim, int /*dtype*/,
+cudaError_t launch_cascade_prepare(const CascadeArgs& c, int head_dim, bool stack_queries,
                                    cudaStream_t stream) {
   const int gh = c.num_q_heads / c.num_kv_heads;
   const long long vecs = (long long)c.num_kv_heads * c.group_size * gh * (head_dim / 8);
-  const int copy_ctas = (int)((vecs + kPrepThreads - 1) / kPrepThreads);
+  const int copy_ctas = stack_queries ? (int)((vecs + kPrepThreads - 1) / kPrepThreads) : 0;
   const long long ctas = (long long)c.num_groups * (1 + copy_ctas) + c.num_seqs;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const dim3 grid((unsigned)ctas);

@@ -360,6 +360,18 @@ struct TensorPolicy {
     }
   }
 
+  // The query row this lane holds (rows >= G are padding), and its load from a
+  // row the caller located (nullptr: a zero row).
+  __device__ __forceinline__ int q_row() const { return r; }
+  __device__ __forceinline__ void load_q_row(const T* row) {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(row);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      qa[kk][0] = row ? __ldg(qrow + kk * 8 + j) : 0u;
+      qa[kk][1] = row ? __ldg(qrow + kk * 8 + 4 + j) : 0u;
+    }
+  }
+
   __device__ __forceinline__ void begin(float scale) {
     scale_log2 = scale;
     m = -INFINITY;

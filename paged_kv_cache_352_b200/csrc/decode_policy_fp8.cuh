@@ -106,6 +106,18 @@ struct Fp8TensorPolicy {
     }
   }
 
+  // The query row this lane holds (rows >= G are padding), and its load from a
+  // row the caller located (nullptr: a zero row).
+  __device__ __forceinline__ int q_row() const { return g; }
+  __device__ __forceinline__ void load_q_row(const T* row) {
+    const uint4* qrow = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+    for (int h = 0; h < CPT; ++h) {
+      qraw[h][0] = row ? __ldg(qrow + 2 * (j + 4 * h)) : make_uint4(0u, 0u, 0u, 0u);
+      qraw[h][1] = row ? __ldg(qrow + 2 * (j + 4 * h) + 1) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
   __device__ __forceinline__ void begin(float scale_log2) {
     float qf[CPT][16];
     float amax = 0.f;

@@ -605,7 +605,13 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
   c.s_parts = lay.s_parts;
   c.s_part_blocks = lay.s_part_blocks;
   c.out_scale = v_scale;
-  if (int e = cuda_status(launch_cascade_prepare(c, head_dim, dtype, st), "cascade prepare launch"))
+  // Both decodes in one launch where the shapes allow (8 stacked query heads
+  // per KV head): its prefix CTAs read the members' query rows and the leader's
+  // table in place, so prepare stacks no queries. Otherwise two decodes on two
+  // streams, the prefix decode over prepare's stacked queries and tables.
+  const bool single = num_groups > 0 && cascade_single_launch(head_dim, gh, gg, dtype, cache_dtype);
+  if (int e = cuda_status(launch_cascade_prepare(c, head_dim, !single, st),
+                          "cascade prepare launch"))
     return e;
 
   // both decodes leave partition states only; the merge writes `out`
@@ -647,13 +653,19 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
   gpre.num_q_heads = num_kv_heads * gg;
   gpre.part_blocks = lay.g_part_blocks;
   gpre.max_parts = lay.g_parts;
-  // Both decodes in one launch where the shapes allow (8 stacked query heads
-  // per KV head), else on two streams.
-  if (num_groups > 0 && gg == 8 && gh < 8) {
-    const cudaError_t e = launch_cascade_decode(gpre, own, head_dim, gh, dtype, cache_dtype, st);
-    if (e == cudaSuccess)
-      return cuda_status(launch_cascade_merge(c, head_dim, dtype, st), "cascade merge launch");
-    if (e != cudaErrorNotSupported) return cuda_status(e, "cascade decode launch");
+  if (single) {
+    gpre.q = q;
+    gpre.block_tables = block_tables;
+    gpre.grp_members = group_members;
+    gpre.grp_prefix_blocks = group_prefix_blocks;
+    gpre.grp_size = group_size;
+    gpre.grp_heads = gh;
+    gpre.grp_src_seqs = num_seqs;
+    gpre.grp_max_prefix_blocks = max_prefix_blocks;
+    if (int e = cuda_status(launch_cascade_decode(gpre, own, head_dim, gh, dtype, cache_dtype, st),
+                            "cascade decode launch"))
+      return e;
+    return cuda_status(launch_cascade_merge(c, head_dim, dtype, st), "cascade merge launch");
   }
   AuxStream* aux = nullptr;
   if (num_groups > 0) {

@@ -83,6 +83,20 @@ struct DecodeArgs {
   int states_only;   // every partition leaves its state in the workspace; nothing writes
                      // `out` and no partitions are merged (a sequence with no blocks
                      // leaves no state): the caller merges them
+  // Rows of shared-prefix groups (the cascade's prefix decode, one launch): when
+  // grp_members is set, sequence index s names group s. Its table is the row of
+  // its leader (member slot 0) in block_tables, its context the group's
+  // grp_prefix_blocks[s] full blocks (none when the leader or that count is out
+  // of range), and query row r of KV head kvh is head kvh * grp_heads + r %
+  // grp_heads of member slot r / grp_heads in q ([grp_src_seqs][Hkv * grp_heads][D];
+  // a zero row for an empty slot). Nothing is read that another kernel of the
+  // same call writes, so these units do not wait for the kernel ahead.
+  const int32_t* grp_members = nullptr;        // [num_seqs][grp_size], -1 pads
+  const int32_t* grp_prefix_blocks = nullptr;  // [num_seqs]
+  int grp_size = 0;
+  int grp_heads = 0;
+  int grp_src_seqs = 0;
+  int grp_max_prefix_blocks = 0;
   // Failure-detection test hook (pa_test_stall_next_decode); both 0 in normal use.
   // stall_first_block: each warp arms the barrier of its first block without
   // issuing the block's copy, so that wait runs out; wait_limit_ns: the limit of
@@ -113,11 +127,13 @@ int decode_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                   int max_context_len, int partition_tokens, bool ordered, DecodeLayout* lay);
 
 // The cascade's decode over the groups' prefixes (`pre`, 8 stacked query heads
-// per KV head) and over every sequence's own blocks (`own`, g_own query heads)
-// as one launch; cudaErrorNotSupported for shapes without that form, for which
-// the two decodes are launched separately.
+// per KV head, located through pre.grp_*) and over every sequence's own blocks
+// (`own`, g_own query heads) as one launch; cudaErrorNotSupported for shapes
+// without that form (cascade_single_launch is false for them), for which the two
+// decodes are launched separately.
 cudaError_t launch_cascade_decode(const DecodeArgs& pre, const DecodeArgs& own, int head_dim,
                                   int g_own, int dtype, int cache_dtype, cudaStream_t stream);
+bool cascade_single_launch(int head_dim, int g_own, int stacked, int dtype, int cache_dtype);
 
 // dtype: query/output type (PA_F16 or PA_BF16); cache_dtype: dtype or PA_FP8_E4M3.
 cudaError_t launch_paged_decode(const DecodeArgs& a, int head_dim, int group, int dtype,
@@ -171,7 +187,7 @@ struct CascadeArgs {
   float out_scale;
 };
 
-cudaError_t launch_cascade_prepare(const CascadeArgs& c, int head_dim, int dtype,
+cudaError_t launch_cascade_prepare(const CascadeArgs& c, int head_dim, bool stack_queries,
                                    cudaStream_t stream);
 cudaError_t launch_cascade_merge(const CascadeArgs& c, int head_dim, int dtype,
                                  cudaStream_t stream);

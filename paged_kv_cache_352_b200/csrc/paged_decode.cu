@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstdlib>
 
 #include "pa_internal.h"
 
@@ -99,6 +100,18 @@ cudaError_t launch_paged_decode(const DecodeArgs& args, int head_dim, int group,
                                     : launch_decode_bf16_d128(a, group, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+// Whether launch_cascade_decode has a form for this shape: 8 stacked heads per
+// KV head over 1, 2 or 4 own query heads per KV head, a supported head_dim and
+// query type, a cache of the query type or of E4M3 codes, and no
+// PA_DECODE_PATH override (which forces one policy for every decode).
+bool cascade_single_launch(int head_dim, int g_own, int stacked, int dtype, int cache_dtype) {
+  if (getenv("PA_DECODE_PATH")) return false;
+  if (stacked != 8 || (g_own != 1 && g_own != 2 && g_own != 4)) return false;
+  if (head_dim != 64 && head_dim != 128) return false;
+  if (dtype != PA_F16 && dtype != PA_BF16) return false;
+  return cache_dtype == dtype || cache_dtype == PA_FP8_E4M3;
 }
 
 cudaError_t launch_cascade_decode(const DecodeArgs& pre_args, const DecodeArgs& own_args,

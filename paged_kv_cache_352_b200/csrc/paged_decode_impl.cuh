@@ -32,12 +32,16 @@ constexpr int min_ctas_hint() {
 }
 
 // One CTA's work: (KV head kvh, partition part) of the sequence that grid row z
-// serves. The body of paged_decode_kernel, and of each half of the cascade's
-// two-part kernel.
-template <class P, typename T, int D, int G, int WARPS, int STAGES>
+// serves. The body of paged_decode_kernel, and of the prefix half of the
+// cascade's two-part kernel (kGroupRows: z is a shared-prefix group, whose
+// table, context and query rows are located through a.grp_*).
+template <class P, typename T, int D, int G, int WARPS, int STAGES, bool kGroupRows = false>
 __device__ __forceinline__ void decode_unit(const DecodeArgs& a, const CUtensorMap* tm_k,
                                             const CUtensorMap* tm_v, int kvh, int part, int z) {
-  grid_dependency_wait();  // every input may come from the kernel ahead in the stream
+  // Every input may come from the kernel ahead in the stream. A group unit reads
+  // only the caller's inputs: the kernel ahead of it (the cascade's prepare) has
+  // itself waited for everything before it, before letting this launch start.
+  if constexpr (!kGroupRows) grid_dependency_wait();
   allow_dependents();
   constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
   extern __shared__ unsigned char smem_raw[];
@@ -54,9 +58,24 @@ __device__ __forceinline__ void decode_unit(const DecodeArgs& a, const CUtensorM
   // Independent loads first, so their latencies overlap: the context length,
   // this warp's first 32 block-table entries (lane i holds the entry of the
   // warp's block i; entries past the sequence are padding, never used) and q.
-  const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+  const int32_t* table;
+  int ctx;
+  if constexpr (kGroupRows) {
+    // the leader's table over the group's full prefix blocks
+    int leader = __ldg(a.grp_members + (size_t)s * a.grp_size);
+    int pb = __ldg(a.grp_prefix_blocks + s);
+    if ((unsigned)leader >= (unsigned)a.grp_src_seqs || pb < 1 || pb > a.grp_max_prefix_blocks ||
+        pb * kBS > a.max_context_len) {
+      leader = 0;  // a rejected group (its members are decoded without it)
+      pb = 0;
+    }
+    table = a.block_tables + (size_t)leader * a.max_blocks_per_seq;
+    ctx = pb * kBS;
+  } else {
+    table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+    ctx = __ldg(a.context_lens + s);
+  }
   const int b_begin = part * a.part_blocks;
-  int ctx = __ldg(a.context_lens + s);
   int win_base = 0;  // the window covers this warp's blocks win_base .. win_base + 31
   int win = -1;
   {
@@ -65,7 +84,21 @@ __device__ __forceinline__ void decode_unit(const DecodeArgs& a, const CUtensorM
   }
   P pol;
   pol.init(lane);
-  pol.prefetch_q(a, s, kvh);
+  if constexpr (kGroupRows) {
+    // stacked row r: head r % grp_heads of member slot r / grp_heads
+    const int r = pol.q_row();
+    const T* row = nullptr;
+    if (r < G) {
+      const int slot = r / a.grp_heads;
+      const int m = __ldg(a.grp_members + (size_t)s * a.grp_size + slot);
+      if ((unsigned)m < (unsigned)a.grp_src_seqs)
+        row = reinterpret_cast<const T*>(a.q) +
+              (((size_t)m * a.num_kv_heads + kvh) * a.grp_heads + (r - slot * a.grp_heads)) * D;
+    }
+    pol.load_q_row(row);
+  } else {
+    pol.prefetch_q(a, s, kvh);
+  }
 
   if (ctx < 0 || ctx > a.max_blocks_per_seq * kBS || ctx > a.max_context_len) {
     if (part == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
@@ -296,8 +329,8 @@ constexpr int min_ctas_hint2() {
 }
 
 // The cascade's two decodes in one launch: CTAs [0, n1) serve `a1` (the
-// groups' shared prefixes, members' query heads stacked; one CTA per KV head and
-// partition, its warps on alternate blocks) and the rest serve `a2` (every
+// groups' shared prefixes, members' query heads stacked, read through the group
+// descriptors; one CTA per KV head and partition, its warps on alternate blocks) and the rest serve `a2` (every
 // sequence's own blocks, states only; one warp per KV head, WARPS KV heads per
 // CTA), each CTA index split into (KV head or head group, partition, sequence)
 // with the first fastest. The long prefix partitions are scheduled first and
@@ -313,8 +346,9 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint2<P1, P2, WARPS>()))
   const int n1 = hkv * a1.max_parts * a1.num_seqs;
   int i = blockIdx.x;
   if (i < n1) {
-    decode_unit<P1, T, D, G1, WARPS, STAGES>(a1, &tm_k, &tm_v, i % hkv, (i / hkv) % a1.max_parts,
-                                             i / (hkv * a1.max_parts));
+    decode_unit<P1, T, D, G1, WARPS, STAGES, true>(a1, &tm_k, &tm_v, i % hkv,
+                                                   (i / hkv) % a1.max_parts,
+                                                   i / (hkv * a1.max_parts));
   } else {
     i -= n1;
     decode_heads_unit<P2, T, D, G2, WARPS, STAGES>(a2, &tm_k, &tm_v, (i % hg) * WARPS,
