@@ -723,7 +723,7 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
             L.pa_paged_decode_cascade(out, runner.q, kc, vc, runner.block_tables,
                                       runner.context_lens, wl.max_context_len, wl.scale,
                                       runner.groups, runner.cascade_ws, runner.dev_error,
-                                      k_scale=ks, v_scale=vs)
+                                      k_scale=ks, v_scale=vs, seq_order=runner.cascade_order)
             return
         L.pa_paged_decode_fp8(out, runner.q, kc, vc, runner.block_tables, runner.context_lens,
                               wl.max_context_len, wl.scale, ks, vs,

@@ -281,6 +281,15 @@ int pa_paged_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
  * by index), the recommended seq_order. Both arrays are host memory. */
 int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order);
 
+/* Host helper for pa_paged_decode_cascade: order[0..n) = sequence indices by
+ * decreasing tokens after their group's prefix (context_lens[i] -
+ * block_size * group_prefix_blocks[seq_group[i]] for a sequence in a group,
+ * context_lens[i] otherwise; ties by index), the recommended seq_order. All
+ * arrays are host memory, as pa_bm_prefix_groups writes them; seq_group and
+ * group_prefix_blocks may be NULL when num_groups is 0. */
+int pa_cascade_order(const int32_t* context_lens, const int32_t* seq_group,
+                     const int32_t* group_prefix_blocks, int num_groups, int n, int32_t* order);
+
 int pa_paged_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int max_blocks_per_seq,
                     const int32_t* context_lens, const int32_t* seq_order, int num_seqs,
@@ -339,24 +348,37 @@ int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache, const
  * systems": copy-on-write sharing; "PagedAttention: The vLLM Paper",
  * "Implementation Essentials": prefix sharing). pa_paged_decode reads such a
  * block once per sequence; this call reads it once per group:
- *   1. a prepare kernel checks each group, stacks its members' query heads as
- *      one KV head's query group and writes the group's prefix table and every
- *      sequence's table of the blocks after its prefix;
- *   2. one decode over the groups' prefix blocks (group_size * G query heads
- *      per KV head), leaving its partition states in the workspace;
- *   3. one decode over every sequence's remaining blocks, likewise;
+ *   1. a prepare kernel checks each group and writes every sequence's table of
+ *      the blocks after its prefix (and, for the two-launch form below, the
+ *      group's prefix table and its members' stacked query heads);
+ *   2. a decode over the groups' prefix blocks (group_size * G query heads per
+ *      KV head: the members' heads stacked as one KV head's query group),
+ *      leaving its partition states in the workspace;
+ *   3. a decode over every sequence's remaining blocks, likewise;
  *   4. a merge of the two sets of softmax states per output row.
- * Step 2 runs on a second stream of the library's, beside step 3 on `stream`,
- * forked after step 1 and joined before step 4 by events; the call is ordered
- * on `stream` like any other. The library makes that stream and its two events
- * on a host thread's first cascade call on a device and keeps them for the
- * life of the process.
+ * When group_size * G is 8 and G < 8, steps 2 and 3 are one launch whose
+ * prefix CTAs come first and read the leader's table and the members' query
+ * rows in place: they start while step 1 runs. Otherwise step 2 runs on a
+ * second stream of the library's, beside step 3 on `stream`, forked after
+ * step 1 and joined before step 4 by events; the library makes that stream and
+ * its two events on a host thread's first such call on a device and keeps them
+ * for the life of the process. Either way the call is ordered on `stream` like
+ * any other.
  * The result is the decode of pa_paged_decode up to floating-point rounding
  * (the same fp32 arithmetic summed in another order).
  *
- * Arguments as for pa_paged_decode (no seq_order, no partition_tokens: both
- * decodes use the library's default split), plus the group descriptor, in
- * device memory, as pa_bm_prefix_groups writes it:
+ * Arguments as for pa_paged_decode (no partition_tokens: both decodes use the
+ * library's default split), plus the group descriptor, in device memory, as
+ * pa_bm_prefix_groups writes it:
+ *   seq_order            device, int32 [num_seqs], a permutation of
+ *                        0..num_seqs-1 giving the order in which the
+ *                        remaining-block decode schedules sequences, or NULL
+ *                        for 0, 1, 2, ...; pa_cascade_order lists them by
+ *                        decreasing length after their prefix, which shortens
+ *                        the launch's tail. Results do not depend on the order;
+ *                        entries outside [0, num_seqs) are flagged
+ *                        (PA_DEVERR_CONTEXT_RANGE) and skipped, and a repeated
+ *                        entry leaves some sequence's output undefined.
  *   group_members        int32 [num_groups][group_size], batch indices, -1 pads;
  *                        slot 0 is the group's leader
  *   group_prefix_blocks  int32 [num_groups]: blocks shared by every member
@@ -371,9 +393,11 @@ int pa_paged_decode_noalloc(void* out, const void* q, const void* k_cache, const
  * names s. A group whose members do not all hold the leader's first prefix
  * blocks as full blocks inside their contexts, or whose descriptor is otherwise
  * inconsistent, is decoded without its prefix (every member over its whole
- * context) and PA_DEVERR_GROUP is set: the outputs stay correct. Host-side
- * errors as for pa_paged_decode. pa_paged_decode_cascade_fp8 decodes E4M3
- * caches with key and value scales, as pa_paged_decode_fp8.
+ * context) and PA_DEVERR_GROUP is set: the outputs stay correct (other bits
+ * may be set too, e.g. PA_DEVERR_BLOCK_RANGE when the claimed prefix runs past
+ * the leader's table). Host-side errors as for pa_paged_decode.
+ * pa_paged_decode_cascade_fp8 decodes E4M3 caches with key and value scales,
+ * as pa_paged_decode_fp8.
  * ------------------------------------------------------------------------- */
 int pa_paged_decode_cascade_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                            int head_dim, int max_context_len,
@@ -382,9 +406,10 @@ int pa_paged_decode_cascade_workspace_size(int num_seqs, int num_q_heads, int nu
 
 int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, int max_blocks_per_seq,
-                            const int32_t* context_lens, int num_seqs, int max_context_len,
-                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                            int num_blocks, float scale, const int32_t* group_members,
+                            const int32_t* context_lens, const int32_t* seq_order,
+                            int num_seqs, int max_context_len, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                            float scale, const int32_t* group_members,
                             const int32_t* group_prefix_blocks, const int32_t* seq_group,
                             const int32_t* seq_member, int num_groups, int group_size,
                             int max_prefix_blocks, void* workspace, size_t workspace_bytes,
@@ -392,9 +417,10 @@ int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const
 
 int pa_paged_decode_cascade_fp8(void* out, const void* q, const void* k_cache,
                                 const void* v_cache, const int32_t* block_tables,
-                                int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
-                                int max_context_len, int num_q_heads, int num_kv_heads,
-                                int head_dim, int block_size, int num_blocks, float scale,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                const int32_t* seq_order, int num_seqs, int max_context_len,
+                                int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, float scale,
                                 float k_scale, float v_scale, const int32_t* group_members,
                                 const int32_t* group_prefix_blocks, const int32_t* seq_group,
                                 const int32_t* seq_member, int num_groups, int group_size,

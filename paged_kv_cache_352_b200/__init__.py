@@ -29,6 +29,7 @@ from ._lib import (  # noqa: F401
     decode_workspace,
     last_error,
     lib,
+    pa_cascade_order,
     pa_copy_blocks,
     pa_longest_first_order,
     pa_paged_decode,

@@ -77,15 +77,16 @@ _SIGS = {
                                      _vp, _c_int, _vp]),
     "pa_paged_decode_cascade_workspace_size": (_c_int, [_c_int] * 10 +
                                                 [ctypes.POINTER(ctypes.c_size_t)]),
-    "pa_paged_decode_cascade": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
-                                         _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
-                                         _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp,
-                                         ctypes.c_size_t, _vp, _c_int, _vp]),
-    "pa_paged_decode_cascade_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int,
+    "pa_paged_decode_cascade": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                         ctypes.c_float, _vp, _vp, _vp, _vp, _c_int, _c_int,
+                                         _c_int, _vp, ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_paged_decode_cascade_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int,
                                              _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                              ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                              _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _vp,
                                              ctypes.c_size_t, _vp, _c_int, _vp]),
+    "pa_cascade_order": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp]),
     "pa_bm_prefix_groups": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                      ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "pa_bm_create": (_c_int, [_c_int, _c_int, _vp, ctypes.POINTER(_vp)]),
@@ -322,6 +323,23 @@ def pa_longest_first_order(context_lens) -> np.ndarray:
     return order
 
 
+def pa_cascade_order(context_lens, groups: "PrefixGroups") -> np.ndarray:
+    """Host int32 order of sequences by decreasing tokens after their group's
+    prefix (ties by index): the recommended ``seq_order`` of
+    ``pa_paged_decode_cascade``."""
+    ctx = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    sg = np.ascontiguousarray(groups.seq_group, dtype=np.int32)
+    gp = np.ascontiguousarray(groups.prefix_blocks, dtype=np.int32)
+    if sg.shape != ctx.shape:
+        raise PAError(PA_ERR_INVALID_ARG, "groups must describe this batch")
+    order = np.empty(len(ctx), np.int32)
+    ng = groups.num_groups
+    _check(lib().pa_cascade_order(ctx.ctypes.data if len(ctx) else None,
+                                  sg.ctypes.data if ng else None, gp.ctypes.data if ng else None,
+                                  ng, len(ctx), order.ctypes.data if len(ctx) else None))
+    return order
+
+
 def pa_paged_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
                     scale, partition_tokens=0, workspace=None, dev_error=None, stream=None,
                     seq_order=None):
@@ -456,11 +474,14 @@ def cascade_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context
 
 def pa_paged_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens,
                             max_context_len, scale, groups: PrefixGroups, workspace,
-                            dev_error=None, stream=None, k_scale=None, v_scale=None):
+                            dev_error=None, stream=None, k_scale=None, v_scale=None,
+                            seq_order=None):
     """Decode attention that reads blocks shared by a group's members once; writes
     ``out`` ``[B, Hq, d]``. ``groups`` comes from ``BlockManager.prefix_groups`` for
     the same batch order, moved to the device (``groups.to(device)``). E4M3 caches
-    take ``k_scale`` and ``v_scale``."""
+    take ``k_scale`` and ``v_scale``. ``seq_order`` (int32 CUDA tensor, a
+    permutation) schedules the own-block decode; ``pa_cascade_order`` gives the
+    recommended one."""
     torch = _torch()
     nb, hkv, bs, d = _cache_dims(k_cache, v_cache)
     B, hq, dq = q.shape
@@ -478,8 +499,9 @@ def pa_paged_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens
         i32 = torch.int32
         head = [_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
                 _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables", i32),
-                block_tables.shape[1], _dev_ptr(context_lens, "context_lens", i32), B,
-                int(max_context_len), hq, hkv, d, bs, nb, float(scale)]
+                block_tables.shape[1], _dev_ptr(context_lens, "context_lens", i32),
+                _order_ptr(seq_order, B), B, int(max_context_len), hq, hkv, d, bs, nb,
+                float(scale)]
         tail = [_dev_ptr(members, "group_members", i32),
                 _dev_ptr(prefix, "group_prefix_blocks", i32), _dev_ptr(sgroup, "seq_group", i32),
                 _dev_ptr(smember, "seq_member", i32),

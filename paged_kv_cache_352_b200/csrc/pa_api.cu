@@ -353,6 +353,26 @@ int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order) {
   return PA_OK;
 }
 
+int pa_cascade_order(const int32_t* context_lens, const int32_t* seq_group,
+                     const int32_t* group_prefix_blocks, int num_groups, int n, int32_t* order) {
+  clear_error();
+  if (n < 0 || num_groups < 0) return fail(PA_ERR_INVALID_ARG, "n and num_groups must be >= 0");
+  if (n == 0) return PA_OK;
+  if (!context_lens || !order || (num_groups > 0 && (!seq_group || !group_prefix_blocks)))
+    return fail(PA_ERR_INVALID_ARG, "null pointer argument");
+  // the tokens a sequence's own-block decode reads: its context after the prefix
+  // of its group (its whole context outside any group)
+  std::vector<int64_t> own(n);
+  for (int i = 0; i < n; ++i) {
+    const int g = num_groups > 0 ? seq_group[i] : -1;
+    const int64_t pre = g >= 0 && g < num_groups ? (int64_t)group_prefix_blocks[g] * kBlockSize : 0;
+    own[i] = std::max<int64_t>(0, (int64_t)context_lens[i] - pre);
+  }
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order, order + n, [&own](int32_t x, int32_t y) { return own[x] > own[y]; });
+  return PA_OK;
+}
+
 }  // extern "C"
 
 namespace {
@@ -537,7 +557,8 @@ int aux_stream(AuxStream** out) {
 
 int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* block_tables, int max_blocks_per_seq,
-                              const int32_t* context_lens, int num_seqs, int max_context_len,
+                              const int32_t* context_lens, const int32_t* seq_order,
+                              int num_seqs, int max_context_len,
                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                               int num_blocks, float scale, float k_scale, float v_scale,
                               const int32_t* group_members, const int32_t* group_prefix_blocks,
@@ -631,6 +652,7 @@ int paged_decode_cascade_impl(void* out, const void* q, const void* k_cache, con
   a.states_only = 1;
   DecodeArgs own = a;
   own.q = q;
+  own.seq_order = seq_order;  // the own-block CTAs in the caller's order
   own.block_tables = c.s_tables;
   own.context_lens = c.s_ctx;
   own.ws_count = reinterpret_cast<int*>(ws + lay.scount_off);
@@ -711,9 +733,10 @@ int pa_paged_decode_cascade_workspace_size(int num_seqs, int num_q_heads, int nu
 
 int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, int max_blocks_per_seq,
-                            const int32_t* context_lens, int num_seqs, int max_context_len,
-                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                            int num_blocks, float scale, const int32_t* group_members,
+                            const int32_t* context_lens, const int32_t* seq_order,
+                            int num_seqs, int max_context_len, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                            float scale, const int32_t* group_members,
                             const int32_t* group_prefix_blocks, const int32_t* seq_group,
                             const int32_t* seq_member, int num_groups, int group_size,
                             int max_prefix_blocks, void* workspace, size_t workspace_bytes,
@@ -721,8 +744,9 @@ int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const
   const NvtxRange nvtx_range("pa_paged_decode_cascade");
   clear_error();
   return paged_decode_cascade_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                                   context_lens, num_seqs, max_context_len, num_q_heads,
-                                   num_kv_heads, head_dim, block_size, num_blocks, scale, 1.f, 1.f,
+                                   context_lens, seq_order, num_seqs, max_context_len,
+                                   num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                   scale, 1.f, 1.f,
                                    group_members, group_prefix_blocks, seq_group, seq_member,
                                    num_groups, group_size, max_prefix_blocks, workspace,
                                    workspace_bytes, dev_error, dtype, dtype, stream);
@@ -730,9 +754,10 @@ int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const
 
 int pa_paged_decode_cascade_fp8(void* out, const void* q, const void* k_cache,
                                 const void* v_cache, const int32_t* block_tables,
-                                int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
-                                int max_context_len, int num_q_heads, int num_kv_heads,
-                                int head_dim, int block_size, int num_blocks, float scale,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                const int32_t* seq_order, int num_seqs, int max_context_len,
+                                int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, float scale,
                                 float k_scale, float v_scale, const int32_t* group_members,
                                 const int32_t* group_prefix_blocks, const int32_t* seq_group,
                                 const int32_t* seq_member, int num_groups, int group_size,
@@ -743,10 +768,10 @@ int pa_paged_decode_cascade_fp8(void* out, const void* q, const void* k_cache,
   if (!positive_finite(k_scale) || !positive_finite(v_scale))
     return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
   return paged_decode_cascade_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                                   context_lens, num_seqs, max_context_len, num_q_heads,
-                                   num_kv_heads, head_dim, block_size, num_blocks, scale, k_scale,
-                                   v_scale, group_members, group_prefix_blocks, seq_group,
-                                   seq_member, num_groups, group_size, max_prefix_blocks,
+                                   context_lens, seq_order, num_seqs, max_context_len,
+                                   num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                   scale, k_scale, v_scale, group_members, group_prefix_blocks,
+                                   seq_group, seq_member, num_groups, group_size, max_prefix_blocks,
                                    workspace, workspace_bytes, dev_error, dtype, PA_FP8_E4M3,
                                    stream);
 }

@@ -800,7 +800,12 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
   off += 4 * (size_t)nseq;
   const size_t off_order = off;
   s->order_tmp.resize(nseq);
-  if (nseq) pa_longest_first_order(p.batch_ctx.data(), nseq, s->order_tmp.data());
+  // longest first; in a cascade step, by the tokens after each sequence's prefix
+  if (nseq && ng)
+    pa_cascade_order(p.batch_ctx.data(), s->sg_tmp.data(), s->gp_tmp.data(), ng, nseq,
+                     s->order_tmp.data());
+  else if (nseq)
+    pa_longest_first_order(p.batch_ctx.data(), nseq, s->order_tmp.data());
   memcpy(h + off, s->order_tmp.data(), 4 * (size_t)nseq);
   off += 4 * (size_t)nseq;
   // group descriptors (cascade steps only): members, prefix lengths, group and slot
@@ -871,13 +876,13 @@ int pa_sched_execute(pa_sched* s, void* k_cache, void* v_cache, void* host_k, vo
       const int32_t* sg = reinterpret_cast<const int32_t*>(dm + off_sg);
       const int32_t* sm = reinterpret_cast<const int32_t*>(dm + off_sm);
       return fp8 ? pa_paged_decode_cascade_fp8(
-                       out, q, k_cache, v_cache, tables, p.max_blocks, ctx, nseq, p.max_ctx,
-                       s->hq, hkv, d, bs, nb, scale, s->k_scale, s->v_scale, gm, gp, sg, sm, ng,
-                       gsz, maxp, s->cascade_ws, s->cascade_ws_bytes, dev_error, s->dtype,
-                       stream)
+                       out, q, k_cache, v_cache, tables, p.max_blocks, ctx, order, nseq,
+                       p.max_ctx, s->hq, hkv, d, bs, nb, scale, s->k_scale, s->v_scale, gm, gp,
+                       sg, sm, ng, gsz, maxp, s->cascade_ws, s->cascade_ws_bytes, dev_error,
+                       s->dtype, stream)
                  : pa_paged_decode_cascade(out, q, k_cache, v_cache, tables, p.max_blocks, ctx,
-                                           nseq, p.max_ctx, s->hq, hkv, d, bs, nb, scale, gm, gp,
-                                           sg, sm, ng, gsz, maxp, s->cascade_ws,
+                                           order, nseq, p.max_ctx, s->hq, hkv, d, bs, nb, scale,
+                                           gm, gp, sg, sm, ng, gsz, maxp, s->cascade_ws,
                                            s->cascade_ws_bytes, dev_error, s->dtype, stream);
     }
     const int r =

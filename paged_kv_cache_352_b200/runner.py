@@ -79,11 +79,15 @@ class DecodeRunner:
         # block once per group of samples (8 / G samples stacked per KV head).
         self.groups = None
         self.cascade_ws = None
+        self.cascade_order = None
         g = wl.num_q_heads // wl.num_kv_heads
         if wl.kind == "shared_prefix" and not duplicate and g <= 4:
             groups = self.bm.prefix_groups(range(wl.num_seqs), 8 // g)
             if groups.num_groups:
                 self.groups = groups.to(self.device)
+                # own blocks longest first (tokens after each sample's prefix)
+                self.cascade_order = torch.from_numpy(
+                    L.pa_cascade_order(self.context_lens_host, groups)).to(self.device)
                 self.cascade_ws = L.cascade_workspace(
                     wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
                     wl.max_context_len, self.max_blocks, self.groups, self.device)
@@ -191,7 +195,8 @@ class DecodeRunner:
         out = self.out if out is None else out
         L.pa_paged_decode_cascade(out, self.q, self.k_cache, self.v_cache, self.block_tables,
                                   self.context_lens, self.wl.max_context_len, self.wl.scale,
-                                  self.groups, self.cascade_ws, self.dev_error)
+                                  self.groups, self.cascade_ws, self.dev_error,
+                                  seq_order=self.cascade_order)
         return out
 
     def decode_step(self, out=None):

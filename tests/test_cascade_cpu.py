@@ -125,8 +125,8 @@ def test_cascade_argument_checks():
         a.update(kw)
         p = dummy.ctypes.data
         return lib.pa_paged_decode_cascade(
-            FAKE, FAKE, FAKE, FAKE, FAKE, a["mb"], FAKE, a["B"], a["maxctx"], a["hq"], a["hkv"],
-            a["d"], a["bs"], a["nb"], 0.1, p, p, p, p, a["ng"], a["gs"], a["mp"], a["ws"],
+            FAKE, FAKE, FAKE, FAKE, FAKE, a["mb"], FAKE, None, a["B"], a["maxctx"], a["hq"],
+            a["hkv"], a["d"], a["bs"], a["nb"], 0.1, p, p, p, p, a["ng"], a["gs"], a["mp"], a["ws"],
             a["wsb"], None, a["dt"], None)
 
     assert call(gs=3) == L.PA_ERR_UNSUPPORTED            # 3 stacked heads per KV head
@@ -175,3 +175,49 @@ def test_prefix_groups_of_empty_and_unshared_batches():
     ws = pa.pa_paged_decode_cascade_workspace_size(4, 8, 8, 64, 300, 19, g.num_groups, 1,
                                                    g.max_prefix_blocks)
     assert ws > 0
+
+
+def _own_tokens_order(ctx, seq_group, prefix_blocks):
+    """The order pa_cascade_order promises, by the rule stated plainly: tokens
+    after the group's prefix (whole context outside a group), longest first,
+    ties by batch index."""
+    own = []
+    for i, c in enumerate(ctx):
+        g = int(seq_group[i])
+        pre = 16 * int(prefix_blocks[g]) if 0 <= g < len(prefix_blocks) else 0
+        own.append(max(0, int(c) - pre))
+    return sorted(range(len(ctx)), key=lambda i: (-own[i], i))
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_cascade_order_lists_own_blocks_longest_first(seed):
+    bm, _, batch = _fork_forest(seed)
+    g = bm.prefix_groups(batch, 4)
+    ctx = np.array([bm.seq_len(s) for s in batch], np.int32)
+    got = pa.pa_cascade_order(ctx, g).tolist()
+    assert got == _own_tokens_order(ctx, g.seq_group, g.prefix_blocks)
+    assert sorted(got) == list(range(len(batch)))
+
+
+def test_cascade_order_edge_cases():
+    lib = L.lib()
+    ctx = np.array([30, 50, 50, 7, 0], np.int32)
+    # no groups: plain longest first, ties by index
+    g0 = L.PrefixGroups(np.zeros((0, 2), np.int32), np.zeros(0, np.int32),
+                        np.full(5, -1, np.int32), np.full(5, -1, np.int32), 2, 0)
+    assert pa.pa_cascade_order(ctx, g0).tolist() == [1, 2, 0, 3, 4]
+    # a group of sequences 1 and 2 with 3 shared blocks (48 tokens): 2 and 2 own
+    # tokens; a group index past num_groups counts as no group; a prefix longer
+    # than the context counts as 0 own tokens
+    sg = np.array([1, 0, 0, 7, 1], np.int32)
+    pb = np.array([3, 4], np.int32)
+    g = L.PrefixGroups(np.array([[1, 2], [0, 4]], np.int32), pb, sg,
+                       np.array([0, 0, 1, -1, 1], np.int32), 2, 4)
+    assert pa.pa_cascade_order(ctx, g).tolist() == _own_tokens_order(ctx, sg, pb)
+    assert pa.pa_cascade_order(ctx, g).tolist() == [3, 1, 2, 0, 4]
+    out = np.empty(5, np.int32)
+    assert lib.pa_cascade_order(ctx.ctypes.data, None, None, 1, 5,
+                                out.ctypes.data) == L.PA_ERR_INVALID_ARG
+    assert lib.pa_cascade_order(None, None, None, 0, 0, None) == L.PA_OK
+    assert lib.pa_cascade_order(ctx.ctypes.data, None, None, 0, -1,
+                                out.ctypes.data) == L.PA_ERR_INVALID_ARG

@@ -60,7 +60,11 @@ def _forest(seed, nb, exact=False):
     return bm, batch, ctx
 
 
-def _run(bm, batch, ctx, hq, hkv, d, dt, nb, seed, group_size, corrupt=None, fp8=None):
+def _run(bm, batch, ctx, hq, hkv, d, dt, nb, seed, group_size, corrupt=None, fp8=None,
+         order=None, keep=None):
+    """order: None, "cascade" (pa_cascade_order) or "random" (a seeded
+    permutation) as the call's seq_order; keep: a dict that receives the raw
+    output bits under "out"."""
     mb = int(max(1, max(-(-int(c) // 16) for c in ctx)))
     tables = bm.block_tables(batch, mb)
     groups = bm.prefix_groups(batch, group_size)
@@ -75,11 +79,16 @@ def _run(bm, batch, ctx, hq, hkv, d, dt, nb, seed, group_size, corrupt=None, fp8
     g = groups.to("cuda")
     ws = pa.cascade_workspace(B, hq, hkv, d, maxctx, mb, g)
     td, cd = torch.from_numpy(tables).cuda(), torch.from_numpy(ctx).cuda()
+    so = None
+    if order == "cascade":
+        so = torch.from_numpy(pa.pa_cascade_order(ctx, groups)).cuda()
+    elif order == "random":
+        so = torch.from_numpy(np.random.default_rng([seed, 7]).permutation(B).astype(np.int32)).cuda()
     if fp8 is None:
         kb = gen.normal_bits([seed, 1], (nb, hkv, 16, d), dt)
         vb = gen.normal_bits([seed, 2], (nb, hkv, 16, d), dt)
         pa.pa_paged_decode_cascade(out, _dev(q, dt), _dev(kb, dt), _dev(vb, dt), td, cd, maxctx,
-                                   scale, g, ws, dev_error=err)
+                                   scale, g, ws, dev_error=err, seq_order=so)
         want = paged_decode(q, kb, vb, tables, ctx, scale, dt)
     else:
         ks, vs = fp8
@@ -88,9 +97,11 @@ def _run(bm, batch, ctx, hq, hkv, d, dt, nb, seed, group_size, corrupt=None, fp8
                   (rng.integers(0, 2, (nb, hkv, 16, d)) << 7)).astype(np.uint8) for _ in range(2)]
         pa.pa_paged_decode_cascade(out, _dev(q, dt), torch.from_numpy(codes[0]).cuda(),
                                    torch.from_numpy(codes[1]).cuda(), td, cd, maxctx, scale, g,
-                                   ws, dev_error=err, k_scale=ks, v_scale=vs)
+                                   ws, dev_error=err, k_scale=ks, v_scale=vs, seq_order=so)
         want = F.paged_decode_fp8(q, codes[0], codes[1], tables, ctx, scale, ks, vs, dt)
     torch.cuda.synchronize()
+    if keep is not None:
+        keep["out"] = tensor_bits(out)
     got = out_to_f64(out, dt)
     for s in range(B):
         assert_close(got[s], want[s], f"seq {s} ctx {ctx[s]}")
@@ -111,6 +122,37 @@ def test_cascade_matches_oracle(hq, hkv, d, dt, gs, seed):
     err, groups = _run(bm, batch, ctx, hq, hkv, d, dt, nb, seed, gs)
     assert err == 0
     assert groups.num_groups >= 1
+
+
+# one launch (8 stacked heads) and two (2 stacked heads)
+@pytest.mark.parametrize("hq,hkv,d,dt,gs", [SHAPES[0], SHAPES[1], SHAPES[4]])
+def test_cascade_results_do_not_depend_on_the_order(hq, hkv, d, dt, gs):
+    """The own-block decode scheduled in pa_cascade_order's order and in a random
+    permutation: outputs bit-identical to the call without an order, and within
+    tolerance of the oracle."""
+    nb = 1200
+    runs = {}
+    for order in (None, "cascade", "random"):
+        bm, batch, ctx = _forest(41 + hq, nb)
+        keep = {}
+        err, groups = _run(bm, batch, ctx, hq, hkv, d, dt, nb, 3, gs, order=order, keep=keep)
+        assert err == 0 and groups.num_groups >= 1
+        runs[order] = keep["out"]
+    assert np.array_equal(runs[None], runs["cascade"])
+    assert np.array_equal(runs[None], runs["random"])
+
+
+def test_cascade_fp8_results_do_not_depend_on_the_order():
+    nb = 900
+    runs = {}
+    for order in (None, "cascade"):
+        bm, batch, ctx = _forest(19, nb)
+        keep = {}
+        err, _ = _run(bm, batch, ctx, 8, 4, 128, "bf16", nb, 12, 4, fp8=(0.05, 0.02),
+                      order=order, keep=keep)
+        assert err == 0
+        runs[order] = keep["out"]
+    assert np.array_equal(runs[None], runs["cascade"])
 
 
 @pytest.mark.parametrize("hq,hkv,d,dt,gs", SHAPES[:2])
@@ -142,6 +184,29 @@ def test_cascade_rejects_a_member_without_the_prefix():
         return tables, groups
 
     err, _ = _run(bm, batch, ctx, 4, 4, 128, "f16", nb, 4, 8, corrupt=corrupt)
+    assert err & pa.PA_DEVERR_GROUP
+
+
+def test_cascade_rejects_a_prefix_past_the_members_contexts():
+    """A group claims one more shared block than its leader holds (still within
+    the batch's longest context): the prefix decode reads past the leader's
+    blocks, the group is rejected and flagged, and every output still matches
+    the oracle."""
+    nb = 1200
+    bm, batch, ctx = _forest(5, nb)
+    cap = int(ctx.max()) // 16
+
+    def corrupt(tables, groups):
+        for k in range(groups.num_groups):
+            leader = int(groups.members[k][0])
+            held = int((tables[leader] >= 0).sum())
+            if held + 1 <= cap:
+                groups.prefix_blocks[k] = held + 1
+                groups.max_prefix_blocks = max(groups.max_prefix_blocks, held + 1)
+                return tables, groups
+        raise AssertionError("no group with room for a longer prefix")
+
+    err, _ = _run(bm, batch, ctx, 4, 4, 128, "f16", nb, 6, 8, corrupt=corrupt)
     assert err & pa.PA_DEVERR_GROUP
 
 
