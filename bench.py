@@ -230,7 +230,7 @@ def _peaks():
 
 
 DECODE_SOURCES = ("paged_decode_impl.cuh", "decode_policies.cuh", "decode_common.cuh",
-                  "pa_device.cuh")
+                  "decode_merge.cuh", "pa_device.cuh", "pa_internal.h")
 # a cascade figure (":cascade" entries) also depends on the cascade's own kernels
 CASCADE_SOURCES = DECODE_SOURCES + ("cascade.cu",)
 
