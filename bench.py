@@ -231,8 +231,10 @@ def _peaks():
 
 DECODE_SOURCES = ("paged_decode_impl.cuh", "decode_policies.cuh", "decode_common.cuh",
                   "decode_merge.cuh", "pa_device.cuh", "pa_internal.h")
-# a cascade figure (":cascade" entries) also depends on the cascade's own kernels
+# a cascade figure (":cascade" entries) also depends on the cascade's own kernels,
+# an 8-bit figure (":fp8" entries) on the E4M3 policies
 CASCADE_SOURCES = DECODE_SOURCES + ("cascade.cu",)
+FP8_SOURCES = DECODE_SOURCES + ("decode_policy_fp8.cuh",)
 
 
 def decode_source_sha(sources=DECODE_SOURCES) -> str:
@@ -252,6 +254,7 @@ def _traffic_for(workload: str):
         with open(path) as f:
             rec = json.load(f).get(workload)
         sha = decode_source_sha(CASCADE_SOURCES if workload.endswith(":cascade")
+                                else FP8_SOURCES if workload.endswith(":fp8")
                                 else DECODE_SOURCES)
     except (OSError, ValueError, AttributeError):
         return None
@@ -756,9 +759,12 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
         nbytes = (unique_decode_bytes(wl, runner) - non_kv) // 2 + non_kv
         kernel = "pa_paged_decode_cascade over E4M3 caches (distinct blocks)"
     achieved = nbytes / t / 1e9
+    traffic = _traffic_for(wl.name + ":fp8") if runner.groups is None else None
     return {"kernel": kernel, "launch_ms": round(t * 1e3, 4),
             "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": round(achieved, 2),
             "frac_of_hbm_peak": round(achieved / peak, 4),
+            "traffic": traffic,
+            "traffic_over_algorithmic": round(traffic / nbytes, 4) if traffic else None,
             "decode_tokens_per_s": round(wl.num_seqs / t, 1),
             "speedup_vs_16bit_decode": round(dec16_s / t, 3) if dec16_s == dec16_s else None,
             "what": "same batch as the 16-bit decode over E4M3 caches (random valid codes, "

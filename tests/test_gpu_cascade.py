@@ -210,6 +210,27 @@ def test_cascade_rejects_a_prefix_past_the_members_contexts():
     assert err & pa.PA_DEVERR_GROUP
 
 
+@pytest.mark.parametrize("lie", ["empty_leader_slot", "prefix_over_the_bound"])
+def test_cascade_rejects_an_inconsistent_group(lie):
+    """A group whose leader slot is empty, or whose prefix count exceeds the
+    caller's max_prefix_blocks: the prefix CTAs read nothing for it (they check
+    the leader and the count themselves), prepare rejects it, and its members
+    are decoded over their whole contexts, flagged and correct."""
+    nb = 1200
+    bm, batch, ctx = _forest(9, nb)
+
+    def corrupt(tables, groups):
+        k = int(np.argmax(groups.prefix_blocks))
+        if lie == "empty_leader_slot":
+            groups.members[k][0] = -1
+        else:
+            groups.prefix_blocks[k] = groups.max_prefix_blocks + 1
+        return tables, groups
+
+    err, _ = _run(bm, batch, ctx, 4, 4, 128, "f16", nb, 10, 8, corrupt=corrupt)
+    assert err & pa.PA_DEVERR_GROUP
+
+
 def test_cascade_rejects_a_slot_that_does_not_name_back():
     """Two members' slots swapped in seq_member: neither is owned by the group;
     both are decoded over their whole contexts, flagged, and correct."""
