@@ -310,6 +310,166 @@ struct Fp8TensorPolicy {
   }
 };
 
+// Fp8TensorPairPolicy: the tensor-core policy over two blocks per loop step. A
+// stage holds two blocks of the warp's list (each its K and V tiles); the step
+// computes both score tiles (two independent mma chains), updates the running
+// maximum, the rescale vote and the sum once for the 32 tokens, and adds both
+// blocks' P.V. The arithmetic per token is the block step's; only the softmax
+// reference moves once per pair instead of once per block (any reference gives
+// the same softmax once the sums and rows agree with it).
+template <typename T, int D, int G>
+struct Fp8TensorPairPolicy : Fp8TensorPolicy<T, D, G> {
+  using Base = Fp8TensorPolicy<T, D, G>;
+  static constexpr int kTileBytes = Base::kTileBytes;
+  static constexpr int kBlockBytes = Base::kStageBytes;  // one block's K and V tiles
+  static constexpr int kStageBytes = 2 * kBlockBytes;    // a pair of blocks
+  static constexpr bool kPairs = true;
+  // 2 pair stages per warp: 64 KB of ring per 4-warp CTA, three CTAs per SM
+  static constexpr int kMinCtasPerSm = 3;
+
+  // The tile copies of one block into dst (the caller arms the barrier).
+  static __device__ __forceinline__ void issue_block(const DecodeArgs& a, const CUtensorMap* tm_k,
+                                                     const CUtensorMap* tm_v, unsigned char* dst,
+                                                     uint64_t* bar, int phys, int kvh) {
+    if constexpr (Base::kSwizzled) {
+      const int y = (phys * a.num_kv_heads + kvh) * kBS;
+      tma_load_2d(dst, tm_k, 0, y, bar);
+      tma_load_2d(dst + kTileBytes, tm_v, 0, y, bar);
+    } else {
+      const size_t off = ((size_t)phys * a.num_kv_heads + kvh) * kTileBytes;
+      bulk_copy_g2s(dst, static_cast<const unsigned char*>(a.k_cache) + off, kTileBytes, bar);
+      bulk_copy_g2s(dst + kTileBytes, static_cast<const unsigned char*>(a.v_cache) + off,
+                    kTileBytes, bar);
+    }
+  }
+
+  // S = Q K^T of one block (columns: tokens (n >> 1) + 4(n & 1) + 8nt)
+  __device__ __forceinline__ void scores(const unsigned char* Ks, float (&sacc)[2][2]) const {
+    const int krow = (this->g >> 1) + 4 * (this->g & 1);
+    uint4 kw[2][Base::CPT];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int h = 0; h < Base::CPT; ++h)
+        kw[nt][h] = *reinterpret_cast<const uint4*>(
+            Ks + Base::chunk_off(krow + 8 * nt, this->j + 4 * h));
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < Base::KSTEPS; ++kk) {
+      const int h = kk >> 2, w = kk & 3;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const uint32_t word = w == 0 ? kw[nt][h].x : w == 1 ? kw[nt][h].y
+                            : w == 2 ? kw[nt][h].z : kw[nt][h].w;
+        uint32_t b0, b1;
+        e4m3x4_to_half2x2(word, b0, b1);
+        MmaOps<__half>::run(sacc[nt], this->qa[kk][0], this->qa[kk][1], b0, b1);
+      }
+    }
+  }
+
+  // O^T += V^T P^T of one block (as in the block step)
+  __device__ __forceinline__ void values(const unsigned char* Vs, int valid, uint32_t pa0,
+                                         uint32_t pa2) {
+    constexpr int VW = D == 128 ? 4 : 2;
+    uint32_t vr[4][VW];
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      const int t = this->j + 4 * mm;
+      if constexpr (D == 128) {
+        const int c = 4 * (this->g & 1) + (this->g >> 1);
+        const uint4 v = *reinterpret_cast<const uint4*>(Vs + Base::chunk_off(t, c));
+        vr[mm][0] = v.x;
+        vr[mm][1] = v.y;
+        vr[mm][2] = v.z;
+        vr[mm][3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(Vs + t * D + 8 * this->g);
+        vr[mm][0] = v.x;
+        vr[mm][1] = v.y;
+      }
+    }
+    if (valid < kBS) {
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm)
+        if (this->j + 4 * mm >= valid) {
+#pragma unroll
+          for (int w = 0; w < VW; ++w) vr[mm][w] = 0u;
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < Base::MT; ++t) {
+      const int w = t >> 1;
+      const uint32_t sel = (t & 1) ? 0x7362u : 0x5140u;
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_half2x2(__byte_perm(vr[0][w], vr[1][w], sel), a0, a1);
+      e4m3x4_to_half2x2(__byte_perm(vr[2][w], vr[3][w], sel), a2, a3);
+      asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+          "{%8,%9}, {%0,%1,%2,%3};"
+          : "+f"(this->o[t][0]), "+f"(this->o[t][1]), "+f"(this->o[t][2]), "+f"(this->o[t][3])
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(pa0), "r"(pa2));
+    }
+  }
+
+  // Two blocks: stage sa (valid tokens va) and sb (vb; 0 when the pair has one block)
+  __device__ __forceinline__ void block2(const unsigned char* sa, int va, const unsigned char* sb,
+                                         int vb) {
+    float s[2][2][2];  // [block][nt][e]
+    scores(sa, s[0]);
+    scores(sb, s[1]);
+    float bmax = -INFINITY;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int valid = b ? vb : va;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool ok = this->g < G && this->j + 4 * e + 8 * nt < valid;
+          s[b][nt][e] = ok ? s[b][nt][e] * this->row_scale : -INFINITY;
+          bmax = fmaxf(bmax, s[b][nt][e]);
+        }
+    }
+    bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+    bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
+    float alpha;
+    const float mref = lazy_reference(this->m, bmax, alpha);
+    float p[2][2][2];
+    float psum = 0.f;
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[b][nt][e] = exp2f(s[b][nt][e] - mref);
+          psum += p[b][nt][e];
+        }
+    this->l = fmaf(this->l, alpha, psum);
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * this->j);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * this->j + 4);
+#pragma unroll
+      for (int t = 0; t < Base::MT; ++t) {
+        this->o[t][0] *= a0;
+        this->o[t][1] *= a1;
+        this->o[t][2] *= a0;
+        this->o[t][3] *= a1;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      uint32_t pa0, pa2;
+      const __half2 h0 = __floats2half2_rn(p[b][0][0], p[b][0][1]);
+      const __half2 h2 = __floats2half2_rn(p[b][1][0], p[b][1][1]);
+      memcpy(&pa0, &h0, 4);
+      memcpy(&pa2, &h2, 4);
+      values((b ? sb : sa) + kTileBytes, b ? vb : va, pa0, pa2);
+    }
+  }
+};
+
 // ---------------------------------------------------------------------------
 // CUDA cores over an E4M3 cache
 // ---------------------------------------------------------------------------
