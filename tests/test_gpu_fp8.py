@@ -219,3 +219,47 @@ def test_fp8_argument_checks():
             pa.pa_reshape_and_cache_fp8(key, key, kc, kc.clone(), sl, bad, 1.0)
     with pytest.raises(pa.PAError):
         pa.pa_reshape_and_cache(key, key, kc, kc.clone(), sl)   # 16-bit entry, 8-bit cache
+
+
+def test_warp_split_two_block_steps_with_bad_ids():
+    """A batch that takes the warp-per-partition split over 8 query heads per KV
+    head, whose loop takes two blocks per step: contexts of 3841..4096 tokens
+    (16 partitions of 256 tokens, the last ones ragged), one out-of-range block id
+    as the second block of a pair and one as the first. The bad ids are flagged,
+    nothing faults, and every other sequence matches the oracle."""
+    B, hq, hkv, d, dt, pt = 64, 32, 4, 128, "bf16", 256
+    rng = np.random.default_rng(21)
+    ctx = rng.integers(3841, 4097, B).astype(np.int32)
+    _, parts, launches = pa.pa_paged_decode_plan(B, hq, hkv, d, int(ctx.max()), pt)
+    assert parts == 16 and launches == 2, "this batch should take the warp-per-partition split"
+    mb = int(-(-ctx.max() // 16))
+    nb = int(sum(-(-int(c) // 16) for c in ctx))
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((B, mb), -1, np.int32)
+    used = 0
+    for s in range(B):
+        n = -(-int(ctx[s]) // 16)
+        tables[s, :n] = perm[used:used + n]
+        used += n
+    codes = rng.integers(0, 256, (2, nb, hkv, 16, d)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3A
+    q = gen.normal_bits([21, 2], (B, hq, d), dt)
+    bad = tables.copy()
+    bad[5, 3] = nb + 7         # the second block of a pair (blocks 2 and 3)
+    bad[6, 18] = 1 << 30       # the first block of a pair in the second partition
+    ks, vs, scale = 0.04, 0.015, 1 / math.sqrt(d)
+    out = torch.empty(B, hq, d, dtype=TDT[dt], device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = pa.decode_workspace(B, hq, hkv, d, int(ctx.max()), pt)
+    pa.pa_paged_decode_fp8(out, _dev16(q, dt), torch.from_numpy(codes[0]).cuda(),
+                           torch.from_numpy(codes[1]).cuda(), torch.from_numpy(bad).cuda(),
+                           torch.from_numpy(ctx).cuda(), int(ctx.max()), scale, ks, vs,
+                           partition_tokens=pt, workspace=ws, dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pa.PA_DEVERR_BLOCK_RANGE
+    got = out_to_f64(out, dt)
+    check = [0, 1, 4, 7, 63]
+    want = F.paged_decode_fp8(q[check], codes[0], codes[1], tables[check], ctx[check], scale,
+                              ks, vs, dt)
+    for i, s in enumerate(check):
+        assert_close(got[s], want[i], f"seq {s} ctx {ctx[s]}")
