@@ -13,13 +13,17 @@
 // transposing butterfly that halves the live values at each exchange. Tiles
 // arrive raw ([16][d] row-major) by 1-D bulk copies.
 //
-// TensorPolicy (G = 4, 8): warp-level mma.sync m16n8k16, fp32 accumulation,
-// query heads as M (padded to 16), tokens / head_dim as N. The S accumulator
-// is reused in registers as the A operand of P V (FlashAttention-2 layout);
-// P enters P V as a 16-bit value plus its rounding residual, keeping ~16
-// significant bits. Tiles arrive by 2-D TMA tensor loads, 128-byte swizzled:
-// token row t, 128-byte column half h at h*2048 + t*128, 16-byte chunks XOR-ed
-// by t % 8, so ldmatrix fragment loads are bank-conflict free.
+// TensorPolicy (G = 4, 8): warp-level mma.sync m16n8k16, fp32 accumulation.
+// S = Q K^T takes the query heads as M (padded to 16) and the block's tokens as
+// N. P V runs transposed, O^T = V^T P^T: the value tile, loaded transposed by
+// ldmatrix, is the A operand (16 head dimensions by the 16 tokens) and P^T the B
+// operand (N = 8 heads), whose k-slots are exactly the tokens a lane holds in
+// its S accumulator, so the probabilities feed B from registers as they are and
+// no accumulator row is padding (half the mma of P as a padded A operand). P
+// enters as a 16-bit value plus its rounding residual, keeping ~16 significant
+// bits. Tiles arrive by 2-D TMA tensor loads, 128-byte swizzled: token row t,
+// 128-byte column half h at h*2048 + t*128, 16-byte chunks XOR-ed by t % 8, so
+// ldmatrix fragment loads are bank-conflict free.
 #pragma once
 
 #include <cuda.h>
@@ -247,6 +251,23 @@ struct CudaCorePolicy {
 template <typename T>
 struct MmaOps;
 
+// d[0..3] += A B for a whole m16n8k16 tile (A rows 0-15 real), f32 accumulate.
+template <typename T>
+__device__ __forceinline__ void mma_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (std::is_same<T, __half>::value) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+
 template <>
 struct MmaOps<__half> {
   // d[0..1] += A B for rows 0-7 of the m16n8k16 tile. Rows 8-15 of A are zero
@@ -335,12 +356,14 @@ struct TensorPolicy {
   static constexpr bool kFp8Cache = false;
   static constexpr int kMinCtasPerSm = 3;
   static constexpr int KSTEPS = D / 16;
-  static constexpr int NTO = D / 8;  // output n-tiles of 8 columns
+  static constexpr int MT = D / 16;  // m-tiles of O^T = V^T P^T (16 dimensions each)
 
   int r, j, mi, ri;
   uint32_t qa[KSTEPS][2];  // A operand of S = Q K^T: row r, columns kk*16 + 2j (+1) and +8
   float m, l;
-  float o[NTO][2];  // rows r of the output n-tiles (rows r + 8 are padding)
+  // O^T m-tile t: [0] / [1] dimension 16t + r of heads 2j / 2j + 1, [2] / [3]
+  // dimension 16t + r + 8 of the same heads
+  float o[MT][4];
   float scale_log2;
 
   __device__ __forceinline__ void init(int lane) {
@@ -377,7 +400,7 @@ struct TensorPolicy {
     m = -INFINITY;
     l = 0.f;
 #pragma unroll
-    for (int n = 0; n < NTO; ++n) o[n][0] = o[n][1] = 0.f;
+    for (int t = 0; t < MT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
   }
 
   static __device__ __forceinline__ void issue(const DecodeArgs& a, const CUtensorMap* tm_k,
@@ -434,26 +457,32 @@ struct TensorPolicy {
     const float p2 = exp2f(x[1][0] - mref), p3 = exp2f(x[1][1] - mref);
     l = fmaf(l, alpha, (p0 + p1) + (p2 + p3));
     if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      // this lane's outputs are heads 2j and 2j + 1, whose factors live in
+      // lanes 4(2j) and 4(2j + 1)
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * j);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * j + 4);
 #pragma unroll
-      for (int n = 0; n < NTO; ++n) {
-        o[n][0] *= alpha;
-        o[n][1] *= alpha;
+      for (int t = 0; t < MT; ++t) {
+        o[t][0] *= a0;
+        o[t][1] *= a1;
+        o[t][2] *= a0;
+        o[t][3] *= a1;
       }
     }
+    // P^T as the B operand: k-slots 2j, 2j + 1 (and + 8) are this lane's own
+    // tokens of row r, so its probabilities feed B as they are
     uint32_t pa0, pa0_lo, pa2, pa2_lo;
     MmaOps<T>::split(p0, p1, pa0, pa0_lo);
     MmaOps<T>::split(p2, p3, pa2, pa2_lo);
-    // ---- O += P V (V transposed into the B operand by ldmatrix.trans)
+    // ---- O^T += V^T P^T: A = V^T (rows: 16 dimensions, k: the block's tokens),
+    // loaded transposed by ldmatrix from the [token][dim] tile; N = the 8 heads
     const uint32_t vbase = smem_addr(Vs);
 #pragma unroll
-    for (int pp = 0; pp < NTO / 2; ++pp) {
-      const int t = (mi & 1) * 8 + ri;
-      uint32_t v0, v1, v2, v3;
-      ldsm_x4_trans(vbase + swz(t, 2 * pp + (mi >> 1)), v0, v1, v2, v3);
-      MmaOps<T>::run(o[2 * pp], pa0_lo, pa2_lo, v0, v1);
-      MmaOps<T>::run(o[2 * pp + 1], pa0_lo, pa2_lo, v2, v3);
-      MmaOps<T>::run(o[2 * pp], pa0, pa2, v0, v1);
-      MmaOps<T>::run(o[2 * pp + 1], pa0, pa2, v2, v3);
+    for (int t = 0; t < MT; ++t) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(vbase + swz((mi >> 1) * 8 + ri, 2 * t + (mi & 1)), a0, a1, a2, a3);
+      mma_full<T>(o[t], a0, a1, a2, a3, pa0_lo, pa2_lo);
+      mma_full<T>(o[t], a0, a1, a2, a3, pa0, pa2);
     }
   }
 
@@ -462,16 +491,21 @@ struct TensorPolicy {
     // the 4 lanes of a row each hold 4 of every block's 16 columns
     float lsum = l + __shfl_xor_sync(0xffffffffu, l, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-    if (r < G) {
-      if (j == 0) {
-        red_m[warp * G + r] = m;
-        red_l[warp * G + r] = lsum;
-      }
-      float* dst = red_acc + (warp * G + r) * D + 2 * j;
+    if (r < G && j == 0) {
+      red_m[warp * G + r] = m;
+      red_l[warp * G + r] = lsum;
+    }
+    // O^T elements: dimensions 16t + r (+ 8) of heads 2j, 2j + 1
 #pragma unroll
-      for (int n = 0; n < NTO; ++n) {
-        dst[n * 8] = o[n][0];
-        dst[n * 8 + 1] = o[n][1];
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * j + e;
+      if (h < G) {
+        float* dst = red_acc + (warp * G + h) * D + r;
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          dst[16 * t] = o[t][e];
+          dst[16 * t + 8] = o[t][2 + e];
+        }
       }
     }
   }
