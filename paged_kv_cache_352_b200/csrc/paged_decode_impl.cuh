@@ -357,13 +357,21 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint2<P1, P2, WARPS>()))
   }
 }
 
+// Whether a policy computes two blocks per loop step (P::kPairs, P::block2).
+template <class P, class = void>
+struct has_pairs : std::false_type {};
+template <class P>
+struct has_pairs<P, std::void_t<decltype(P::kPairs)>> : std::bool_constant<P::kPairs> {};
+
 // Split-KV with one warp per partition, for short partitions (at most
 // kWarpPartMaxBlocks blocks): warp w of CTA (kvh, y, z) streams partition
 // y * WARPS + w of sequence seq_order[z] through its own ring and leaves that
 // partition's state (m, l, unnormalised rows) in the workspace; no warp waits
 // for another. merge_partitions_kernel then writes every output. Compared with
 // one CTA per partition, each pipeline ramp and state write is amortised over
-// WARPS times more blocks, and no CTA-wide merge runs per partition.
+// WARPS times more blocks, and no CTA-wide merge runs per partition. A policy
+// with kPairs takes two blocks per loop step (one ring stage and one barrier
+// for both, one P::block2 call).
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
     paged_decode_warp_parts_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
@@ -419,48 +427,118 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   __syncwarp();
 
   int win_base = 0;
-  auto issue = [&](int j) {
-    if (j >= win_base + 32) {
-      win_base = j & ~31;
-      win = win_base + lane < my_n ? __ldg(table + b_begin + win_base + lane) : -1;
-    }
-    const int phys = __shfl_sync(0xffffffffu, win, j - win_base);
-    if (lane == 0) {
+  bool aborted;
+  int j = 0;  // loop steps taken (blocks, or pairs of blocks)
+  int issued;
+  if constexpr (!has_pairs<P>::value) {
+    auto issue = [&](int j) {
+      if (j >= win_base + 32) {
+        win_base = j & ~31;
+        win = win_base + lane < my_n ? __ldg(table + b_begin + win_base + lane) : -1;
+      }
+      const int phys = __shfl_sync(0xffffffffu, win, j - win_base);
+      if (lane == 0) {
+        const int st = j % STAGES;
+        uint64_t* bar = &wbars[st];
+        const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
+        wvalid[st] = ok;
+        if (a.stall_first_block && j == 0) {
+          mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
+        } else if (!ok) {
+          report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
+          mbar_arrive(bar);
+        } else {
+          P::issue(a, &tm_k, &tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
+        }
+      }
+    };
+    for (int j = 0; j < STAGES && j < my_n; ++j) issue(j);
+    issued = my_n < STAGES ? my_n : STAGES;
+    pol.begin(a.scale_log2);
+
+    aborted = a.stall_first_block && my_n > 0 &&
+              !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
+    if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+    for (; !aborted && j < my_n; ++j) {
       const int st = j % STAGES;
-      uint64_t* bar = &wbars[st];
-      const bool ok = (unsigned)phys < (unsigned)a.num_blocks;
-      wvalid[st] = ok;
-      if (a.stall_first_block && j == 0) {
-        mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
-      } else if (!ok) {
-        report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
-        mbar_arrive(bar);
-      } else {
-        P::issue(a, &tm_k, &tm_v, wring + (size_t)st * P::kStageBytes, bar, phys, kvh);
+      if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
+        if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+        aborted = true;
+        break;
+      }
+      if (wvalid[st])
+        pol.block(wring + (size_t)st * P::kStageBytes, ctx - (b_begin + j) * kBS, scratch);
+      __syncwarp();
+      if (j + STAGES < my_n) {
+        if (lane == 0) fence_proxy_async_smem();
+        issue(j + STAGES);
+        issued = j + STAGES + 1;
       }
     }
-  };
-  for (int j = 0; j < STAGES && j < my_n; ++j) issue(j);
-  int issued = my_n < STAGES ? my_n : STAGES;
-  pol.begin(a.scale_log2);
+  } else {
+    // Two blocks per step: stage jp % STAGES holds blocks 2jp and 2jp + 1 of this
+    // warp, behind one barrier; wvalid bit 0 / 1 says block 2jp / 2jp + 1 was copied.
+    const int my_pairs = (my_n + 1) / 2;
+    auto issue = [&](int jp) {
+      const int j0 = 2 * jp;
+      if (j0 >= win_base + 32) {
+        win_base = j0 & ~31;
+        win = win_base + lane < my_n ? __ldg(table + b_begin + win_base + lane) : -1;
+      }
+      // j0 - win_base is even and below 32, so both entries are in the window
+      const int phys0 = __shfl_sync(0xffffffffu, win, j0 - win_base);
+      const int phys1 = __shfl_sync(0xffffffffu, win, j0 + 1 - win_base);
+      if (lane == 0) {
+        const int st = jp % STAGES;
+        uint64_t* bar = &wbars[st];
+        unsigned char* dst = wring + (size_t)st * P::kStageBytes;
+        const bool has1 = j0 + 1 < my_n;
+        const bool ok0 = (unsigned)phys0 < (unsigned)a.num_blocks;
+        const bool ok1 = has1 && (unsigned)phys1 < (unsigned)a.num_blocks;
+        wvalid[st] = (ok0 ? 1 : 0) | (ok1 ? 2 : 0);
+        if (!ok0 || (has1 && !ok1)) report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
+        if (a.stall_first_block && jp == 0) {
+          mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
+        } else if (!ok0 && !ok1) {
+          mbar_arrive(bar);  // complete the phase without data; the pair is skipped
+        } else {
+          mbar_arrive_expect_tx(bar, (ok0 ? P::kBlockBytes : 0) + (ok1 ? P::kBlockBytes : 0));
+          if (ok0) P::issue_block(a, &tm_k, &tm_v, dst, bar, phys0, kvh);
+          if (ok1) P::issue_block(a, &tm_k, &tm_v, dst + P::kBlockBytes, bar, phys1, kvh);
+        }
+      }
+    };
+    for (int jp = 0; jp < STAGES && jp < my_pairs; ++jp) issue(jp);
+    issued = my_pairs < STAGES ? my_pairs : STAGES;
+    pol.begin(a.scale_log2);
 
-  bool aborted = a.stall_first_block && my_n > 0 &&
-                 !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
-  if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
-  int j = 0;
-  for (; !aborted && j < my_n; ++j) {
-    const int st = j % STAGES;
-    if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
-      if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
-      aborted = true;
-      break;
-    }
-    if (wvalid[st]) pol.block(wring + (size_t)st * P::kStageBytes, ctx - (b_begin + j) * kBS, scratch);
-    __syncwarp();
-    if (j + STAGES < my_n) {
-      if (lane == 0) fence_proxy_async_smem();
-      issue(j + STAGES);
-      issued = j + STAGES + 1;
+    aborted = a.stall_first_block && my_pairs > 0 &&
+              !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
+    if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+    for (; !aborted && j < my_pairs; ++j) {
+      const int st = j % STAGES;
+      if (!mbar_wait_bounded(&wbars[st], (uint32_t)((j / STAGES) & 1))) {
+        if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
+        aborted = true;
+        break;
+      }
+      const int v = wvalid[st];
+      if (v) {
+        unsigned char* sa = wring + (size_t)st * P::kStageBytes;
+        const int b0 = b_begin + 2 * j;
+        // a block that was not copied enters with no valid tokens (masked, its
+        // value rows cleared) and the other block's tiles as a readable stand-in
+        const int va = (v & 1) ? ctx - b0 * kBS : 0;
+        const int vb = (v & 2) ? ctx - (b0 + 1) * kBS : 0;
+        pol.block2((v & 1) ? sa : sa + P::kBlockBytes, va, (v & 2) ? sa + P::kBlockBytes : sa,
+                   vb);
+      }
+      __syncwarp();
+      if (j + STAGES < my_pairs) {
+        if (lane == 0) fence_proxy_async_smem();
+        issue(j + STAGES);
+        issued = j + STAGES + 1;
+      }
     }
   }
   if (aborted) {
@@ -471,159 +549,6 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
   // The CTA's WARPS consecutive partitions merge on chip (through shared memory,
   // reusing the tile ring) into one state row, row blockIdx.y of the sequence's
   // rows: the merge kernel then reads WARPS times fewer states.
-  __syncthreads();
-  float* red_m = reinterpret_cast<float*>(smem);  // [WARPS][G]
-  float* red_l = red_m + WARPS * G;                // [WARPS][G]
-  float* red_acc = red_l + WARPS * G;              // [WARPS][G][D]
-  pol.to_red(red_m, red_l, red_acc, warp, lane);
-  __syncthreads();
-  const size_t row0 = (((size_t)s * a.num_kv_heads + kvh) * a.max_parts + blockIdx.y) * G;
-  for (int item = threadIdx.x; item < G * D; item += blockDim.x) {
-    const int g = item / D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_m[w * G + g]);
-    const float Mref = M == -INFINITY ? 0.f : M;
-    float L = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) {
-      const float sc = exp2f(red_m[w * G + g] - Mref);
-      L = fmaf(sc, red_l[w * G + g], L);
-      A = fmaf(sc, red_acc[(w * G) * D + item], A);
-    }
-    a.ws_acc[(row0 + g) * D + (item % D)] = A;
-    if (item % D == 0) {
-      a.ws_m[row0 + g] = M;
-      a.ws_l[row0 + g] = L;
-    }
-  }
-}
-
-// The warp-per-partition split with a pair policy (P::kPairs): as
-// paged_decode_warp_parts_kernel, but each ring stage holds two consecutive blocks
-// of the warp's partition, copied behind one barrier and computed by one
-// P::block2 step.
-template <class P, typename T, int D, int G, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
-    paged_decode_warp_parts_pair_kernel(const DecodeArgs a,
-                                        const __grid_constant__ CUtensorMap tm_k,
-                                        const __grid_constant__ CUtensorMap tm_v) {
-  grid_dependency_wait();
-  allow_dependents();
-  constexpr size_t kRing = size_t(WARPS) * STAGES * P::kStageBytes;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + P::kAlign - 1) & ~(uintptr_t)(P::kAlign - 1));
-  const int kvh = blockIdx.x;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int part = blockIdx.y * WARPS + warp;
-  const int s = a.seq_order ? __ldg(a.seq_order + blockIdx.z) : (int)blockIdx.z;
-  if ((unsigned)s >= (unsigned)a.num_seqs) {
-    if (blockIdx.y == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
-    return;
-  }
-  const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
-  const int b_begin = part * a.part_blocks;
-  int ctx = __ldg(a.context_lens + s);
-  int win = -1;  // lane i holds the table entry of the warp's block win_base + i
-  {
-    const int idx = b_begin + lane;
-    if (lane < a.part_blocks && idx < a.max_blocks_per_seq) win = __ldg(table + idx);
-  }
-  P pol;
-  pol.init(lane);
-  pol.prefetch_q(a, s, kvh);
-  if (ctx < 0 || ctx > a.max_blocks_per_seq * kBS || ctx > a.max_context_len) {
-    if (part == 0 && kvh == 0 && lane == 0) report(a.dev_error, PA_DEVERR_CONTEXT_RANGE);
-    ctx = 0;
-  }
-  const int nblk = (ctx + kBS - 1) / kBS;
-  const int nparts = (nblk + a.part_blocks - 1) / a.part_blocks;
-  if ((int)blockIdx.y * WARPS >= nparts) return;  // the whole CTA
-  const int my_n = part < nparts ? min(nblk, b_begin + a.part_blocks) - b_begin : 0;
-  const int my_pairs = (my_n + 1) / 2;
-
-  unsigned char* wring = smem + (size_t)warp * STAGES * P::kStageBytes;
-  uint64_t* wbars = reinterpret_cast<uint64_t*>(smem + kRing) + warp * STAGES;
-  int* wvalid = reinterpret_cast<int*>(smem + kRing + WARPS * STAGES * sizeof(uint64_t)) +
-                warp * STAGES;
-  if (lane == 0) {
-#pragma unroll
-    for (int st = 0; st < STAGES; ++st) mbar_init(&wbars[st], 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
-
-  // Start the copies of pair jp (blocks 2jp and 2jp + 1 of this warp) into stage
-  // jp % STAGES. wvalid bit 0 / 1: block 2jp / 2jp + 1 was copied.
-  int win_base = 0;
-  auto issue = [&](int jp) {
-    const int j0 = 2 * jp;
-    if (j0 >= win_base + 32) {
-      win_base = j0 & ~31;
-      win = win_base + lane < my_n ? __ldg(table + b_begin + win_base + lane) : -1;
-    }
-    // j0 - win_base is even and below 32, so both entries are in the window
-    const int phys0 = __shfl_sync(0xffffffffu, win, j0 - win_base);
-    const int phys1 = __shfl_sync(0xffffffffu, win, j0 + 1 - win_base);
-    if (lane == 0) {
-      const int st = jp % STAGES;
-      uint64_t* bar = &wbars[st];
-      unsigned char* dst = wring + (size_t)st * P::kStageBytes;
-      const bool has1 = j0 + 1 < my_n;
-      const bool ok0 = (unsigned)phys0 < (unsigned)a.num_blocks;
-      const bool ok1 = has1 && (unsigned)phys1 < (unsigned)a.num_blocks;
-      wvalid[st] = (ok0 ? 1 : 0) | (ok1 ? 2 : 0);
-      if (!ok0 || (has1 && !ok1)) report(a.dev_error, PA_DEVERR_BLOCK_RANGE);
-      if (a.stall_first_block && jp == 0) {
-        mbar_arrive_expect_tx(bar, 16);  // test hook: bytes that no copy will bring
-      } else if (!ok0 && !ok1) {
-        mbar_arrive(bar);  // complete the phase without data; the pair is skipped
-      } else {
-        mbar_arrive_expect_tx(bar, (ok0 ? P::kBlockBytes : 0) + (ok1 ? P::kBlockBytes : 0));
-        if (ok0) P::issue_block(a, &tm_k, &tm_v, dst, bar, phys0, kvh);
-        if (ok1) P::issue_block(a, &tm_k, &tm_v, dst + P::kBlockBytes, bar, phys1, kvh);
-      }
-    }
-  };
-  for (int jp = 0; jp < STAGES && jp < my_pairs; ++jp) issue(jp);
-  int issued = my_pairs < STAGES ? my_pairs : STAGES;
-  pol.begin(a.scale_log2);
-
-  bool aborted = a.stall_first_block && my_pairs > 0 &&
-                 !mbar_wait_bounded(&wbars[0], 0u, a.wait_limit_ns);
-  if (aborted && lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
-  int jp = 0;
-  for (; !aborted && jp < my_pairs; ++jp) {
-    const int st = jp % STAGES;
-    if (!mbar_wait_bounded(&wbars[st], (uint32_t)((jp / STAGES) & 1))) {
-      if (lane == 0) report(a.dev_error, PA_DEVERR_WAIT_TIMEOUT);
-      aborted = true;
-      break;
-    }
-    const int v = wvalid[st];
-    if (v) {
-      unsigned char* sa = wring + (size_t)st * P::kStageBytes;
-      const int b0 = b_begin + 2 * jp;
-      // a block that was not copied enters with no valid tokens (masked, its
-      // value rows cleared) and the other block's tiles as a readable stand-in
-      const int va = (v & 1) ? ctx - b0 * kBS : 0;
-      const int vb = (v & 2) ? ctx - (b0 + 1) * kBS : 0;
-      pol.block2((v & 1) ? sa : sa + P::kBlockBytes, va, (v & 2) ? sa + P::kBlockBytes : sa, vb);
-    }
-    __syncwarp();
-    if (jp + STAGES < my_pairs) {
-      if (lane == 0) fence_proxy_async_smem();
-      issue(jp + STAGES);
-      issued = jp + STAGES + 1;
-    }
-  }
-  if (aborted) {
-    for (int k = jp; k < issued; ++k)
-      if (!(a.stall_first_block && k == 0))
-        mbar_wait_bounded(&wbars[k % STAGES], (uint32_t)((k / STAGES) & 1));
-  }
   __syncthreads();
   float* red_m = reinterpret_cast<float*>(smem);  // [WARPS][G]
   float* red_l = red_m + WARPS * G;                // [WARPS][G]
@@ -769,12 +694,12 @@ cudaError_t launch_kernel(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   return launch_dependent(kern, grid, dim3(WARPS * 32), smem, stream, a, tk, tv);
 }
 
-// The warp-per-partition split with a pair policy, then the merge launch.
+// The warp-per-partition split with a two-block policy, then the merge launch.
 template <class P, typename T, int D, int G, int WARPS, int STAGES>
 cudaError_t launch_pair_parts(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   const size_t smem = smem_bytes<P, WARPS, STAGES, G, D>(a.max_parts);
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
-  auto kern = paged_decode_warp_parts_pair_kernel<P, T, D, G, WARPS, STAGES>;
+  auto kern = paged_decode_warp_parts_kernel<P, T, D, G, WARPS, STAGES>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
