@@ -168,6 +168,16 @@ def test_cascade_prefix_is_the_whole_context(hq, hkv, d, dt, gs):
                for i in np.nonzero(grouped)[0])
 
 
+@pytest.mark.parametrize("hq,hkv,d,dt,gs", [(4, 4, 128, "f16", 8), (8, 4, 128, "bf16", 4)])
+def test_cascade_fp8_prefix_is_the_whole_context(hq, hkv, d, dt, gs):
+    """Over 8-bit caches: forked whole-block prompts without appends, so every
+    member's own-block decode is empty and its output is the prefix alone."""
+    nb = 800
+    bm, batch, ctx = _forest(78, nb, exact=True)
+    err, groups = _run(bm, batch, ctx, hq, hkv, d, dt, nb, 6, gs, fp8=(0.05, 0.02))
+    assert err == 0 and groups.num_groups >= 1
+
+
 def test_cascade_rejects_a_member_without_the_prefix():
     """One member's first prefix block is pointed elsewhere: the group is decoded
     without its prefix (flagged), and every output still matches the oracle over
