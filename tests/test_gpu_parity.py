@@ -4,7 +4,8 @@ Small versions of every workload are compared in full: block tables, slot
 mappings and copy pairs bit for bit, the whole key and value pools bit for bit
 (untouched slots included), and every attention output within tolerance.
 Full-size workloads run in the launch configuration the benchmark times and
-are checked on sampled outputs and sampled cache slots.
+are checked on sampled outputs and sampled cache slots, over 16-bit caches and
+(GQA and long contexts) over E4M3 caches.
 """
 
 import math
@@ -404,3 +405,49 @@ def test_planted_key(name):
         _sync()
         assert_close(out_to_f64(out, wl.dtype), ref, f"{name} planted key, partition {pt}")
     assert r.error_bits() == 0
+
+
+@pytest.mark.parametrize("name", ["gqa_32_8_bf16", "long_ctx_split_kv"])
+def test_full_size_fp8_sampled_parity(name):
+    """The same batches over E4M3 caches of random valid codes, in the launch
+    configuration the benchmark's 8-bit figure times (the runner's tables,
+    lengths, order and partitions: CTA mode for GQA, the warp-per-partition split
+    with two blocks per loop step for long contexts), checked on sampled rows
+    against the oracle's attention over the dequantized codes."""
+    from oracle import fp8 as F
+    from oracle.attention import softmax_attention
+    from oracle.fpbits import bits_to_f64
+    wl = workloads.workload(name)
+    r = DecodeRunner(wl)
+    g = torch.Generator(device="cuda").manual_seed(353)
+    shape = tuple(r.k_cache.shape)
+
+    def codes():
+        c = torch.randint(0, 0x7E, shape, generator=g, device="cuda", dtype=torch.uint8)
+        return c | (torch.randint(0, 2, shape, generator=g, device="cuda",
+                                  dtype=torch.uint8) << 7)
+    kc, vc = codes(), codes()
+    del r.k_cache, r.v_cache
+    torch.cuda.empty_cache()
+    ks, vs = 0.05, 0.02
+    out = torch.empty_like(r.q)
+    pa.pa_paged_decode_fp8(out, r.q, kc, vc, r.block_tables, r.context_lens,
+                           wl.max_context_len, wl.scale, ks, vs,
+                           partition_tokens=r.partition_tokens or 0, workspace=r.workspace,
+                           dev_error=r.dev_error, seq_order=r.seq_order)
+    _sync()
+    assert r.error_bits() == 0
+    got = out_to_f64(out, wl.dtype)
+    rows = _sample_rows(wl, np.random.default_rng(353))
+    G = wl.num_q_heads // wl.num_kv_heads
+    ref = np.zeros((len(rows), wl.head_dim))
+    for i, (s, h) in enumerate(rows):
+        ctx = int(wl.context_lens[s])
+        n = -(-ctx // 16)
+        blocks = torch.from_numpy(r.block_tables_host[s, :n].astype(np.int64)).cuda()
+        kvh = h // G
+        kb = kc[blocks, kvh].reshape(n * 16, -1)[:ctx].cpu().numpy()
+        vb = vc[blocks, kvh].reshape(n * 16, -1)[:ctx].cpu().numpy()
+        ref[i] = softmax_attention(bits_to_f64(r.q_host[s, h], wl.dtype), F.dequantize(kb, ks),
+                                   F.dequantize(vb, vs), wl.scale)
+    assert_close(np.stack([got[s, h] for s, h in rows]), ref, f"{name} over E4M3 caches")
