@@ -232,9 +232,11 @@ def _peaks():
 DECODE_SOURCES = ("paged_decode_impl.cuh", "decode_policies.cuh", "decode_common.cuh",
                   "decode_merge.cuh", "pa_device.cuh", "pa_internal.h")
 # a cascade figure (":cascade" entries) also depends on the cascade's own kernels,
-# an 8-bit figure (":fp8" entries) on the E4M3 policies
+# an 8-bit figure (":fp8" entries) on the E4M3 policies, an 8-bit cascade figure
+# (":cascade:fp8") on both
 CASCADE_SOURCES = DECODE_SOURCES + ("cascade.cu",)
 FP8_SOURCES = DECODE_SOURCES + ("decode_policy_fp8.cuh",)
+CASCADE_FP8_SOURCES = CASCADE_SOURCES + ("decode_policy_fp8.cuh",)
 
 
 def decode_source_sha(sources=DECODE_SOURCES) -> str:
@@ -254,6 +256,7 @@ def _traffic_for(workload: str):
         with open(path) as f:
             rec = json.load(f).get(workload)
         sha = decode_source_sha(CASCADE_SOURCES if workload.endswith(":cascade")
+                                else CASCADE_FP8_SOURCES if workload.endswith(":cascade:fp8")
                                 else FP8_SOURCES if workload.endswith(":fp8")
                                 else DECODE_SOURCES)
     except (OSError, ValueError, AttributeError):
@@ -759,7 +762,7 @@ def measure_fp8_decode(wl, runner, device, l2_flush, dec16_s, peak, iters: int =
         nbytes = (unique_decode_bytes(wl, runner) - non_kv) // 2 + non_kv
         kernel = "pa_paged_decode_cascade over E4M3 caches (distinct blocks)"
     achieved = nbytes / t / 1e9
-    traffic = _traffic_for(wl.name + ":fp8") if runner.groups is None else None
+    traffic = _traffic_for(wl.name + (":fp8" if runner.groups is None else ":cascade:fp8"))
     return {"kernel": kernel, "launch_ms": round(t * 1e3, 4),
             "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": round(achieved, 2),
             "frac_of_hbm_peak": round(achieved / peak, 4),
