@@ -1,10 +1,11 @@
-"""Seeded random shapes through pa_paged_decode and pa_paged_decode_fp8 on a B200
-against the oracle: every head layout (1..8 query heads per KV head), both head
-dimensions and query types, 16-bit and E4M3 caches, ragged contexts with the
-edge lengths (0, 1, 15, 16, 17) mixed in, caller-chosen and library partitions,
-with and without a scheduling order, NaN patterns in the slots past each
-context. Each case is generated from its own seed, so a failure names a
-reproducible shape."""
+"""Seeded random shapes through pa_paged_decode, pa_paged_decode_fp8 and
+pa_paged_decode_cascade on a B200 against the oracle: every head layout (1..8
+query heads per KV head), both head dimensions and query types, 16-bit and E4M3
+caches, ragged contexts with the edge lengths (0, 1, 15, 16, 17) mixed in,
+caller-chosen and library partitions, with and without a scheduling order, NaN
+patterns in the slots past each context; for the cascade, random fork forests
+under every supported (group size, query heads per KV head) pair. Each case is
+generated from its own seed, so a failure names a reproducible shape."""
 
 import math
 
@@ -16,6 +17,7 @@ import paged_kv_cache_352_b200 as pa
 from oracle import fp8 as F
 from oracle.attention import paged_decode
 from tests.parity import assert_close, out_to_f64
+from tests.test_gpu_cascade import _forest, _run
 from workloads import gen
 
 pytestmark = pytest.mark.gpu
@@ -153,3 +155,32 @@ def test_random_warp_split_batch_matches_oracle(seed):
     got = out_to_f64(out, dt)
     for i, s in enumerate(check):
         assert_close(got[s], want[i], f"{what} seq {s} ctx {ctx[s]}")
+
+
+# (query heads per KV head, group size): every pair whose stacked rows (their
+# product) are 1, 2, 4 or 8; 8 runs both decodes in one launch
+CASCADE_LAYOUTS = [(1, 1), (1, 2), (1, 4), (1, 8), (2, 1), (2, 2), (2, 4), (4, 1), (4, 2),
+                   (8, 1)]
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_cascade_matches_oracle(seed):
+    """Random fork forests (prompts forked into samples that append their own
+    tokens, or prompts of whole blocks with no own tokens, plus an empty
+    sequence) through the cascade: every output row within tolerance of the
+    oracle's decode over the whole context, and no device error."""
+    rng = np.random.default_rng([355, seed])
+    G, gs = CASCADE_LAYOUTS[seed % len(CASCADE_LAYOUTS)]
+    hkv = int(rng.choice([1, 2, 4, 8]))
+    d = int(rng.choice([64, 128]))
+    dt = str(rng.choice(["f16", "bf16"]))
+    exact = bool(rng.integers(0, 4) == 0)
+    order = [None, "cascade", "random"][int(rng.integers(0, 3))]
+    fp8 = None
+    if rng.integers(0, 2):
+        fp8 = (float(rng.uniform(0.02, 0.08)), float(rng.uniform(0.004, 0.013)))
+    nb = 1200
+    bm, batch, ctx = _forest(int(rng.integers(1 << 30)), nb, exact=exact)
+    err, groups = _run(bm, batch, ctx, hkv * G, hkv, d, dt, nb, seed, gs, fp8=fp8, order=order)
+    assert err == 0, (f"seed {seed}: G{G} group size {gs} hkv{hkv} d{d} {dt} order {order} "
+                      f"fp8 {fp8}: device error {err}")
