@@ -729,11 +729,13 @@ cudaError_t launch_pair_parts(const DecodeArgs& a, int dtype, cudaStream_t strea
                           stream, a);
 }
 
-// The cascade's two decodes as one launch of cascade_decode_kernel (4 x 2 tiles).
+// The cascade's two decodes as one launch of cascade_decode_kernel: 4 x 2
+// tiles, 4 x 3 over E4M3 caches (a stage holds half the bytes; 62.5 -> 62.2 us
+// on the shared-prefix batch, 4 x 4 slower at 68.3 us).
 template <class P1, int G1, class P2, int G2, typename T, int D>
 cudaError_t launch_dual(const DecodeArgs& a1, const DecodeArgs& a2, int dtype,
                         cudaStream_t stream) {
-  constexpr int WARPS = 4, STAGES = 2;
+  constexpr int WARPS = 4, STAGES = P1::kFp8Cache ? 3 : 2;
   const size_t s1 = smem_bytes<P1, WARPS, STAGES, G1, D>(a1.max_parts);
   const size_t s2 = smem_bytes<P2, WARPS, STAGES, G2, D>(a2.max_parts);
   const size_t smem = s1 > s2 ? s1 : s2;
@@ -776,10 +778,12 @@ cudaError_t launch_dual(const DecodeArgs& a1, const DecodeArgs& a2, int dtype,
                           tk, tv);
 }
 
-// Warps per CTA x stages per warp. 4 x 2 (64 KiB of K/V in flight per CTA at
-// head_dim 128, three CTAs per SM) measured best or within 2% of best on every
-// workload; PA_DECODE_TILE="WxS" selects another built shape for A/B
-// measurements (4x3, 8x2, 2x3).
+// Warps per CTA x stages per warp. Over 16-bit caches 4 x 2 (64 KiB of K/V in
+// flight per CTA at head_dim 128, three CTAs per SM) measured best or within 2%
+// of best on every workload. Over E4M3 caches a stage holds half the bytes and
+// 4 x 3 measured faster than 4 x 2 (7B-like MHA 99.1 -> 97.7 us, GQA 32/8 85.2 ->
+// 84.9 us per launch; 8 x 2 and 2 x 3 slower). PA_DECODE_TILE="WxS" selects
+// another built shape for A/B measurements (4x2, 4x3, 8x2, 2x3).
 int tile_variant() {
   static const int v = [] {
     const char* e = getenv("PA_DECODE_TILE");
@@ -787,6 +791,7 @@ int tile_variant() {
     if (!strcmp(e, "4x3")) return 1;
     if (!strcmp(e, "8x2")) return 2;
     if (!strcmp(e, "2x3")) return 3;
+    if (!strcmp(e, "4x2")) return 4;
     return 0;
   }();
   return v;
@@ -798,7 +803,10 @@ cudaError_t launch_tiles(const DecodeArgs& a, int dtype, cudaStream_t stream) {
     case 1: return launch_kernel<P, T, D, G, 4, 3>(a, dtype, stream);
     case 2: return launch_kernel<P, T, D, G, 8, 2>(a, dtype, stream);
     case 3: return launch_kernel<P, T, D, G, 2, 3>(a, dtype, stream);
-    default: return launch_kernel<P, T, D, G, 4, 2>(a, dtype, stream);
+    case 4: return launch_kernel<P, T, D, G, 4, 2>(a, dtype, stream);
+    default:
+      if constexpr (P::kFp8Cache) return launch_kernel<P, T, D, G, 4, 3>(a, dtype, stream);
+      else return launch_kernel<P, T, D, G, 4, 2>(a, dtype, stream);
   }
 }
 
