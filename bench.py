@@ -231,10 +231,10 @@ def _peaks():
 
 DECODE_SOURCES = ("paged_decode_impl.cuh", "decode_policies.cuh", "decode_common.cuh",
                   "decode_merge.cuh", "pa_device.cuh", "pa_internal.h")
-# a cascade figure (":cascade" entries) also depends on the cascade's own kernels,
-# an 8-bit figure (":fp8" entries) on the E4M3 policies, an 8-bit cascade figure
-# (":cascade:fp8") on both
-CASCADE_SOURCES = DECODE_SOURCES + ("cascade.cu",)
+# a cascade figure (":cascade" entries) also depends on the cascade's own kernels
+# and its partition layout, an 8-bit figure (":fp8" entries) on the E4M3
+# policies, an 8-bit cascade figure (":cascade:fp8") on both
+CASCADE_SOURCES = DECODE_SOURCES + ("cascade.cu", "pa_api.cu")
 FP8_SOURCES = DECODE_SOURCES + ("decode_policy_fp8.cuh",)
 CASCADE_FP8_SOURCES = CASCADE_SOURCES + ("decode_policy_fp8.cuh",)
 

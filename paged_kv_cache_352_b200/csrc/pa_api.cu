@@ -486,7 +486,14 @@ int cascade_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim
                 max_prefix_blocks, max_blocks_per_seq);
   const int ng = num_groups > 0 ? num_groups : 0;
   const int pmax = num_groups > 0 ? max_prefix_blocks : 1;
-  L->g_part_blocks = default_partition_blocks(ng > 0 ? ng : 1, num_kv_heads, pmax, false);
+  // The own-block CTAs run beside the prefix CTAs (in the same launch, or on a
+  // second stream), so they count toward filling the GPU: a prefix is split
+  // below the cap only when groups and sequences together give fewer than
+  // kSplitTargetUnits (group or sequence, KV head) pairs. On 16 groups of 8
+  // samples with 62-block prefixes and 32 KV heads, one partition per prefix
+  // measured faster than two: 62.3 -> 58.0 us over 8-bit caches, 88.9 -> 88.5 us
+  // over 16-bit ones (16- or 21-block partitions: slower still).
+  L->g_part_blocks = default_partition_blocks(ng + num_seqs, num_kv_heads, pmax, false);
   L->g_parts = (pmax + L->g_part_blocks - 1) / L->g_part_blocks;
   const int own_blocks = std::max(1, (max_context_len + kBlockSize - 1) / kBlockSize);
   L->s_part_blocks = default_partition_blocks(num_seqs > 0 ? num_seqs : 1, num_kv_heads,
