@@ -189,8 +189,6 @@ __global__ void __launch_bounds__(kPrepThreads) cascade_prepare_kernel(const Cas
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) cascade_merge_kernel(const CascadeArgs c,
                                                                          int gh) {
-  grid_dependency_wait();  // the partition states come from the decodes
-  allow_dependents();
   constexpr int kSet = 4;
   const int row = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -199,10 +197,19 @@ __global__ void __launch_bounds__(kMergeWarps * 32) cascade_merge_kernel(const C
   const int h = row - s * c.num_q_heads;
   const int kvh = h / gh, hh = h - kvh * gh;
   const int gg = c.group_size * gh;
-  // three independent loads in one round (prepare writes all three for every sequence)
+  // Prepare's rows for this sequence (three independent loads in one round),
+  // read before the wait for the decodes. This kernel starts only once every CTA
+  // of the decode launch ahead of it has let it start (or exited), and every
+  // own-block CTA does so only after its own wait, which returns once prepare
+  // has completed and its writes are performed; loads through L2 then see them.
+  // (With the decodes on two streams, the launch ahead is the own-block decode,
+  // whose CTAs likewise wait first.) Measured on the shared-prefix batch: 88.3 ->
+  // 87.0 us per call (8-bit 57.9 -> 57.4 us).
   const int pb = __ldcg(c.s_pbase + s);
   const int np_raw = __ldcg(c.s_np + s);
   const int own_ctx = __ldcg(c.s_ctx + s);
+  grid_dependency_wait();  // the partition states come from the decodes
+  allow_dependents();
   const int np = pb < 0 ? 0 : np_raw;
   const int ob = (own_ctx + kBlockSize - 1) / kBlockSize;
   const int no = (ob + c.s_part_blocks - 1) / c.s_part_blocks;
