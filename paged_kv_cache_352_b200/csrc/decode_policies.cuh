@@ -275,10 +275,10 @@ struct MmaOps<__half> {
   // zeros and their results discarded instead of occupying registers.
   static __device__ __forceinline__ void run(float (&d)[2], uint32_t a0, uint32_t a2,
                                              uint32_t b0, uint32_t b1) {
-    float dead0, dead1;
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%11,%12,%12};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(dead0), "=f"(dead1)
+    asm("{\n\t.reg .f32 dead0, dead1;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,dead0,dead1}, {%2,%3,%4,%5}, "
+        "{%6,%7}, {%8,%9,%10,%10};\n\t}"
+        : "=f"(d[0]), "=f"(d[1])
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
   }
   // (x0, x1) as a packed 16-bit pair `hi` plus the packed rounding residual `lo`
@@ -298,10 +298,10 @@ struct MmaOps<__nv_bfloat16> {
   // zeros and their results discarded instead of occupying registers.
   static __device__ __forceinline__ void run(float (&d)[2], uint32_t a0, uint32_t a2,
                                              uint32_t b0, uint32_t b1) {
-    float dead0, dead1;
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%11,%12,%12};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(dead0), "=f"(dead1)
+    asm("{\n\t.reg .f32 dead0, dead1;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,dead0,dead1}, {%2,%3,%4,%5}, "
+        "{%6,%7}, {%8,%9,%10,%10};\n\t}"
+        : "=f"(d[0]), "=f"(d[1])
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(0.f));
   }
   static __device__ __forceinline__ void split(float x0, float x1, uint32_t& hi, uint32_t& lo) {

@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(WARPS * 32, (min_ctas_hint<P, WARPS>()))
         }
       }
     };
-    for (int j = 0; j < STAGES && j < my_n; ++j) issue(j);
+    for (int k = 0; k < STAGES && k < my_n; ++k) issue(k);
     issued = my_n < STAGES ? my_n : STAGES;
     pol.begin(a.scale_log2);
 
