@@ -957,6 +957,7 @@ def measure_config(name: str, args, device, peak: float, peak_kind: str, read_re
     with the headline's protocol) and its decode against the roofline. For the
     per-workload object of the bench line; everything it allocates is released."""
     import torch
+    from paged_kv_cache_352_b200 import _lib as L
     from paged_kv_cache_352_b200.runner import DecodeRunner
     import workloads
     wl = workloads.workload(name)
@@ -993,6 +994,10 @@ def measure_config(name: str, args, device, peak: float, peak_kind: str, read_re
         res["note"] = ("0.11 MB per launch: one launch latency, so the 70 % bandwidth target "
                        "cannot apply")
     if r.groups is not None:
+        res["cascade_plan"] = L.pa_paged_decode_cascade_plan(
+            wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.max_context_len,
+            r.max_blocks, r.groups.num_groups, r.groups.group_size, r.groups.max_prefix_blocks,
+            dtype=wl.dtype)
         res["logical_decode_gbs"] = round(decode_bytes(wl) / dec_s / 1e9, 2)
         res["plain_decode"] = time_plain_decode(r, device, l2_flush, dec_s)
         res["copy_blocks"] = time_copy_blocks(r, wl, device)

@@ -281,6 +281,25 @@ int pa_paged_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
  * by index), the recommended seq_order. Both arrays are host memory. */
 int pa_longest_first_order(const int32_t* context_lens, int n, int32_t* order);
 
+/* The plan pa_paged_decode_cascade (fp8_cache == 0) or pa_paged_decode_cascade_fp8
+ * (fp8_cache != 0) would follow for these host bounds, which are those of
+ * pa_paged_decode_cascade_workspace_size; dtype is the query type (PA_F16 or
+ * PA_BF16). Outputs: blocks per partition and partitions of a group's shared
+ * prefix (0 and 0 when num_groups is 0), blocks per partition and partitions
+ * of a sequence's own blocks, and the kernel launches the call makes: 3
+ * (prepare, both decodes in one launch, merge; also with no groups), 4 when the
+ * two decodes run on two streams (fewer than 8 stacked query heads per KV
+ * head), 0 for an empty batch. Prefixes are split below the decode's
+ * partition cap only when groups and sequences together give fewer than about
+ * 1024 (group or sequence, KV head) pairs. Host only; nothing is launched.
+ * Returns PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED for the shapes the cascade
+ * refuses. */
+int pa_paged_decode_cascade_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int max_context_len, int max_blocks_per_seq, int block_size,
+                                 int num_groups, int group_size, int max_prefix_blocks, int dtype,
+                                 int fp8_cache, int* prefix_part_blocks, int* prefix_parts,
+                                 int* own_part_blocks, int* own_parts, int* launches);
+
 /* Host helper for pa_paged_decode_cascade: order[0..n) = sequence indices by
  * decreasing tokens after their group's prefix (context_lens[i] -
  * block_size * group_prefix_blocks[seq_group[i]] for a sequence in a group,

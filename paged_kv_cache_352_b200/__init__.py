@@ -38,6 +38,7 @@ from ._lib import (  # noqa: F401
     pa_paged_decode_fp8,
     pa_paged_decode_noalloc,
     pa_paged_decode_plan,
+    pa_paged_decode_cascade_plan,
     pa_paged_decode_workspace_size,
     pa_reshape_and_cache,
     pa_reshape_and_cache_fp8,

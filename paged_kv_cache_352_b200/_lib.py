@@ -68,6 +68,7 @@ _SIGS = {
     "pa_paged_decode_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                       _c_int, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int),
                                       ctypes.POINTER(_c_int)]),
+    "pa_paged_decode_cascade_plan": (_c_int, [_c_int] * 12 + [ctypes.POINTER(_c_int)] * 5),
     "pa_reshape_and_cache_fp8": (_c_int, [_vp, _vp, _c_i64, _c_i64, _vp, _vp, _vp, _c_int, _c_int,
                                           _c_int, _c_int, _c_int, _c_int, ctypes.c_float,
                                           ctypes.c_float, _vp, _vp]),
@@ -301,6 +302,22 @@ def pa_paged_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_cont
                                       max_context_len, block_size, partition_tokens, int(ordered),
                                       ctypes.byref(pb), ctypes.byref(mp), ctypes.byref(nl)))
     return pb.value, mp.value, nl.value
+
+
+def pa_paged_decode_cascade_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                 max_blocks_per_seq, num_groups, group_size, max_prefix_blocks,
+                                 dtype="f16", fp8_cache=False, block_size=BLOCK_SIZE):
+    """The plan of a cascade call with these host bounds: a dict with the prefix's
+    blocks per partition and partitions, the own blocks' blocks per partition and
+    partitions, and the kernel launches."""
+    code = {"f16": PA_F16, "bf16": PA_BF16}[dtype]
+    out = [ctypes.c_int(0) for _ in range(5)]
+    _check(lib().pa_paged_decode_cascade_plan(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, max_blocks_per_seq,
+        block_size, num_groups, group_size, max_prefix_blocks, code, int(bool(fp8_cache)),
+        *[ctypes.byref(x) for x in out]))
+    keys = ("prefix_part_blocks", "prefix_parts", "own_part_blocks", "own_parts", "launches")
+    return dict(zip(keys, (x.value for x in out)))
 
 
 def decode_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,

@@ -738,6 +738,37 @@ int pa_paged_decode_cascade_workspace_size(int num_seqs, int num_q_heads, int nu
   return PA_OK;
 }
 
+int pa_paged_decode_cascade_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int max_context_len, int max_blocks_per_seq, int block_size,
+                                 int num_groups, int group_size, int max_prefix_blocks, int dtype,
+                                 int fp8_cache, int* prefix_part_blocks, int* prefix_parts,
+                                 int* own_part_blocks, int* own_parts, int* launches) {
+  clear_error();
+  if (!prefix_part_blocks || !prefix_parts || !own_part_blocks || !own_parts || !launches)
+    return fail(PA_ERR_INVALID_ARG, "null output pointer");
+  if (block_size != kBlockSize)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d: only %d is supported", block_size,
+                kBlockSize);
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "dtype %d: expected PA_F16 or PA_BF16", dtype);
+  CascadeLayout lay;
+  if (int st = cascade_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                              max_blocks_per_seq, num_groups, group_size, max_prefix_blocks, &lay))
+    return st;
+  const int gh = num_q_heads / num_kv_heads;
+  const bool single =
+      num_groups > 0 &&
+      cascade_single_launch(head_dim, gh, group_size * gh, dtype, fp8_cache ? PA_FP8_E4M3 : dtype);
+  *prefix_part_blocks = num_groups > 0 ? lay.g_part_blocks : 0;
+  *prefix_parts = num_groups > 0 ? lay.g_parts : 0;
+  *own_part_blocks = lay.s_part_blocks;
+  *own_parts = lay.s_parts;
+  // prepare, the decode(s), merge: the two decodes share a launch where the
+  // shapes allow, else the prefix decode runs on a second stream
+  *launches = num_seqs == 0 ? 0 : (num_groups > 0 && !single) ? 4 : 3;
+  return PA_OK;
+}
+
 int pa_paged_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, int max_blocks_per_seq,
                             const int32_t* context_lens, const int32_t* seq_order,

@@ -213,12 +213,14 @@ class DecodeRunner:
 
     def decode_launches(self) -> int:
         """Kernel launches of the step's decode call."""
+        wl = self.wl
         if self.groups is not None:
             # prepare, both decodes in one launch (8 stacked query heads per KV
             # head; else two launches), merge
-            g = self.wl.num_q_heads // self.wl.num_kv_heads
-            return 3 if g * self.groups.group_size == 8 and g < 8 else 4
-        wl = self.wl
+            return L.pa_paged_decode_cascade_plan(
+                wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.max_context_len,
+                self.max_blocks, self.groups.num_groups, self.groups.group_size,
+                self.groups.max_prefix_blocks, dtype=wl.dtype)["launches"]
         _, _, n = L.pa_paged_decode_plan(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
                                          wl.head_dim, wl.max_context_len,
                                          self.partition_tokens or 0, ordered=True)

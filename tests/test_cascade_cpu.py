@@ -221,3 +221,32 @@ def test_cascade_order_edge_cases():
     assert lib.pa_cascade_order(None, None, None, 0, 0, None) == L.PA_OK
     assert lib.pa_cascade_order(ctx.ctypes.data, None, None, 0, -1,
                                 out.ctypes.data) == L.PA_ERR_INVALID_ARG
+
+
+def test_cascade_plan():
+    """pa_paged_decode_cascade_plan: a group prefix stays one partition (up to the
+    decode's 128-block cap) when groups and sequences together give the GPU
+    enough (group or sequence, KV head) pairs, and is split into partitions of
+    at least 32 blocks when they do not; launches are 3 for the single-launch
+    shapes (8 stacked query heads) and for batches without groups, 4 when the
+    two decodes run on two streams, 0 for an empty batch."""
+    # 16 prompts forked 8 ways, 62-block prefixes, 32 KV heads: 4608 pairs
+    p = L.pa_paged_decode_cascade_plan(128, 32, 32, 128, 1200, 76, 16, 8, 62)
+    assert p == {"prefix_part_blocks": 62, "prefix_parts": 1, "own_part_blocks": 75,
+                 "own_parts": 1, "launches": 3}
+    assert L.pa_paged_decode_cascade_plan(128, 32, 32, 128, 1200, 76, 16, 8, 62, dtype="bf16",
+                                          fp8_cache=True)["launches"] == 3
+    # a prefix longer than the cap is split at the cap
+    p = L.pa_paged_decode_cascade_plan(128, 32, 32, 128, 6000, 376, 16, 8, 300)
+    assert (p["prefix_part_blocks"], p["prefix_parts"]) == (128, 3)
+    # 1 group of 2 and 2 KV heads: 6 pairs, so 1024 / 6 -> 171 parts wanted, floored at 32 blocks
+    p = L.pa_paged_decode_cascade_plan(2, 2, 2, 64, 4000, 250, 1, 2, 200)
+    assert (p["prefix_part_blocks"], p["prefix_parts"]) == (32, 7)
+    assert p["launches"] == 4          # 2 stacked heads: the two decodes on two streams
+    p = L.pa_paged_decode_cascade_plan(40, 16, 4, 128, 900, 60, 0, 2, 1)
+    assert (p["prefix_part_blocks"], p["prefix_parts"], p["launches"]) == (0, 0, 3)
+    assert L.pa_paged_decode_cascade_plan(0, 16, 4, 128, 0, 1, 0, 2, 1)["launches"] == 0
+    with pytest.raises(pa.PAError):    # 3 x 4 stacked heads per KV head
+        L.pa_paged_decode_cascade_plan(8, 16, 4, 128, 900, 60, 2, 3, 10)
+    with pytest.raises(pa.PAError):
+        L.pa_paged_decode_cascade_plan(8, 16, 4, 96, 900, 60, 2, 2, 10)
